@@ -1,0 +1,304 @@
+"""Seeded synthetic inputs for the IndexCache decode path.
+
+This module is the one place that draws random inputs. Both the float64
+oracle (under ``oracle/``) and the CUDA path read the tensors it returns, so
+both sides see identical bytes: values are drawn in fp32, rounded once to
+bf16 (round-to-nearest-even) or quantised once to fp8 e4m3, and never
+re-rounded afterwards.
+
+It holds none of the method's arithmetic (no indexer scores, no top-k, no
+attention). The only derived quantities are input-construction steps:
+
+* bf16 rounding (``torch.Tensor.to(torch.bfloat16)``, RNE);
+* per-token fp8 e4m3 quantisation of indexer keys with scale
+  ``max|k_s| / 448`` (the cache-append step that precedes the hot path);
+* planted keys: a key pointed along ``sum_h w_h q_h`` of its query, with a
+  fixed norm, so that the query prefers it (the "planted relevant tokens" of
+  the tiny and 1M-context workloads).
+
+Workload shapes follow the five configurations of the IndexCache decode study
+(Hy4 IndexCache explainer, "Where the saving actually lands": 78 layers and a
+1M-token context; porting issue on Hy4-preview, indexer bullet: 21 full layers
+of 78 starting F F F S S S; MLA shape RoPE-64, head 576, top-k 2048).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+D_LATENT = 512  # latent value width of an MLA row
+D_ROPE = 64     # rotary part of an MLA row
+D_QK = D_LATENT + D_ROPE  # 576: the head dim of the MLA query/key
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _randn(shape, g, device, scale=1.0) -> torch.Tensor:
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if scale != 1.0:
+        x.mul_(scale)
+    return x
+
+
+def _rand(shape, g, device, scale=1.0) -> torch.Tensor:
+    x = torch.rand(shape, generator=g, device=device, dtype=torch.float32)
+    if scale != 1.0:
+        x.mul_(scale)
+    return x
+
+
+def quantize_e4m3_rows(k: torch.Tensor):
+    """Per-token (last-dim row) fp8 e4m3 quantisation.
+
+    Returns ``(codes uint8 [..., d], scale fp32 [...])`` with
+    ``scale = max|k| / 448`` and ``codes = e4m3(k / scale)`` rounded to
+    nearest even by torch's cast. A row of zeros gets scale 0 and zero codes.
+    """
+    amax = k.abs().amax(dim=-1)
+    scale = (amax / 448.0).to(torch.float32)
+    safe = torch.where(scale > 0, scale, torch.ones_like(scale))
+    codes = (k / safe.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, scale
+
+
+def planted_direction(q: torch.Tensor, w: torch.Tensor) -> torch.Tensor:
+    """Unit vector along sum_h w_h q_h for each query: q [B,H,d], w [B,H] -> [B,d]."""
+    u = (w.float().unsqueeze(-1) * q.float()).sum(dim=1)
+    return u / u.norm(dim=-1, keepdim=True).clamp_min(1e-30)
+
+
+def schedule_from_f_positions(L: int, f_positions) -> str:
+    s = ["S"] * L
+    for p in f_positions:
+        s[int(p)] = "F"
+    return "".join(s)
+
+
+def hy4_schedule(L: int = 78, n_full: int = 21, seed: int = 2) -> str:
+    """The 78-layer F/S pattern: F at 0,1,2, S at 3,4,5, the remaining F
+    positions drawn without replacement from layers 6..L-1 with a seeded
+    ``numpy.random.default_rng``."""
+    rng = np.random.default_rng(seed)
+    rest = rng.choice(np.arange(6, L), n_full - 3, replace=False)
+    return schedule_from_f_positions(L, [0, 1, 2] + sorted(int(x) for x in rest))
+
+
+def every_nth_schedule(L: int, n: int) -> str:
+    """Refresh the index every n layers: F at 0, n, 2n, ..."""
+    return "".join("F" if l % n == 0 else "S" for l in range(L))
+
+
+@dataclasses.dataclass
+class Layer:
+    """One layer's inputs. Indexer fields are None on S layers."""
+    q_idx: Optional[torch.Tensor] = None    # [B,H_I,d_I] bf16
+    w: Optional[torch.Tensor] = None        # [B,H_I] fp32
+    k_idx: Optional[torch.Tensor] = None    # [Bk,N,d_I] bf16 or uint8 (e4m3 codes)
+    k_scale: Optional[torch.Tensor] = None  # [Bk,N] fp32 (fp8 keys only)
+    q: Optional[torch.Tensor] = None        # [B,H,576] bf16
+    kv: Optional[torch.Tensor] = None       # [Bkv,N,576] bf16
+    sink: Optional[torch.Tensor] = None     # [H] fp32
+    gate: Optional[torch.Tensor] = None     # [B,H,512] bf16 or None
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    B: int
+    N: int
+    H_I: int
+    d_I: int
+    topk: int
+    H: int
+    schedule: str
+    layers: List[Layer]
+    k_fp8: bool = False
+    shared_keys: bool = False     # one indexer key cache for all B queries
+    shared_kv: bool = False       # one latent KV cache for all B queries
+    n_valid: Optional[torch.Tensor] = None  # [B] int64, causal limit
+    planted: Optional[torch.Tensor] = None  # [B,P] int64 planted positions
+    sm_scale: float = 1.0 / math.sqrt(D_QK)
+    seed: int = 0
+
+    @property
+    def L(self) -> int:
+        return len(self.schedule)
+
+
+def _indexer_inputs(B, N, H_I, d_I, Bk, g, device, key_scale, w_scale):
+    q = _randn((B, H_I, d_I), g, device, 1.0 / math.sqrt(d_I)).to(torch.bfloat16)
+    w = _rand((B, H_I), g, device, w_scale)
+    k = _randn((Bk, N, d_I), g, device, key_scale)
+    return q, w, k
+
+
+def _plant(k_f32, q, w, positions, norm):
+    """Overwrite keys at ``positions`` [Bk,P] with norm * planted_direction."""
+    u = planted_direction(q, w)  # [B,d]
+    for b in range(positions.shape[0]):
+        k_f32[b, positions[b]] = (norm * u[b]).unsqueeze(0)
+    return k_f32
+
+
+def _attn_inputs(B, N, H, Bkv, g, device, gate: bool):
+    q = _randn((B, H, D_QK), g, device).to(torch.bfloat16)
+    kv = _randn((Bkv, N, D_QK), g, device).to(torch.bfloat16)
+    sink = _randn((H,), g, device, 0.5)
+    gt = _randn((B, H, D_LATENT), g, device).to(torch.bfloat16) if gate else None
+    return q, kv, sink, gt
+
+
+# Norm of a planted key, in units of a typical key's norm (sigma_k*sqrt(d_I)).
+# Two typical norms puts the planted score well past mean + 4 sigma of the
+# unplanted scores (checked against the oracle in the tests).
+PLANT_NORM = 2.0
+
+
+def tiny(device="cpu", seed: int = 0) -> Workload:
+    """4-layer stack F S S S, N=4096, B=1, H_I=4, d_I=64, k=256, H=8, 8 planted."""
+    B, N, H_I, d_I, H, K = 1, 4096, 4, 64, 8, 256
+    g = _gen(seed, device)
+    q_i, w, k = _indexer_inputs(B, N, H_I, d_I, B, g, device, 1.0 / math.sqrt(d_I), 0.25)
+    rng = np.random.default_rng(seed)
+    pos = torch.as_tensor(np.sort(rng.choice(N, 8, replace=False)), dtype=torch.int64).view(1, 8)
+    k = _plant(k, q_i, w, pos.to(device), PLANT_NORM).to(torch.bfloat16)
+    layers = []
+    for l in range(4):
+        q, kv, sink, _ = _attn_inputs(B, N, H, B, g, device, gate=False)
+        lay = Layer(q=q, kv=kv, sink=sink)
+        if l == 0:
+            lay.q_idx, lay.w, lay.k_idx = q_i, w, k
+        layers.append(lay)
+    return Workload("tiny_stack4_N4096", B, N, H_I, d_I, K, H, "FSSS", layers,
+                    planted=pos, seed=seed)
+
+
+def single_f(device="cpu", seed: int = 1, N: int = 131072, B: int = 8, H_I: int = 64,
+             d_I: int = 128, topk: int = 2048, H: int = 128, gate: bool = True,
+             shared: bool = False) -> Workload:
+    """One F layer at model shape: per-query caches (default) or one shared cache."""
+    g = _gen(seed, device)
+    Bk = 1 if shared else B
+    q_i, w, k = _indexer_inputs(B, N, H_I, d_I, Bk, g, device, 1.0 / math.sqrt(d_I), 1.0 / H_I)
+    q, kv, sink, gt = _attn_inputs(B, N, H, Bk, g, device, gate)
+    lay = Layer(q_idx=q_i, w=w, k_idx=k.to(torch.bfloat16), q=q, kv=kv, sink=sink, gate=gt)
+    return Workload(f"single_F_B{B}_N{N}", B, N, H_I, d_I, topk, H, "F", [lay],
+                    shared_keys=shared, shared_kv=shared, seed=seed)
+
+
+def stack(device="cpu", seed: int = 2, L: int = 78, n_full: int = 21, B: int = 32,
+          N: int = 131072, H_I: int = 64, d_I: int = 128, topk: int = 2048, H: int = 128,
+          rho: float = 0.8, schedule: Optional[str] = None, gate: bool = True) -> Workload:
+    """The 78-layer F/S decode stack: one key cache and one KV cache per layer,
+    shared by all B queries; keys independent per layer; indexer and attention
+    queries correlated across layers, q_l = rho q_{l-1} + sqrt(1-rho^2) eps_l."""
+    sched = schedule if schedule is not None else hy4_schedule(L, n_full, seed)
+    assert len(sched) == L
+    g = _gen(seed, device)
+    c = math.sqrt(1.0 - rho * rho)
+    qi_prev = q_prev = None
+    layers = []
+    for l in range(L):
+        eps_i = _randn((B, H_I, d_I), g, device, 1.0 / math.sqrt(d_I))
+        eps_q = _randn((B, H, D_QK), g, device)
+        qi_f = eps_i if qi_prev is None else rho * qi_prev + c * eps_i
+        q_f = eps_q if q_prev is None else rho * q_prev + c * eps_q
+        qi_prev, q_prev = qi_f, q_f
+        lay = Layer(q=q_f.to(torch.bfloat16))
+        lay.kv = _randn((1, N, D_QK), g, device).to(torch.bfloat16)
+        lay.sink = _randn((H,), g, device, 0.5)
+        lay.gate = _randn((B, H, D_LATENT), g, device).to(torch.bfloat16) if gate else None
+        if sched[l] == "F":
+            lay.q_idx = qi_f.to(torch.bfloat16)
+            lay.w = _rand((B, H_I), g, device, 1.0 / H_I)
+            lay.k_idx = _randn((1, N, d_I), g, device, 1.0 / math.sqrt(d_I)).to(torch.bfloat16)
+        layers.append(lay)
+    return Workload(f"stack{L}_B{B}_N{N}", B, N, H_I, d_I, topk, H, sched, layers,
+                    shared_keys=True, shared_kv=True, seed=seed)
+
+
+def long_context(device="cpu", seed: int = 3, N: int = 1048576, B: int = 4, H_I: int = 64,
+                 d_I: int = 128, topk: int = 2048, H: int = 128, fp8: bool = False,
+                 n_planted: int = 64) -> Workload:
+    """1M-context decode, per-query caches, planted tokens at evenly spaced
+    positions floor((i + 1/2) N / P); keys bf16 or fp8 e4m3 with per-token scale.
+    Both key variants come from the same fp32 draw."""
+    g = _gen(seed, device)
+    q_i, w, k = _indexer_inputs(B, N, H_I, d_I, B, g, device, 1.0 / math.sqrt(d_I), 1.0 / H_I)
+    pos = torch.tensor([int((i + 0.5) * N / n_planted) for i in range(n_planted)],
+                       dtype=torch.int64).repeat(B, 1)
+    k = _plant(k, q_i, w, pos.to(device), PLANT_NORM)
+    q, kv, sink, _ = _attn_inputs(B, N, H, B, g, device, gate=False)
+    lay = Layer(q_idx=q_i, w=w, q=q, kv=kv, sink=sink)
+    if fp8:
+        lay.k_idx, lay.k_scale = quantize_e4m3_rows(k)
+    else:
+        lay.k_idx = k.to(torch.bfloat16)
+    return Workload(f"long_ctx_B{B}_N{N}_{'fp8' if fp8 else 'bf16'}", B, N, H_I, d_I, topk, H, "F",
+                    [lay], k_fp8=fp8, planted=pos, seed=seed)
+
+
+def prefill(device="cpu", seed: int = 4, P: int = 262144, C: int = 2048, H_I: int = 64,
+            d_I: int = 128, topk: int = 2048, H: int = 128) -> Workload:
+    """Chunked prefill: C causal queries at positions P..P+C-1 over one shared
+    cache of P + C tokens; query i sees tokens 0..P+i."""
+    N = P + C
+    g = _gen(seed, device)
+    q_i, w, k = _indexer_inputs(C, N, H_I, d_I, 1, g, device, 1.0 / math.sqrt(d_I), 1.0 / H_I)
+    q, kv, sink, _ = _attn_inputs(C, N, H, 1, g, device, gate=False)
+    lay = Layer(q_idx=q_i, w=w, k_idx=k.to(torch.bfloat16), q=q, kv=kv, sink=sink)
+    n_valid = torch.arange(P + 1, P + C + 1, dtype=torch.int64, device=device)
+    return Workload(f"prefill_C{C}_P{P}", C, N, H_I, d_I, topk, H, "F", [lay],
+                    shared_keys=True, shared_kv=True, n_valid=n_valid, seed=seed)
+
+
+def indexer_case(B, N, H_I, d_I, shared=False, fp8=False, causal=False, seed=11, device="cpu"):
+    """A bare indexer input set (used by unit tests)."""
+    g = _gen(seed, device)
+    Bk = 1 if shared else B
+    q, w, k = _indexer_inputs(B, N, H_I, d_I, Bk, g, device, 1.0 / math.sqrt(d_I), 1.0 / H_I)
+    if fp8:
+        codes, scale = quantize_e4m3_rows(k)
+        kk, ks = codes, scale
+    else:
+        kk, ks = k.to(torch.bfloat16), None
+    n_valid = None
+    if causal:
+        n_valid = torch.randint(0, N + 1, (B,), generator=g, device=device, dtype=torch.int64)
+        n_valid[0] = N
+    return q, w, kk, ks, n_valid
+
+
+def scores_case(B, N, seed=12, ties=False, neg_inf_frac=0.0, device="cpu"):
+    """Random fp32 score rows for top-k tests; optional heavy ties and -inf."""
+    g = _gen(seed, device)
+    s = torch.randn((B, N), generator=g, device=device, dtype=torch.float32)
+    if ties:
+        s = torch.round(s * 4.0) / 4.0  # few distinct values, many exact ties
+    if neg_inf_frac > 0:
+        m = torch.rand((B, N), generator=g, device=device) < neg_inf_frac
+        s[m] = float("-inf")
+    return s
+
+
+def attention_case(B, N, H, k, shared=False, gate=True, n_invalid=0, seed=13, device="cpu"):
+    """Bare sparse-MLA inputs: q, kv, idx (distinct per row, -1 padding at the
+    end of each row when n_invalid > 0), sink, gate."""
+    g = _gen(seed, device)
+    Bkv = 1 if shared else B
+    q, kv, sink, gt = _attn_inputs(B, N, H, Bkv, g, device, gate)
+    idx = torch.empty((B, k), dtype=torch.int32, device=device)
+    for b in range(B):
+        perm = torch.randperm(N, generator=g, device=device)[:k]
+        idx[b] = perm.to(torch.int32)
+        if n_invalid:
+            idx[b, k - n_invalid:] = -1
+    return q, kv, idx, sink, gt
