@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Decode throughput of the 78-layer IndexCache F/S stack at 128K context.
+
+Workload (one replica per GPU): 78 layers, schedule F F F S S S ... with 21 F
+layers, 32 decode queries, 131072 cached tokens per layer, indexer 64 heads x
+128 dims (bf16 keys), top-k 2048, sparse MLA with 128 heads of 576 dims,
+per-head sink and sigmoid gate. Synthetic seeded inputs drawn on the device.
+
+A step is one pass of the whole hot path over the stack: on each F layer the
+lightning indexer and top-k, on every layer the sparse MLA attention over the
+shared index buffer. The metric is decode tokens/s = queries x steps / time.
+
+Prints ONE JSON line (rank 0). ``--impl reference`` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tokens/s per 78-layer F/S stack at 128K ctx; indexer GB/s vs HBM peak"
+UNIT = "tokens/s"
+
+L, N_FULL, B, N, H_I, D_I, TOPK, H = 78, 21, 32, 131072, 64, 128, 2048, 128
+D_QK, D_V = 576, 512
+WORKLOAD = "stack78_B32_N131072_topk2048"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples at 100 ms, for the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.rows = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self, begin: bool):
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = self.rows
+        if self.t0 is not None and self.t1 is not None:
+            inside = [r for t, r in rows if self.t0 - 0.15 <= t <= self.t1 + 0.15]
+            rows = inside if inside else [r for _, r in rows]
+        else:
+            rows = [r for _, r in rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if len(r) > 8 and num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if len(r) > 8 and num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = []
+        for i, n in enumerate(names):
+            if any(len(r) > 8 and r[5 + i].lower().startswith("active") for r in rows):
+                reasons.append(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+def cpu_sample_step(seed: int = 7):
+    """One bounded oracle sample of the workload: one query through one F
+    layer (indexer over all 131072 tokens + top-k) and one attention layer.
+    Returns (seconds_F, seconds_attention, threads)."""
+    import numpy as np
+    import torch
+    import oracle
+    from lightning_indexer_cross_b200 import workloads as W
+
+    g = torch.Generator().manual_seed(seed)
+    q_i = (torch.randn((1, H_I, D_I), generator=g) / math.sqrt(D_I)).to(torch.bfloat16)
+    w = torch.rand((1, H_I), generator=g) / H_I
+    k = (torch.randn((1, N, D_I), generator=g) / math.sqrt(D_I)).to(torch.bfloat16)
+    q = torch.randn((1, H, D_QK), generator=g).to(torch.bfloat16)
+    kv = torch.randn((1, N, D_QK), generator=g).to(torch.bfloat16)
+    sink = torch.randn((H,), generator=g) * 0.5
+    gate = torch.randn((1, H, D_V), generator=g).to(torch.bfloat16)
+    t0 = time.perf_counter()
+    sc = oracle.indexer_scores(q_i, w, k)
+    idx = oracle.topk_indices(sc, TOPK)
+    t1 = time.perf_counter()
+    oracle.sparse_mla(q, kv, idx, sink, gate, 1.0 / math.sqrt(D_QK))
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_tokens_per_s(tf, ta):
+    # per decoded token (one query): 21 F layers (indexer + top-k + attention)
+    # and 57 S layers (attention)
+    return 1.0 / (N_FULL * tf + L * ta)
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup_ref):
+        cpu_sample_step()
+    tf_all, ta_all = [], []
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        tf, ta = cpu_sample_step(seed=100 + s)
+        tf_all.append(tf)
+        ta_all.append(ta)
+    wall = time.perf_counter() - t0
+    tf, ta = sum(tf_all) / len(tf_all), sum(ta_all) / len(ta_all)
+    v = cpu_tokens_per_s(tf, ta)
+    sample = (f"1 query: indexer+top-k over N={N} on 1 F layer and sparse MLA on 1 layer per step, "
+              f"extrapolated to the 78-layer schedule (21 F + 78 attention)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * wall / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": L, "full_layers": N_FULL, "queries": B, "ctx": N,
+                   "topk": TOPK, "sample": "1 query per step"},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- native arm
+def distinct_rows(trace, sched):
+    import torch
+    tot = 0
+    for l in range(len(sched)):
+        u = torch.unique(trace[l][trace[l] >= 0])
+        tot += u.numel()
+    return tot
+
+
+def run_native(args):
+    import torch
+    from lightning_indexer_cross_b200 import _abi, ops
+    from lightning_indexer_cross_b200 import workloads as W
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hbm_gbs, tf_burst, tf_sust, peak_kind = peaks()
+
+    wl = W.stack(dev, seed=2 + rank, L=L, n_full=N_FULL, B=B, N=N, H_I=H_I, d_I=D_I, topk=TOPK, H=H)
+    st = ops.stack_from_workload(wl, trace=False)
+    torch.cuda.synchronize()
+
+    # one traced step to count distinct gathered rows (algorithmic attention bytes)
+    st_tr = ops.stack_from_workload(wl, trace=True)
+    st_tr.step()
+    torch.cuda.synchronize()
+    rows_distinct = distinct_rows(st_tr.trace, wl.schedule)
+    launches_per_step = st_tr.step()
+    torch.cuda.synchronize()
+    if st_tr.device_status() != 0:
+        raise RuntimeError("device status not OK after a traced step")
+    del st_tr
+
+    stream = torch.cuda.Stream(device=dev)
+    graph = None
+    if not args.no_graph:
+        st.step()  # first call sets kernel attributes before capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            st.step()
+        torch.cuda.synchronize()
+
+    def one_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            st.step()
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clk.mark(True)
+    e0.record(cur)
+    for _ in range(args.steps):
+        one_step()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    clk.mark(False)
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, world)
+    if st.device_status() != 0:
+        raise RuntimeError("device status not OK after the timed steps")
+    value = world * B * args.steps / (ms_max / 1000.0)
+
+    # ------------------------------------------------------------------ per-kernel timing
+    kern = time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst)
+    clk.stop()
+    clocks = clk.summary()
+
+    # ------------------------------------------------------------------ e2e (host buffers)
+    e2e = None if args.no_e2e else time_e2e(wl, st, args, dev, world)
+
+    # dominant kernel: largest total time per step
+    per_step = {
+        "indexer": kern["indexer"]["us"] * N_FULL,
+        "topk": kern["topk"]["us"] * N_FULL,
+        "sparse_mla": kern["sparse_mla"]["us"] * L,
+    }
+    dom = max(per_step, key=per_step.get)
+    roof = dict(kern[dom]["roofline"])
+    roof["kernel"] = dom
+    roof["traffic"] = load_traffic(dom)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": L, "full_layers": N_FULL, "schedule": wl.schedule,
+                   "queries": B, "global_batch": B * world, "ctx": N, "indexer_heads": H_I, "d_I": D_I,
+                   "topk": TOPK, "heads": H, "head_dim": D_QK, "parallelism": f"replicas{world}",
+                   "graph": graph is not None,
+                   "l2": "working set per step ~12.5 GB of KV/key caches > 126 MB L2; no flush needed"},
+        "roofline": roof,
+        "kernels": {k: {kk: vv for kk, vv in v.items()} for k, v in kern.items()},
+        "kernel_share_of_step": {k: v / sum(per_step.values()) for k, v in per_step.items()},
+        "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops": tf_burst, "kind": peak_kind},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, ta = cpu_sample_step()
+        tf, ta = cpu_sample_step(seed=8)
+        line["cpu_baseline"] = {
+            "value": cpu_tokens_per_s(tf, ta), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": "1 query: indexer+top-k over N=131072 on 1 F layer + sparse MLA on 1 layer, "
+                      "extrapolated to 21 F + 78 attention layers"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if one exists for
+    the current kernel build; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+        return d.get(kernel)
+    except Exception:
+        return None
+
+
+def _time_loop(fn, n, stream):
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1000.0 / n  # us
+
+
+def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
+    """Each kernel family alone, on the stream it is launched on, rotating over
+    the layers' own inputs (so each launch streams fresh data from HBM)."""
+    import torch
+    from lightning_indexer_cross_b200 import _abi, ops
+    stream = torch.cuda.current_stream()
+    f_layers = [l for l in range(wl.L) if wl.schedule[l] == "F"]
+    scores = torch.empty((B, N), dtype=torch.float32, device=dev)
+    ws_i = ops.new_workspace(_abi.ic_indexer_workspace_size(), dev)
+    ws_t = ops.new_workspace(_abi.ic_topk_workspace_size(B, N, TOPK), dev)
+    ws_m = ops.new_workspace(_abi.ic_sparse_mla_workspace_size(B, H, TOPK), dev)
+    idx = torch.empty((B, TOPK), dtype=torch.int32, device=dev)
+    out = torch.empty((B, H, D_V), dtype=torch.bfloat16, device=dev)
+    reps = max(3 * len(f_layers), min(args.steps, 200))
+
+    def ind(i):
+        lay = wl.layers[f_layers[i % len(f_layers)]]
+        ops.indexer_score(lay.q_idx, lay.w, lay.k_idx, None, None, scores=scores, workspace=ws_i)
+
+    def tk(i):
+        ops.topk(scores, TOPK, None, idx=idx, workspace=ws_t)
+
+    idx_by_layer = []
+    for l in f_layers:
+        ind_l = f_layers.index(l)
+        ind(ind_l)
+        tk(0)
+        idx_by_layer.append(idx.clone())
+
+    def mla(i):
+        l = i % wl.L
+        lay = wl.layers[l]
+        gi = [j for j in range(len(f_layers)) if f_layers[j] <= l][-1]
+        ops.sparse_mla_decode(lay.q, lay.kv, idx_by_layer[gi], lay.sink, lay.gate, out=out, want_lse=False,
+                              workspace=ws_m)
+
+    for fn in (ind, tk, mla):
+        for i in range(3):
+            fn(i)
+    torch.cuda.synchronize()
+    t_ind = _time_loop(ind, reps, stream)
+    # top-k reads scores written just before (as in the stack); time it alone
+    t_tk = _time_loop(tk, reps, stream)
+    t_mla = _time_loop(mla, max(reps, wl.L), stream)
+
+    # algorithmic work per launch
+    ind_bytes = N * D_I * 2 + B * H_I * D_I * 2 + B * H_I * 4 + B * N * 4
+    ind_flops = 2.0 * B * H_I * D_I * N
+    tk_bytes = B * N * 4 + B * TOPK * 4
+    mla_rows = rows_distinct / wl.L
+    mla_bytes = mla_rows * D_QK * 2 + B * H * D_QK * 2 + B * H * D_V * 2 * 2 + B * TOPK * 4
+    mla_flops = 2.0 * B * H * TOPK * (D_QK + D_V)
+
+    def roofline(bytes_, flops, us):
+        t_hbm = bytes_ / (hbm_gbs * 1e9)
+        t_tc = flops / (tf_burst * 1e12)
+        if t_tc > t_hbm:
+            ach = flops / (us * 1e-6) / 1e12
+            return {"bound": "tensor", "achieved": ach, "peak": tf_burst, "unit": "TFLOP/s",
+                    "frac": ach / tf_burst, "algorithmic_flops": flops, "algorithmic_bytes": bytes_}
+        ach = bytes_ / (us * 1e-6) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s", "frac": ach / hbm_gbs,
+                "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
+
+    return {
+        "indexer": {"us": t_ind, "launches": reps, "gbs": ind_bytes / (t_ind * 1e-6) / 1e9,
+                    "roofline": roofline(ind_bytes, ind_flops, t_ind)},
+        "topk": {"us": t_tk, "launches": reps, "elems_per_s": B * N / (t_tk * 1e-6),
+                 "roofline": roofline(tk_bytes, 0.0, t_tk)},
+        "sparse_mla": {"us": t_mla, "launches": max(reps, wl.L), "gbs": mla_bytes / (t_mla * 1e-6) / 1e9,
+                       "distinct_rows_per_layer": mla_rows,
+                       "roofline": roofline(mla_bytes, mla_flops, t_mla)},
+    }
+
+
+def time_e2e(wl, st, args, dev, world):
+    """Same metric through the public call with host buffers: per step, the
+    per-layer queries (indexer q and weights on F layers, attention q and gate
+    on every layer) are copied from pinned host memory, the stack runs, and the
+    last layer's attention output is read back to the host."""
+    import torch
+    ins_dev, ins_host = [], []
+    for l, lay in enumerate(wl.layers):
+        for t in (lay.q_idx, lay.w, lay.q, lay.gate):
+            if t is not None:
+                ins_dev.append(t)
+                ins_host.append(t.detach().cpu().pin_memory())
+    out_host = torch.empty(st.outs[-1].shape, dtype=st.outs[-1].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in ins_host)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for d, h in zip(ins_dev, ins_host):
+            d.copy_(h, non_blocking=True)
+        st.step()
+        out_host.copy_(st.outs[-1], non_blocking=True)
+
+    n = max(3, min(args.steps, 20))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    cur = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(n):
+        step()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"value": world * B * n / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--warmup-ref", type=int, default=1)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,198 @@
+/*
+ * indexcache.h -- C ABI of the B200 (sm_100a) IndexCache decode hot path.
+ *
+ * The path (Hy4 IndexCache explainer, "What is IndexCache" and narrative on
+ * the ticket rail; Hy4-preview porting issue, "Indexer", sink and gate
+ * bullets):
+ *
+ *   F layer:  scores = lightning indexer over every cached token
+ *             index  = top-k(scores)            -> shared index buffer
+ *   S layer:  index  = the buffer as the last preceding F layer left it
+ *   every layer: out = sparse MLA attention over the indexed rows, with a
+ *             per-head softmax sink and a sigmoid output gate.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, owned by the caller. The
+ *     library never allocates or frees device memory, never synchronises the
+ *     stream it is given (except ic_last_device_status, which says so), and
+ *     launches only on that stream.
+ *   - Tensors are dense row-major with the shapes stated; every pointer must
+ *     be 16-byte aligned.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is launched. A failed launch returns IC_ERR_CUDA. Errors found on the
+ *     device (an index outside [-1, N), a bounded wait that gave up) are
+ *     recorded in a status word at the start of the caller's workspace; read
+ *     it with ic_last_device_status.
+ *   - Workspaces: size them with the matching *_workspace_size call and
+ *     zero a new one once before its first use (the status word must start
+ *     at IC_OK). The status word keeps the first device error until
+ *     ic_last_device_status reads and clears it; every other byte is
+ *     scratch that each call initialises itself. Calls that share a
+ *     workspace must not overlap in time on the device.
+ */
+#ifndef INDEXCACHE_H_
+#define INDEXCACHE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* ic_stream_t; /* same object as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  IC_OK = 0,
+  IC_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or schedule */
+  IC_ERR_UNSUPPORTED = 2,  /* a valid shape this build has no kernel for */
+  IC_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  IC_ERR_TIMEOUT = 4,      /* device: a bounded wait inside a kernel gave up */
+  IC_ERR_BAD_INDEX = 5     /* device: an index outside [-1, N) was read (it was treated as -1) */
+} ic_status_t;
+
+typedef enum { IC_BF16 = 0, IC_FP8_E4M3 = 1, IC_F32 = 2 } ic_dtype_t;
+
+/* Human-readable name of a status code (static storage). */
+const char* ic_status_string(ic_status_t s);
+
+/* ---------------------------------------------------------------------------
+ * ic_indexer_score -- the lightning indexer.
+ *
+ * Defines (Hy4 IndexCache explainer, Jargon "Indexer": a cheap pass that
+ * scores every cached position; the score form is DeepSeek's lightning
+ * indexer):
+ *     scores[b, s] = sum_h w[b,h] * max(0, sum_d q[b,h,d] * k_b[s,d])
+ * for s < n_valid[b]; scores[b, s] = -inf for n_valid[b] <= s < N.
+ *
+ *   q        [B, H_I, d_I] bf16.
+ *   w        [B, H_I] fp32 head weights of each query.
+ *   k        key cache of query b at k + b*k_batch_stride elements, [N, d_I],
+ *            bf16 (k_dtype IC_BF16) or e4m3 codes (IC_FP8_E4M3).
+ *            k_batch_stride = 0: one cache shared by all B queries.
+ *   k_scale  fp32 per-token scale, e4m3 keys only (NULL otherwise): the key
+ *            of token s is decode(code[s,:]) * k_scale[s]; query b's scales
+ *            at k_scale + b*scale_batch_stride. Scales must be >= 0.
+ *   n_valid  int64 [B] causal limits (device), or NULL: every s < N valid.
+ *   scores   [B, N] fp32 output, row stride N.
+ *   Supported: d_I in {64, 128}; 1 <= H_I <= 128; N >= 1; B >= 1.
+ *   workspace >= ic_indexer_workspace_size() bytes (holds the status word).
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_indexer_score(const void* q, const float* w, const void* k, const float* k_scale,
+                             ic_dtype_t k_dtype, int B, int H_I, int d_I, int64_t N,
+                             int64_t k_batch_stride, int64_t scale_batch_stride,
+                             const int64_t* n_valid, float* scores, void* workspace,
+                             size_t ws_bytes, ic_stream_t stream);
+size_t ic_indexer_workspace_size(void);
+
+/* ---------------------------------------------------------------------------
+ * ic_topk -- top-k selection (Hy4 IndexCache explainer, Jargon "Top-k
+ * selection"; k = 2048 at model shape per the Hy4-preview porting issue).
+ *
+ * For each row b, writes to idx[b, :] the token indices of the k largest
+ * scores[b, s] over s < n_valid[b] (all N when n_valid is NULL). Ties at the
+ * k-th value are resolved toward the lower index. The order of the indices
+ * within a row is unspecified. When fewer than k positions compete, they
+ * are all written and the row is padded with -1.
+ *   scores [B, N] fp32 (row stride N); idx [B, k] int32.
+ *   Supported: 1 <= k <= 16384, N < 2^31.
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_valid, int k,
+                    int32_t* idx, void* workspace, size_t ws_bytes, ic_stream_t stream);
+size_t ic_topk_workspace_size(int B, int64_t N, int k);
+
+/* ---------------------------------------------------------------------------
+ * ic_sparse_mla_decode -- DSA token-level sparse attention, MLA shape,
+ * with a per-head sink and a sigmoid output gate (Hy4 IndexCache explainer,
+ * Jargon "DSA"; Hy4-preview porting issue: head 576 = 512 latent + 64 RoPE,
+ * "learnable per-head sink (softmax-denominator bias)", "elementwise sigmoid
+ * gate").
+ *
+ * For query b, head h, selected tokens j (idx[b,j] in [0, N)):
+ *     z_j = sm_scale * sum_{d<576} q[b,h,d] * kv_b[idx_j, d]
+ *     o   = sum_j exp(z_j) kv_b[idx_j, 0:512] / (exp(sink[h]) + sum_j exp(z_j))
+ *     out[b,h,:] = sigmoid(gate[b,h,:]) * o     (gate NULL: out = o)
+ *     lse[b,h]   = log(exp(sink[h]) + sum_j exp(z_j))   (if lse != NULL)
+ * Entries equal to -1 are skipped.
+ *
+ *   q     [B, H, 576] bf16 (RoPE already applied to dims 512..575).
+ *   kv    latent cache of query b at kv + b*kv_batch_stride elements,
+ *         [N, 576] bf16; kv_batch_stride = 0: one cache shared by all.
+ *   idx   [B, k] int32.   sink [H] fp32.   gate [B, H, 512] bf16 or NULL.
+ *   out   [B, H, 512], bf16 (out_dtype IC_BF16) or fp32 (IC_F32).
+ *   lse   [B, H] fp32 natural-log sum, or NULL.
+ *   Supported: any H >= 1 (heads run in blocks of 128); k >= 1;
+ *   sm_scale > 0 and finite.
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_sparse_mla_decode(const void* q, const void* kv, int64_t kv_batch_stride, int64_t N,
+                                 const int32_t* idx, int k, const float* sink, const void* gate,
+                                 float sm_scale, int B, int H, ic_dtype_t out_dtype, void* out,
+                                 float* lse, void* workspace, size_t ws_bytes, ic_stream_t stream);
+size_t ic_sparse_mla_workspace_size(int B, int H, int k);
+
+/* ---------------------------------------------------------------------------
+ * ic_layer_stack -- the IndexCache decode step over L layers.
+ *
+ * Layer l with schedule[l] == 'F' runs ic_indexer_score and ic_topk and
+ * overwrites index_buf; with 'S' it leaves index_buf as the last preceding
+ * F layer wrote it (Hy4-preview porting issue, "Indexer" bullet: shared
+ * layers reuse the last preceding full layer's top-k). Every layer then runs
+ * ic_sparse_mla_decode reading index_buf in place. schedule[0] must be 'F'.
+ *
+ *   layers     [L] host array of per-layer device pointers (ic_layer_t).
+ *              On S layers q_idx, w, k_idx and k_scale are ignored.
+ *   schedule   host string of L characters from {'F','S'}.
+ *   shape      host struct of sizes shared by every layer.
+ *   index_buf  [B, topk] int32 device buffer, owned by the caller.
+ *   idx_trace  optional [L, B, topk] int32 device buffer: if not NULL, the
+ *              index buffer each layer attended over is copied there.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int B;                       /* queries */
+  int64_t N;                   /* cached tokens */
+  int H_I, d_I;                /* indexer heads and dim */
+  ic_dtype_t k_dtype;          /* IC_BF16 or IC_FP8_E4M3 */
+  int topk;                    /* k */
+  int H;                       /* attention heads */
+  float sm_scale;              /* softmax scale of the 576-d logits */
+  ic_dtype_t out_dtype;        /* IC_BF16 or IC_F32 */
+  int64_t k_batch_stride;      /* elements between queries' key caches (0 = shared) */
+  int64_t scale_batch_stride;  /* elements between queries' key scales (0 = shared) */
+  int64_t kv_batch_stride;     /* elements between queries' latent caches (0 = shared) */
+  const int64_t* n_valid;      /* device [B] causal limits, or NULL */
+} ic_stack_shape_t;
+
+typedef struct {
+  const void* q_idx;     /* [B, H_I, d_I] bf16 (F layers) */
+  const float* w;        /* [B, H_I] fp32 (F layers) */
+  const void* k_idx;     /* indexer key cache (F layers) */
+  const float* k_scale;  /* e4m3 key scales or NULL (F layers) */
+  const void* q;         /* [B, H, 576] bf16 */
+  const void* kv;        /* latent cache */
+  const float* sink;     /* [H] fp32 */
+  const void* gate;      /* [B, H, 512] bf16 or NULL */
+  void* out;             /* [B, H, 512] out_dtype */
+  float* lse;            /* [B, H] fp32 or NULL */
+} ic_layer_t;
+
+ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule,
+                           const ic_stack_shape_t* shape, int32_t* index_buf, int32_t* idx_trace,
+                           void* workspace, size_t ws_bytes, ic_stream_t stream);
+size_t ic_layer_stack_workspace_size(const ic_stack_shape_t* shape);
+
+/* ---------------------------------------------------------------------------
+ * ic_last_device_status -- synchronises `stream`, then reads and clears the
+ * device status word at the start of `workspace` (any of the workspaces
+ * above). Returns IC_OK, IC_ERR_TIMEOUT or IC_ERR_BAD_INDEX (or IC_ERR_CUDA
+ * if the synchronisation itself failed).
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_last_device_status(void* workspace, ic_stream_t stream);
+
+/* Number of kernels the last successful call on this host thread enqueued
+ * (for launch accounting in benchmarks). */
+int ic_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* INDEXCACHE_H_ */

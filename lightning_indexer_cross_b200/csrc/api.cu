@@ -1,0 +1,392 @@
+// C ABI of the IndexCache hot path: argument validation (on the host, before
+// any launch), workspace layouts, TMA descriptor encoding, and the F/S layer
+// stack driver (Hy4-preview porting issue, "Indexer" bullet: shared layers
+// reuse the last preceding full layer's top-k).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/indexcache.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local int g_launches = 0;
+
+constexpr size_t kStatusBytes = 256;  // status word + padding (keeps regions aligned)
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+template <typename T>
+inline T ceil_div(T a, T b) { return (a + b - 1) / b; }
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// ------------------------------------------------------------------ indexer
+int indexer_hp(int H_I) {
+  int hp = ((H_I + 15) / 16) * 16;
+  if (hp <= 16) return 16;
+  if (hp <= 32) return 32;
+  if (hp <= 64) return 64;
+  return 128;
+}
+
+ic_status_t indexer_impl(const void* q, const float* w, const void* k, const float* k_scale, ic_dtype_t k_dtype,
+                         int B, int H_I, int d_I, int64_t N, int64_t k_batch_stride, int64_t scale_batch_stride,
+                         const int64_t* n_valid, float* scores, int* status, cudaStream_t stream) {
+  if (!q || !w || !k || !scores) return IC_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H_I < 1 || N >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  if (k_dtype != IC_BF16 && k_dtype != IC_FP8_E4M3) return IC_ERR_UNSUPPORTED;
+  if (d_I != 64 && d_I != 128) return IC_ERR_UNSUPPORTED;
+  if (H_I > 128) return IC_ERR_UNSUPPORTED;
+  const bool fp8 = k_dtype == IC_FP8_E4M3;
+  if (fp8 && !k_scale) return IC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(w) || !aligned16(scores) || (k_scale && !aligned16(k_scale)))
+    return IC_ERR_INVALID_ARG;
+  if (k_batch_stride < 0 || scale_batch_stride < 0) return IC_ERR_INVALID_ARG;
+  const int esz = fp8 ? 1 : 2;
+  const bool per_query = k_batch_stride != 0 && B > 1;
+  if (per_query && ((k_batch_stride * esz) % 16 != 0 || k_batch_stride < N * d_I)) return IC_ERR_INVALID_ARG;
+  if (fp8 && per_query && scale_batch_stride < N) return IC_ERR_INVALID_ARG;
+
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return IC_ERR_CUDA;
+  CUtensorMap map;
+  const cuuint64_t bk = per_query ? static_cast<cuuint64_t>(B) : 1;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d_I), static_cast<cuuint64_t>(N), bk};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d_I) * esz,
+                                 static_cast<cuuint64_t>(per_query ? k_batch_stride : N * d_I) * esz};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(fp8 ? d_I : 64), 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
+
+  ic::IndexerArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.w = w;
+  a.k_scale = k_scale;
+  a.scale_batch_stride = per_query ? scale_batch_stride : 0;
+  a.n_valid = n_valid;
+  a.scores = scores;
+  a.status = status;
+  a.B = B;
+  a.H_I = H_I;
+  a.N = N;
+  const int HP = indexer_hp(H_I);
+  a.G = per_query ? 1 : std::min(256 / HP, B);
+  a.tiles = static_cast<int>(ceil_div<int64_t>(N, 128));
+  const int64_t groups = ceil_div<int64_t>(B, a.G);
+  a.total_items = groups * a.tiles;
+  a.per_query = per_query ? 1 : 0;
+  const int grid = static_cast<int>(std::min<int64_t>(num_sms(), a.total_items));
+  cudaError_t e = ic::launch_indexer(map, a, HP, d_I, fp8, grid, stream);
+  if (e != cudaSuccess) return IC_ERR_CUDA;
+  g_launches += 1;
+  return IC_OK;
+}
+
+// ------------------------------------------------------------------ top-k
+struct TopkLayout {
+  int cpr;
+  int64_t slice;
+  size_t hist_off, tie_off, cnt_off, total;
+};
+
+TopkLayout topk_layout(int B, int64_t N) {
+  TopkLayout L{};
+  const int64_t target = std::max<int64_t>(1, 592 / std::max(B, 1));
+  int64_t cpr = std::min<int64_t>(ceil_div<int64_t>(N, 4096), target);
+  cpr = std::max<int64_t>(cpr, 1);
+  int64_t slice = ceil_div<int64_t>(N, cpr);
+  slice = ceil_div<int64_t>(slice, 4) * 4;
+  cpr = ceil_div<int64_t>(N, slice);
+  L.cpr = static_cast<int>(cpr);
+  L.slice = slice;
+  L.hist_off = 0;
+  L.tie_off = align256(L.hist_off + size_t(3) * B * 2048 * 4);
+  L.cnt_off = align256(L.tie_off + size_t(B) * L.cpr * 4);
+  L.total = align256(L.cnt_off + size_t(B) * 2 * 4);
+  return L;
+}
+
+ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_valid, int k, int32_t* idx,
+                      uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream) {
+  if (!scores || !idx || !ws) return IC_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || N >= (int64_t(1) << 31) || k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
+  if (!aligned16(scores) || !aligned16(idx)) return IC_ERR_INVALID_ARG;
+  TopkLayout L = topk_layout(B, N);
+  if (ws_bytes < L.total) return IC_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(ws, 0, L.total, stream) != cudaSuccess) return IC_ERR_CUDA;
+  ic::TopkArgs a{};
+  a.scores = scores;
+  a.n_valid = n_valid;
+  a.idx = idx;
+  a.hist = reinterpret_cast<uint32_t*>(ws + L.hist_off);
+  a.tie_counts = reinterpret_cast<uint32_t*>(ws + L.tie_off);
+  a.counters = reinterpret_cast<uint32_t*>(ws + L.cnt_off);
+  a.status = status;
+  a.B = B;
+  a.N = N;
+  a.k = k;
+  a.cpr = L.cpr;
+  a.slice = L.slice;
+  int launches = 0;
+  cudaError_t e = ic::launch_topk(a, stream, &launches);
+  if (e != cudaSuccess) return IC_ERR_CUDA;
+  g_launches += launches + 1;  // + the memset
+  return IC_OK;
+}
+
+// ------------------------------------------------------------------ sparse MLA
+int mla_ts(int B, int H, int k) {
+  const int hb = (H + 127) / 128;
+  const int sms = num_sms();
+  for (int ts : {256, 128}) {
+    const int64_t ctas = ceil_div<int64_t>(k, ts) * B * hb;
+    if (ctas * 5 >= static_cast<int64_t>(sms) * 4) return ts;
+  }
+  return 64;
+}
+
+struct MlaLayout {
+  int ts, splits;
+  size_t o_off, ml_off, total;
+};
+
+MlaLayout mla_layout(int B, int H, int k) {
+  MlaLayout L{};
+  L.ts = mla_ts(B, H, k);
+  L.splits = ceil_div(k, L.ts);
+  L.o_off = 0;
+  L.ml_off = align256(L.o_off + size_t(B) * H * L.splits * 512 * 4);
+  L.total = align256(L.ml_off + size_t(B) * H * L.splits * 2 * 4);
+  return L;
+}
+
+ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int64_t N, const int32_t* idx, int k,
+                     const float* sink, const void* gate, float sm_scale, int B, int H, ic_dtype_t out_dtype,
+                     void* out, float* lse, uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream) {
+  if (!q || !kv || !idx || !sink || !out || !ws) return IC_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || k < 1 || N < 1 || N >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || sm_scale == INFINITY) return IC_ERR_INVALID_ARG;
+  if (out_dtype != IC_BF16 && out_dtype != IC_F32) return IC_ERR_UNSUPPORTED;
+  if (kv_batch_stride < 0 || (kv_batch_stride != 0 && kv_batch_stride < N * 576)) return IC_ERR_INVALID_ARG;
+  if ((kv_batch_stride * 2) % 16 != 0) return IC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) || (gate && !aligned16(gate)))
+    return IC_ERR_INVALID_ARG;
+  MlaLayout L = mla_layout(B, H, k);
+  if (ws_bytes < L.total) return IC_ERR_INVALID_ARG;
+  ic::MlaArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.kv = static_cast<const __nv_bfloat16*>(kv);
+  a.kv_batch_stride = B > 1 ? kv_batch_stride : 0;
+  a.N = N;
+  a.idx = idx;
+  a.k = k;
+  a.sink = sink;
+  a.gate = static_cast<const __nv_bfloat16*>(gate);
+  a.sm_scale = sm_scale;
+  a.B = B;
+  a.H = H;
+  a.splits = L.splits;
+  a.ts = L.ts;
+  a.part_o = reinterpret_cast<float*>(ws + L.o_off);
+  a.part_ml = reinterpret_cast<float*>(ws + L.ml_off);
+  a.out = out;
+  a.out_f32 = out_dtype == IC_F32 ? 1 : 0;
+  a.lse = lse;
+  a.status = status;
+  int launches = 0;
+  cudaError_t e = ic::launch_sparse_mla(a, stream, &launches);
+  if (e != cudaSuccess) return IC_ERR_CUDA;
+  g_launches += launches;
+  return IC_OK;
+}
+
+// ------------------------------------------------------------------ stack
+struct StackLayout {
+  size_t scores_off, topk_off, mla_off, total;
+  TopkLayout tk;
+  MlaLayout ml;
+};
+
+StackLayout stack_layout(const ic_stack_shape_t& s) {
+  StackLayout L{};
+  L.tk = topk_layout(s.B, s.N);
+  L.ml = mla_layout(s.B, s.H, s.topk);
+  L.scores_off = kStatusBytes;
+  L.topk_off = align256(L.scores_off + size_t(s.B) * s.N * 4);
+  L.mla_off = align256(L.topk_off + L.tk.total);
+  L.total = align256(L.mla_off + L.ml.total);
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ic_status_string(ic_status_t s) {
+  switch (s) {
+    case IC_OK: return "IC_OK";
+    case IC_ERR_INVALID_ARG: return "IC_ERR_INVALID_ARG: bad pointer, size, alignment or schedule";
+    case IC_ERR_UNSUPPORTED: return "IC_ERR_UNSUPPORTED: valid shape with no kernel in this build";
+    case IC_ERR_CUDA: return "IC_ERR_CUDA: a CUDA call or launch failed";
+    case IC_ERR_TIMEOUT: return "IC_ERR_TIMEOUT: a bounded wait inside a kernel gave up";
+    case IC_ERR_BAD_INDEX: return "IC_ERR_BAD_INDEX: an index outside [-1, N) was read";
+  }
+  return "unknown ic_status_t";
+}
+
+int ic_last_launch_count(void) { return g_launches; }
+
+size_t ic_indexer_workspace_size(void) { return kStatusBytes; }
+
+ic_status_t ic_indexer_score(const void* q, const float* w, const void* k, const float* k_scale, ic_dtype_t k_dtype,
+                             int B, int H_I, int d_I, int64_t N, int64_t k_batch_stride, int64_t scale_batch_stride,
+                             const int64_t* n_valid, float* scores, void* workspace, size_t ws_bytes,
+                             ic_stream_t stream) {
+  g_launches = 0;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
+  return indexer_impl(q, w, k, k_scale, k_dtype, B, H_I, d_I, N, k_batch_stride, scale_batch_stride, n_valid,
+                      scores, static_cast<int*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ic_topk_workspace_size(int B, int64_t N, int k) {
+  (void)k;
+  if (B < 1 || N < 1) return kStatusBytes;
+  return kStatusBytes + topk_layout(B, N).total;
+}
+
+ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_valid, int k, int32_t* idx,
+                    void* workspace, size_t ws_bytes, ic_stream_t stream) {
+  g_launches = 0;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return topk_impl(scores, B, N, n_valid, k, idx, ws + kStatusBytes, ws_bytes - kStatusBytes,
+                   reinterpret_cast<int*>(ws), reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ic_sparse_mla_workspace_size(int B, int H, int k) {
+  if (B < 1 || H < 1 || k < 1) return kStatusBytes;
+  return kStatusBytes + mla_layout(B, H, k).total;
+}
+
+ic_status_t ic_sparse_mla_decode(const void* q, const void* kv, int64_t kv_batch_stride, int64_t N,
+                                 const int32_t* idx, int k, const float* sink, const void* gate, float sm_scale,
+                                 int B, int H, ic_dtype_t out_dtype, void* out, float* lse, void* workspace,
+                                 size_t ws_bytes, ic_stream_t stream) {
+  g_launches = 0;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  return mla_impl(q, kv, kv_batch_stride, N, idx, k, sink, gate, sm_scale, B, H, out_dtype, out, lse,
+                  ws + kStatusBytes, ws_bytes - kStatusBytes, reinterpret_cast<int*>(ws),
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ic_layer_stack_workspace_size(const ic_stack_shape_t* shape) {
+  if (!shape || shape->B < 1 || shape->N < 1 || shape->H < 1 || shape->topk < 1) return kStatusBytes;
+  return stack_layout(*shape).total;
+}
+
+ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule, const ic_stack_shape_t* shape,
+                           int32_t* index_buf, int32_t* idx_trace, void* workspace, size_t ws_bytes,
+                           ic_stream_t stream) {
+  g_launches = 0;
+  if (!layers || !schedule || !shape || !index_buf || !workspace || L < 1) return IC_ERR_INVALID_ARG;
+  if (!aligned16(workspace) || !aligned16(index_buf) || (idx_trace && !aligned16(idx_trace)))
+    return IC_ERR_INVALID_ARG;
+  const ic_stack_shape_t& s = *shape;
+  if (s.B < 1 || s.N < 1 || s.topk < 1 || s.H < 1) return IC_ERR_INVALID_ARG;
+  // schedule: exactly L characters from {F, S}, starting with F
+  for (int l = 0; l < L; ++l)
+    if (schedule[l] != 'F' && schedule[l] != 'S') return IC_ERR_INVALID_ARG;
+  if (schedule[L] != '\0' || schedule[0] != 'F') return IC_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l) {
+    const ic_layer_t& y = layers[l];
+    if (!y.q || !y.kv || !y.sink || !y.out) return IC_ERR_INVALID_ARG;
+    if (schedule[l] == 'F' && (!y.q_idx || !y.w || !y.k_idx)) return IC_ERR_INVALID_ARG;
+    if (schedule[l] == 'F' && s.k_dtype == IC_FP8_E4M3 && !y.k_scale) return IC_ERR_INVALID_ARG;
+  }
+  StackLayout SL = stack_layout(s);
+  if (ws_bytes < SL.total) return IC_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  float* scores = reinterpret_cast<float*>(ws + SL.scores_off);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int total = 0;
+  for (int l = 0; l < L; ++l) {
+    const ic_layer_t& y = layers[l];
+    if (schedule[l] == 'F') {
+      g_launches = 0;
+      ic_status_t r = indexer_impl(y.q_idx, y.w, y.k_idx, y.k_scale, s.k_dtype, s.B, s.H_I, s.d_I, s.N,
+                                   s.k_batch_stride, s.scale_batch_stride, s.n_valid, scores, status, st);
+      if (r != IC_OK) return r;
+      total += g_launches;
+      g_launches = 0;
+      r = topk_impl(scores, s.B, s.N, s.n_valid, s.topk, index_buf, ws + SL.topk_off, SL.tk.total, status, st);
+      if (r != IC_OK) return r;
+      total += g_launches;
+    }
+    g_launches = 0;
+    ic_status_t r = mla_impl(y.q, y.kv, s.kv_batch_stride, s.N, index_buf, s.topk, y.sink, y.gate, s.sm_scale,
+                             s.B, s.H, s.out_dtype, y.out, y.lse, ws + SL.mla_off, SL.ml.total, status, st);
+    if (r != IC_OK) return r;
+    total += g_launches;
+    if (idx_trace) {
+      const size_t n = size_t(s.B) * s.topk;
+      if (cudaMemcpyAsync(idx_trace + size_t(l) * n, index_buf, n * 4, cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess)
+        return IC_ERR_CUDA;
+    }
+  }
+  g_launches = total;
+  return IC_OK;
+}
+
+ic_status_t ic_last_device_status(void* workspace, ic_stream_t stream) {
+  if (!workspace) return IC_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return IC_ERR_CUDA;
+  if (v != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return IC_ERR_CUDA;
+  if (v == IC_ERR_TIMEOUT || v == IC_ERR_BAD_INDEX) return static_cast<ic_status_t>(v);
+  return v == 0 ? IC_OK : IC_ERR_CUDA;
+}
+
+}  // extern "C"

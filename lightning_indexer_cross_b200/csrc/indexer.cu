@@ -1,0 +1,361 @@
+// Lightning indexer on sm_100a tensor cores.
+//
+//   score[b, s] = sum_h w[b,h] * max(0, q[b,h,:] . k_b[s,:])
+//
+// (Hy4 IndexCache explainer, Jargon "Indexer": the cheap pass that scores
+// every cached position; DeepSeek lightning-indexer form.)
+//
+// Mapping. One tcgen05.mma per 16-wide slice of d_I computes a tile
+//   D[128 keys x n] = K_tile[128 x d_I] . Qg[n x d_I]^T,    n = G * HP
+// where Qg stacks the (padded) heads of G queries that read the same key
+// tile. Keys are the M side, so each TMEM lane holds one key's n head logits
+// and the epilogue thread owning that lane does ReLU, the w_h weighting and
+// the head sum in registers -- no cross-thread reduction. With one cache per
+// query G = 1 (n = HP, the decode case); with one cache shared by many
+// queries G = 256 / HP (prefill chunks, the layer stack), so each key byte
+// feeds up to 256 head columns.
+//
+// Warp roles (one CTA per SM, persistent over a contiguous range of
+// (query group, key tile) work items):
+//   warp 0      TMA producer: 128-key tiles of the key cache into a ring of
+//               shared-memory stages (128-byte swizzle, K-major).
+//   warp 1      TMEM owner and MMA issuer (one elected lane).
+//   warps 2..5  epilogue: TMEM -> registers -> score row; also stage the
+//               query group's Q (swizzled, zero-padded heads) and weights.
+//   warps 6..9  (e4m3 keys only) convert e4m3 tiles to bf16 in shared memory.
+//               tcgen05 kind::f16 needs both operands bf16, and the e4m3 ->
+//               bf16 widening is exact; the per-token scale is applied to the
+//               head sum, since ReLU(c x) = c ReLU(x) for c >= 0.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ic {
+
+namespace {
+
+constexpr int kTileKeys = 128;
+constexpr int kMaxCols = 256;  // MMA N limit for M = 128
+constexpr int kEpiWarp0 = 2;
+constexpr int kNumEpiThreads = 128;
+
+template <int D_I, bool FP8>
+struct IdxCfg {
+  static constexpr int kBlocks = D_I / 64;                        // 64-element (128 B) swizzle blocks
+  static constexpr int kTileBytes = kTileKeys * D_I * 2;          // bf16 tile
+  static constexpr int kRawBytes = FP8 ? kTileKeys * D_I : 0;     // e4m3 tile
+  static constexpr int kStages = FP8 ? 2 : (D_I == 128 ? 4 : 6);  // bf16 stages
+  static constexpr int kRawStages = FP8 ? 4 : 0;
+  static constexpr int kQBytes = kMaxCols * D_I * 2;
+  static constexpr int kThreads = FP8 ? 320 : 192;
+  // smem layout offsets (from a 1024-aligned base)
+  static constexpr int kOffStages = 0;
+  static constexpr int kOffRaw = kOffStages + kStages * kTileBytes;
+  static constexpr int kOffQ = kOffRaw + kRawStages * kRawBytes;
+  static constexpr int kOffW = kOffQ + kQBytes;
+  static constexpr int kOffNv = kOffW + kMaxCols * 4;
+  static constexpr int kOffBar = kOffNv + 16 * 8;
+  static constexpr int kNumBars = 2 * kStages + 2 * kRawStages + 4 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+};
+
+template <int D_I, int HP, bool FP8>
+__global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
+  using C = IdxCfg<D_I, FP8>;
+  constexpr int GMAX = kMaxCols / HP;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem + C::kOffStages;
+  uint8_t* raw = smem + C::kOffRaw;
+  uint8_t* qs = smem + C::kOffQ;
+  float* ws = reinterpret_cast<float*>(smem + C::kOffW);
+  int64_t* nvs = reinterpret_cast<int64_t*>(smem + C::kOffNv);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* full = bars;                          // [kStages] bf16 tile ready
+  uint64_t* empty = full + C::kStages;            // [kStages] bf16 tile consumed
+  uint64_t* raw_full = empty + C::kStages;        // [kRawStages]
+  uint64_t* raw_empty = raw_full + C::kRawStages; // [kRawStages]
+  uint64_t* acc_full = raw_empty + C::kRawStages; // [2]
+  uint64_t* acc_empty = acc_full + 2;             // [2]
+  uint64_t* q_ready = acc_empty + 2;              // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // This CTA's contiguous share of the (group, tile) work list.
+  const int64_t total = a.total_items;
+  const int64_t lo = total * blockIdx.x / gridDim.x;
+  const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
+  const int ncols = a.G * HP;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&full[i], FP8 ? 128 : 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < C::kRawStages; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 128);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kNumEpiThreads);
+    }
+    mbar_init(q_ready, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&kmap);
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int64_t it = 0;
+      for (int64_t wi = lo; wi < hi; ++wi, ++it) {
+        const int grp = static_cast<int>(wi / a.tiles);
+        const int t = static_cast<int>(wi % a.tiles);
+        const int z = a.per_query ? grp : 0;
+        if constexpr (!FP8) {
+          const int st = static_cast<int>(it % C::kStages);
+          const uint32_t ph = static_cast<uint32_t>((it / C::kStages) & 1);
+          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status)) break;
+          mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+#pragma unroll
+          for (int bk = 0; bk < C::kBlocks; ++bk)
+            tma_load_3d(stages + st * C::kTileBytes + bk * (kTileKeys * 128), &kmap, &full[st], bk * 64,
+                        t * kTileKeys, z);
+        } else {
+          const int st = static_cast<int>(it % C::kRawStages);
+          const uint32_t ph = static_cast<uint32_t>((it / C::kRawStages) & 1);
+          if (!mbar_wait(&raw_empty[st], ph ^ 1, abort_flag, a.status)) break;
+          mbar_arrive_expect_tx(&raw_full[st], C::kRawBytes);
+          tma_load_3d(raw + st * C::kRawBytes, &kmap, &raw_full[st], 0, t * kTileKeys, z);
+        }
+      }
+      if (*abort_flag) {
+        // wind down: let every load this thread issued land before exiting
+        const int S = FP8 ? C::kRawStages : C::kStages;
+        uint64_t* fb = FP8 ? raw_full : full;
+        const int64_t issued = it;  // loads actually issued before the abort
+        for (int64_t j = (issued > S ? issued - S : 0); j < issued; ++j)
+          mbar_drain(&fb[j % S], static_cast<uint32_t>((j / S) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, ncols, false, false);
+      const uint32_t q_addr = smem_u32(qs);
+      int cur_grp = -1;
+      uint32_t q_phase = 0;
+      int64_t it = 0;
+      for (int64_t wi = lo; wi < hi; ++wi, ++it) {
+        const int grp = static_cast<int>(wi / a.tiles);
+        if (grp != cur_grp) {
+          if (!mbar_wait(q_ready, q_phase, abort_flag, a.status)) break;
+          q_phase ^= 1;
+          cur_grp = grp;
+        }
+        const int st = static_cast<int>(it % C::kStages);
+        const uint32_t ph = static_cast<uint32_t>((it / C::kStages) & 1);
+        const int acc = static_cast<int>(it & 1);
+        const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
+        if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status)) break;
+        if (!mbar_wait(&full[st], ph, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(stages + st * C::kTileBytes);
+        const uint32_t d_tmem = tmem_base + acc * 256;
+#pragma unroll
+        for (int kk = 0; kk < D_I / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * (kMaxCols * 128) + (kk & 3) * 32;
+          mma_bf16_ss(d_tmem, sw128_desc(a_addr + koff, 16, 1024), sw128_desc(q_addr + qoff, 16, 1024), idesc,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[st]);
+        mma_commit(&acc_full[acc]);
+      }
+      // make sure nothing issued is still running before TMEM is released
+      mma_commit(q_ready);
+      mbar_drain(q_ready, q_phase);
+    }
+  } else if (warp < kEpiWarp0 + 4) {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..127
+    const int quad = warp & 3;                     // TMEM lane quadrant this warp may access
+    const int row = quad * 32 + lane;              // key row inside the tile
+    int cur_grp = -1;
+    int64_t it = 0;
+    for (int64_t wi = lo; wi < hi; ++wi, ++it) {
+      const int grp = static_cast<int>(wi / a.tiles);
+      const int t = static_cast<int>(wi % a.tiles);
+      if (grp != cur_grp) {
+        // All MMAs of the previous group finished (their accumulators were
+        // drained below), so Q and the weights can be replaced.
+        if (*abort_flag) break;
+        named_bar_sync(1, kNumEpiThreads);
+        const int b0 = grp * a.G;
+        constexpr int kChunksPerRow = D_I / 8;
+        for (int i = et; i < ncols * kChunksPerRow; i += kNumEpiThreads) {
+          const int r = i / kChunksPerRow;
+          const int c8 = i % kChunksPerRow;
+          const int g = r / HP, h = r % HP, b = b0 + g;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (h < a.H_I && b < a.B)
+            v = *reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * a.H_I + h) * D_I + c8 * 8);
+          st_shared_v4(smem_u32(qs + (c8 >> 3) * (kMaxCols * 128) + sw128_offset(r, c8 & 7)), v);
+        }
+        for (int i = et; i < kMaxCols; i += kNumEpiThreads) {
+          const int g = i / HP, h = i % HP, b = b0 + g;
+          ws[i] = (g < a.G && h < a.H_I && b < a.B) ? a.w[static_cast<int64_t>(b) * a.H_I + h] : 0.f;
+        }
+        if (et < GMAX) {
+          const int b = b0 + et;
+          nvs[et] = (et < a.G && b < a.B) ? (a.n_valid ? a.n_valid[b] : a.N) : 0;
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, kNumEpiThreads);
+        if (et == 0) mbar_arrive(q_ready);
+        cur_grp = grp;
+      }
+      const int acc = static_cast<int>(it & 1);
+      const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
+      const bool got = mbar_wait(&acc_full[acc], aph, abort_flag, a.status);
+      __syncwarp();  // tcgen05.ld below is warp-collective
+      if (!got) break;
+      tc_fence_after();
+      float sum[GMAX];
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) sum[g] = 0.f;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256;
+#pragma unroll
+      for (int c0 = 0; c0 < kMaxCols; c0 += 32) {
+        if (c0 < ncols) {
+          float v[32];
+          tmem_ld32(taddr + c0, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int col = c0 + j;
+            sum[col / HP] = fmaf(ws[col], fmaxf(v[j], 0.f), sum[col / HP]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      const int64_t s = static_cast<int64_t>(t) * kTileKeys + row;
+      if (s < a.N) {
+        float scale = 1.f;
+        if constexpr (FP8) {
+          const int64_t zb = a.per_query ? grp : 0;
+          scale = a.k_scale[zb * a.scale_batch_stride + s];
+        }
+        const int b0 = grp * a.G;
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+          if (g < a.G && b0 + g < a.B) {
+            const float val = (s < nvs[g]) ? sum[g] * scale : -INFINITY;
+            a.scores[static_cast<int64_t>(b0 + g) * a.N + s] = val;
+          }
+        }
+      }
+    }
+  } else if constexpr (FP8) {
+    // ------------------------------------------------------------ e4m3 -> bf16
+    const int ct = threadIdx.x - (kEpiWarp0 + 4) * 32;  // 0..127
+    int64_t it = 0;
+    for (int64_t wi = lo; wi < hi; ++wi, ++it) {
+      const int rs = static_cast<int>(it % C::kRawStages);
+      const uint32_t rph = static_cast<uint32_t>((it / C::kRawStages) & 1);
+      const int bs = static_cast<int>(it % C::kStages);
+      const uint32_t bph = static_cast<uint32_t>((it / C::kStages) & 1);
+      if (!mbar_wait(&raw_full[rs], rph, abort_flag, a.status)) break;
+      if (!mbar_wait(&empty[bs], bph ^ 1, abort_flag, a.status)) break;
+      const uint8_t* src = raw + rs * C::kRawBytes;
+      uint8_t* dst = stages + bs * C::kTileBytes;
+      constexpr int kChunks16 = D_I / 16;  // 16-element e4m3 chunks per row
+#pragma unroll 2
+      for (int i = ct; i < kTileKeys * kChunks16; i += 128) {
+        const int r = i / kChunks16, c = i % kChunks16;
+        const uint4 in = *reinterpret_cast<const uint4*>(src + r * D_I + c * 16);
+        const uint32_t w4[4] = {in.x, in.y, in.z, in.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2_raw lo2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w4[j] & 0xFFFF), __NV_E4M3);
+          const __half2_raw hi2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w4[j] >> 16), __NV_E4M3);
+          const float2 flo = __half22float2(*reinterpret_cast<const __half2*>(&lo2));
+          const float2 fhi = __half22float2(*reinterpret_cast<const __half2*>(&hi2));
+          o[2 * j] = pack_bf16x2(flo.x, flo.y);
+          o[2 * j + 1] = pack_bf16x2(fhi.x, fhi.y);
+        }
+        // 16 bf16 = two 16-byte chunks: element offsets c*16 and c*16+8
+        const int e0 = c * 16;
+        const uint32_t base = smem_u32(dst + (e0 >> 6) * (kTileKeys * 128));
+        const int ch = (e0 & 63) >> 3;
+        st_shared_v4(base + sw128_offset(r, ch), make_uint4(o[0], o[1], o[2], o[3]));
+        st_shared_v4(base + sw128_offset(r, ch + 1), make_uint4(o[4], o[5], o[6], o[7]));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&raw_empty[rs]);
+      mbar_arrive(&full[bs]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int D_I, int HP, bool FP8>
+cudaError_t launch_indexer_inst(const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t stream) {
+  using C = IdxCfg<D_I, FP8>;
+  auto kern = indexer_tc_kernel<D_I, HP, FP8>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, a);
+  return cudaGetLastError();
+}
+
+template <int D_I, bool FP8>
+cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t s) {
+  switch (HP) {
+    case 16: return launch_indexer_inst<D_I, 16, FP8>(map, a, grid, s);
+    case 32: return launch_indexer_inst<D_I, 32, FP8>(map, a, grid, s);
+    case 64: return launch_indexer_inst<D_I, 64, FP8>(map, a, grid, s);
+    case 128: return launch_indexer_inst<D_I, 128, FP8>(map, a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int indexer_smem_bytes(int d_I, bool fp8) {
+  if (d_I == 64) return fp8 ? IdxCfg<64, true>::kSmemBytes : IdxCfg<64, false>::kSmemBytes;
+  return fp8 ? IdxCfg<128, true>::kSmemBytes : IdxCfg<128, false>::kSmemBytes;
+}
+
+cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
+                           cudaStream_t stream) {
+  if (d_I == 64) return fp8 ? dispatch_hp<64, true>(HP, map, a, grid, stream) : dispatch_hp<64, false>(HP, map, a, grid, stream);
+  if (d_I == 128) return fp8 ? dispatch_hp<128, true>(HP, map, a, grid, stream) : dispatch_hp<128, false>(HP, map, a, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ic

@@ -1,0 +1,72 @@
+// Kernel argument structs and launchers of the IndexCache hot path (internal
+// to the library; the public boundary is include/indexcache.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cuda_bf16.h>
+
+namespace ic {
+
+struct IndexerArgs {
+  const __nv_bfloat16* q;      // [B, H_I, d_I]
+  const float* w;              // [B, H_I]
+  const float* k_scale;        // e4m3 keys: per-token scale
+  int64_t scale_batch_stride;  // elements between queries' scales
+  const int64_t* n_valid;      // [B] or null
+  float* scores;               // [B, N]
+  int* status;
+  int B, H_I;
+  int64_t N;
+  int G;              // queries per group (share one key tile)
+  int tiles;          // 128-key tiles per group
+  int64_t total_items;  // groups * tiles
+  int per_query;      // 1: key cache z-coordinate = group (G == 1)
+};
+
+int indexer_smem_bytes(int d_I, bool fp8);
+cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
+                           cudaStream_t stream);
+
+struct TopkArgs {
+  const float* scores;      // [B, N]
+  const int64_t* n_valid;   // [B] or null
+  int32_t* idx;             // [B, k]
+  uint32_t* hist;           // [3][B][2048]
+  uint32_t* tie_counts;     // [B][cpr]
+  uint32_t* counters;       // [B][2]: emitted-above count, done CTAs
+  int* status;
+  int B;
+  int64_t N;
+  int k;
+  int cpr;                  // CTAs per row
+  int64_t slice;            // elements per CTA slice
+};
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches);
+
+struct MlaArgs {
+  const __nv_bfloat16* q;    // [B, H, 576]
+  const __nv_bfloat16* kv;   // latent caches
+  int64_t kv_batch_stride;   // elements
+  int64_t N;
+  const int32_t* idx;        // [B, k]
+  int k;
+  const float* sink;         // [H]
+  const __nv_bfloat16* gate; // [B, H, 512] or null
+  float sm_scale;
+  int B, H;
+  int splits;                // ceil(k / TS)
+  int ts;                    // tokens per CTA
+  float* part_o;             // [B, H, splits, 512]
+  float* part_ml;            // [B, H, splits, 2]  (running max in log2 units, sum)
+  void* out;                 // [B, H, 512]
+  int out_f32;
+  float* lse;                // [B, H] or null
+  int* status;
+};
+int mla_smem_bytes(int ts);
+cudaError_t launch_sparse_mla(const MlaArgs& a, cudaStream_t stream, int* launches);
+
+}  // namespace ic

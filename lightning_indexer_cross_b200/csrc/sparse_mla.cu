@@ -1,0 +1,401 @@
+// Sparse MLA decode attention with a per-head sink and a sigmoid output gate
+// on sm_100a tensor cores.
+//
+// For query b, head h, selected rows j (Hy4 IndexCache explainer, Jargon
+// "DSA": token-level selection; Hy4-preview porting issue: head 576 = 512
+// latent + 64 RoPE, per-head "softmax-denominator bias", sigmoid gate):
+//   z_j = sm_scale * q[b,h,:] . kv[idx_j, :]            (576-d)
+//   o   = sum_j e^{z_j} kv[idx_j, :512] / (e^{sink_h} + sum_j e^{z_j})
+//   out = sigmoid(gate[b,h,:]) * o
+//
+// Main kernel: one CTA per (token split of TS <= 256 selected rows, query,
+// block of 128 heads). Tensor memory holds 512 fp32 columns per lane, and the
+// 128 x 512 output alone would fill it, so the CTA works in two phases:
+//   QK   S[128 heads x TS] = Q . KV^T over 9 slices of 64 dims (tcgen05,
+//        M = 128 heads, N = TS tokens) into TMEM columns [0, TS);
+//   soft the epilogue warps read S (one head per TMEM lane), take the exact
+//        max over the CTA's tokens, write P = 2^{z log2e - m} as bf16 into
+//        shared memory in the K-major layout of an MMA A operand;
+//   PV   O_lo = P . V[:, 0:256] into columns [256, 512), then
+//        O_hi = P . V[:, 256:512] into columns [0, 256) (S is dead by then);
+//        V rows are the same gathered 576-d rows, read as an MN-major B
+//        operand (64 tokens x 256 dims per stage).
+// It writes an unnormalised partial (m, l, O) per split. The combine kernel
+// merges the splits, adds e^{sink} once to the denominator, applies the gate
+// and writes out / lse.
+//
+// Gathers are cp.async (16 B, zero fill for -1 rows) into 128-byte-swizzled
+// stages; producer threads fence the async proxy before signalling the MMA.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ic {
+
+namespace {
+
+constexpr int kD = 576;
+constexpr int kDv = 512;
+constexpr int kHeads = 128;      // heads per CTA (MMA M)
+constexpr int kQKChunks = kD / 64;
+constexpr int kStages = 3;
+constexpr int kLookahead = kStages - 1;
+constexpr int kProdThreads = 128;  // warps 0..3
+constexpr int kMmaWarp = 4;
+constexpr int kEpiWarp0 = 5;       // warps 5..8
+constexpr int kThreads = 288;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int TS>
+struct MlaCfg {
+  static constexpr int kQKStage = kHeads * 128 + TS * 128;
+  static constexpr int kPVStage = 64 * 256 * 2;
+  static constexpr int kStageBytes = kQKStage > kPVStage ? kQKStage : kPVStage;
+  static constexpr int kPBytes = kHeads * TS * 2;
+  static constexpr int kOffStages = 0;
+  static constexpr int kOffP = kStages * kStageBytes;
+  static constexpr int kOffIdx = kOffP + kPBytes;
+  static constexpr int kOffBar = kOffIdx + TS * 4;
+  static constexpr int kNumBars = 2 * kStages + 3;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr int kNumSt = kQKChunks + 2 * (TS / 64);
+};
+
+template <int TS>
+__global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a) {
+  using C = MlaCfg<TS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem + C::kOffStages;
+  uint8_t* ps = smem + C::kOffP;
+  int32_t* idx_s = reinterpret_cast<int32_t*>(smem + C::kOffIdx);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = full + kStages;
+  uint64_t* s_full = empty + kStages;
+  uint64_t* p_ready = s_full + 1;
+  uint64_t* o_full = p_ready + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int sp = blockIdx.x;   // token split
+  const int b = blockIdx.y;    // query
+  const int hb = blockIdx.z;   // head block
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tok0 = sp * TS;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], kProdThreads);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_ready, 128);
+    mbar_init(o_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // selected rows of this split; anything outside [0, N) is treated as -1
+  for (int j = threadIdx.x; j < TS; j += kThreads) {
+    int v = -1;
+    if (tok0 + j < a.k) {
+      v = a.idx[static_cast<int64_t>(b) * a.k + tok0 + j];
+      if (v < -1 || static_cast<int64_t>(v) >= a.N) {
+        record_status(a.status, IC_ERR_BAD_INDEX);
+        v = -1;
+      }
+    }
+    idx_s[j] = v;
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp < kMmaWarp) {
+    // ------------------------------------------------------------ producers
+    const int pt = threadIdx.x;
+    const __nv_bfloat16* kvb = a.kv + static_cast<int64_t>(b) * a.kv_batch_stride;
+    const __nv_bfloat16* qb = a.q + (static_cast<int64_t>(b) * a.H) * kD;
+    int s = 0;
+    bool ok = true;
+    for (; s < C::kNumSt; ++s) {
+      const int st = s % kStages;
+      const uint32_t ph = static_cast<uint32_t>((s / kStages) & 1);
+      if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status)) {
+        ok = false;
+        break;
+      }
+      uint8_t* base = stages + st * C::kStageBytes;
+      const uint32_t base_u = smem_u32(base);
+      if (s < kQKChunks) {
+        const int c = s;
+        for (int i = pt; i < kHeads * 8; i += kProdThreads) {
+          const int r = i >> 3, cc = i & 7;
+          const int head = hb * kHeads + r;
+          const bool v = head < a.H;
+          const __nv_bfloat16* src = v ? qb + static_cast<int64_t>(head) * kD + c * 64 + cc * 8 : a.q;
+          cp_async16(base_u + sw128_offset(r, cc), src, v ? 16u : 0u);
+        }
+        for (int i = pt; i < TS * 8; i += kProdThreads) {
+          const int j = i >> 3, cc = i & 7;
+          const int tok = idx_s[j];
+          const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + c * 64 + cc * 8 : a.kv;
+          cp_async16(base_u + kHeads * 128 + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
+        }
+      } else {
+        const int p = s - kQKChunks;
+        const int jh = p / (TS / 64), tc = p % (TS / 64);
+        for (int i = pt; i < 64 * 32; i += kProdThreads) {
+          const int j = i >> 5, bb = (i >> 3) & 3, cc = i & 7;
+          const int tok = idx_s[tc * 64 + j];
+          const __nv_bfloat16* src =
+              tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + jh * 256 + bb * 64 + cc * 8 : a.kv;
+          cp_async16(base_u + bb * 8192 + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
+        }
+      }
+      cp_async_commit();
+      if (s >= kLookahead) {
+        cp_async_wait<kLookahead>();
+        fence_proxy_async_smem();
+        mbar_arrive(&full[(s - kLookahead) % kStages]);
+      }
+    }
+    // land everything still in flight (also on the abort path)
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    if (ok)
+      for (int r = (s > kLookahead ? s - kLookahead : 0); r < s; ++r) mbar_arrive(&full[r % kStages]);
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(128, TS, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+      const uint32_t p_addr = smem_u32(ps);
+      bool ok = true;
+      int s = 0;
+      for (; s < kQKChunks && ok; ++s) {
+        const int st = s % kStages;
+        if (!mbar_wait(&full[st], (s / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t base = smem_u32(stages + st * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tmem_base, sw128_desc(base + kk * 32, 16, 1024),
+                      sw128_desc(base + kHeads * 128 + kk * 32, 16, 1024), idesc_qk, (s | kk) != 0);
+        mma_commit(&empty[st]);
+      }
+      if (ok) {
+        mma_commit(s_full);
+        ok = mbar_wait(p_ready, 0, abort_flag, a.status);
+        tc_fence_after();
+      }
+      for (; s < C::kNumSt && ok; ++s) {
+        const int st = s % kStages;
+        if (!mbar_wait(&full[st], (s / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const int p = s - kQKChunks;
+        const int jh = p / (TS / 64), tc = p % (TS / 64);
+        const uint32_t d_tmem = tmem_base + (jh == 0 ? 256u : 0u);
+        const uint32_t base = smem_u32(stages + st * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(d_tmem, sw128_desc(p_addr + tc * (kHeads * 128) + kk * 32, 16, 1024),
+                      sw128_desc(base + kk * 2048, 8192, 1024), idesc_pv, (tc | kk) != 0);
+        mma_commit(&empty[st]);
+      }
+      // o_full also serves as the "all MMAs retired" fence on the abort path
+      mma_commit(o_full);
+      if (!ok) mbar_drain(o_full, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + output
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;           // head row within the block
+    const int head = hb * kHeads + r;
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const float c2 = a.sm_scale * kLog2e;
+    float mx = -INFINITY, l = 0.f;
+    bool ok = mbar_wait(s_full, 0, abort_flag, a.status);
+    __syncwarp();  // tcgen05.ld is warp-collective
+    if (ok) {
+      tc_fence_after();
+      float m = -INFINITY;
+#pragma unroll 1
+      for (int c0 = 0; c0 < TS; c0 += 32) {
+        float v[32];
+        tmem_ld32(taddr + c0, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (idx_s[c0 + j] >= 0) m = fmaxf(m, v[j]);
+      }
+      mx = m * c2;
+#pragma unroll 1
+      for (int c0 = 0; c0 < TS; c0 += 32) {
+        float v[32];
+        tmem_ld32(taddr + c0, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float p0 = idx_s[c0 + j] >= 0 ? exp2f(fmaf(v[j], c2, -mx)) : 0.f;
+          const float p1 = idx_s[c0 + j + 1] >= 0 ? exp2f(fmaf(v[j + 1], c2, -mx)) : 0.f;
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+          l += __low2float(pb) + __high2float(pb);
+          pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
+        }
+        const uint32_t blk = smem_u32(ps + (c0 >> 6) * (kHeads * 128));
+        const int ch0 = (c0 & 63) >> 3;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          st_shared_v4(blk + sw128_offset(r, ch0 + q4),
+                       make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]));
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(p_ready);
+      ok = mbar_wait(o_full, 0, abort_flag, a.status);
+      __syncwarp();
+    }
+    if (ok) {
+      tc_fence_after();
+      const int64_t row = (static_cast<int64_t>(b) * a.H + head) * a.splits + sp;
+      float* po = a.part_o + row * kDv;
+#pragma unroll 1
+      for (int jh = 0; jh < 2; ++jh) {
+        const uint32_t colbase = jh == 0 ? 256u : 0u;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          float v[32];
+          tmem_ld32(taddr + colbase + c0, v);
+          if (head < a.H) {
+            float4* dst = reinterpret_cast<float4*>(po + jh * 256 + c0);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+          }
+        }
+      }
+      if (head < a.H) {
+        a.part_ml[row * 2 + 0] = mx;
+        a.part_ml[row * 2 + 1] = l;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// One warp per (query, head): merge the splits' (m, l, O), add the sink to
+// the denominator once, normalise, gate, write out and lse.
+__global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  if (gw >= static_cast<int64_t>(a.B) * a.H) return;
+  const int h = static_cast<int>(gw % a.H);
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + gw * a.splits;
+  const float* po = a.part_o + gw * a.splits * kDv;
+  const float sink2 = a.sink[h] * kLog2e;
+  float M = sink2;
+  for (int s = lane; s < a.splits; s += 32) M = fmaxf(M, ml[s].x);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float den = 0.f;
+  for (int s = lane; s < a.splits; s += 32) {
+    const float2 v = ml[s];
+    den += v.x == -INFINITY ? 0.f : exp2f(v.x - M) * v.y;
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+  den += exp2f(sink2 - M);
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  for (int s = 0; s < a.splits; ++s) {
+    const float ms = ml[s].x;
+    if (ms == -INFINITY) continue;
+    const float wgt = exp2f(ms - M);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 o = *reinterpret_cast<const float4*>(po + s * kDv + i * 128 + lane * 4);
+      acc[4 * i] = fmaf(wgt, o.x, acc[4 * i]);
+      acc[4 * i + 1] = fmaf(wgt, o.y, acc[4 * i + 1]);
+      acc[4 * i + 2] = fmaf(wgt, o.z, acc[4 * i + 2]);
+      acc[4 * i + 3] = fmaf(wgt, o.w, acc[4 * i + 3]);
+    }
+  }
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int d0 = i * 128 + lane * 4;
+    float o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = acc[4 * i + e] * inv;
+    if (a.gate) {
+      const uint2 graw = *reinterpret_cast<const uint2*>(a.gate + gw * kDv + d0);
+      const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&graw.x);
+      const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&graw.y);
+      const float g[4] = {__low2float(g01), __high2float(g01), __low2float(g23), __high2float(g23)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] *= 1.f / (1.f + __expf(-g[e]));
+    }
+    if (a.out_f32) {
+      *reinterpret_cast<float4*>(static_cast<float*>(a.out) + gw * kDv + d0) = make_float4(o[0], o[1], o[2], o[3]);
+    } else {
+      uint2 pk;
+      pk.x = pack_bf16x2(o[0], o[1]);
+      pk.y = pack_bf16x2(o[2], o[3]);
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + d0) = pk;
+    }
+  }
+  if (a.lse && lane == 0) a.lse[gw] = (M + log2f(den)) / kLog2e;
+}
+
+template <int TS>
+cudaError_t launch_ts(const MlaArgs& a, cudaStream_t stream) {
+  using C = MlaCfg<TS>;
+  auto kern = sparse_mla_kernel<TS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.splits, a.B, (a.H + kHeads - 1) / kHeads);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int mla_smem_bytes(int ts) {
+  switch (ts) {
+    case 64: return MlaCfg<64>::kSmemBytes;
+    case 128: return MlaCfg<128>::kSmemBytes;
+    default: return MlaCfg<256>::kSmemBytes;
+  }
+}
+
+cudaError_t launch_sparse_mla(const MlaArgs& a, cudaStream_t stream, int* launches) {
+  cudaError_t e;
+  switch (a.ts) {
+    case 64: e = launch_ts<64>(a, stream); break;
+    case 128: e = launch_ts<128>(a, stream); break;
+    case 256: e = launch_ts<256>(a, stream); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  const int64_t warps = static_cast<int64_t>(a.B) * a.H;
+  mla_combine_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(a);
+  *launches += 2;
+  return cudaGetLastError();
+}
+
+}  // namespace ic

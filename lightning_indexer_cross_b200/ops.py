@@ -1,0 +1,165 @@
+"""Torch-tensor front end of the C ABI.
+
+PyTorch provides device memory and the stream; every step of the computation
+runs in the library's CUDA kernels. Functions here check shapes/dtypes,
+allocate outputs and workspaces with torch, and pass raw pointers through
+``_abi``. They refuse CPU tensors: there is no CPU implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import List, Optional, Sequence
+
+import torch
+
+from . import _abi
+
+D_QK = 576
+D_V = 512
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("lightning_indexer_cross_b200 ops need CUDA tensors (no CPU path exists)")
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """Zeroed byte workspace (the status word must start at IC_OK)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def indexer_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: Optional[torch.Tensor] = None,
+                  n_valid: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """scores[b,s] = sum_h w[b,h] ReLU(q[b,h] . k[s]). k: [Bk,N,d_I] bf16 or uint8 (e4m3 codes)."""
+    _need_cuda(q, w, k, k_scale, n_valid)
+    B, H_I, d_I = q.shape
+    Bk, N, dk = k.shape
+    assert dk == d_I and Bk in (1, B)
+    fp8 = k.dtype == torch.uint8
+    assert q.dtype == torch.bfloat16 and w.dtype == torch.float32
+    assert k.dtype in (torch.bfloat16, torch.uint8)
+    if scores is None:
+        scores = torch.empty((B, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(_abi.ic_indexer_workspace_size(), q.device)
+    kbs = k.stride(0) if Bk > 1 else 0
+    sbs = (k_scale.stride(0) if (k_scale is not None and k_scale.shape[0] > 1) else 0)
+    _abi.ic_indexer_score(_ptr(q), _ptr(w), _ptr(k), _ptr(k_scale), _abi.IC_FP8_E4M3 if fp8 else _abi.IC_BF16,
+                          B, H_I, d_I, N, kbs, sbs, _ptr(n_valid), _ptr(scores), _ptr(workspace),
+                          workspace.numel(), _stream_ptr(stream))
+    return scores
+
+
+def topk(scores: torch.Tensor, k: int, n_valid: Optional[torch.Tensor] = None,
+         idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _need_cuda(scores, n_valid)
+    B, N = scores.shape
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    if workspace is None:
+        workspace = new_workspace(_abi.ic_topk_workspace_size(B, N, k), scores.device)
+    _abi.ic_topk(_ptr(scores), B, N, _ptr(n_valid), k, _ptr(idx), _ptr(workspace), workspace.numel(),
+                 _stream_ptr(stream))
+    return idx
+
+
+def sparse_mla_decode(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sink: torch.Tensor,
+                      gate: Optional[torch.Tensor] = None, sm_scale: Optional[float] = None,
+                      out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                      workspace: Optional[torch.Tensor] = None, stream=None):
+    _need_cuda(q, kv, idx, sink, gate)
+    B, H, D = q.shape
+    Bkv, N, Dk = kv.shape
+    assert D == D_QK and Dk == D_QK and Bkv in (1, B)
+    k = idx.shape[1]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D_QK)
+    if out is None:
+        out = torch.empty((B, H, D_V), dtype=out_dtype, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(_abi.ic_sparse_mla_workspace_size(B, H, k), q.device)
+    od = _abi.IC_F32 if out.dtype == torch.float32 else _abi.IC_BF16
+    kvs = kv.stride(0) if Bkv > 1 else 0
+    _abi.ic_sparse_mla_decode(_ptr(q), _ptr(kv), kvs, N, _ptr(idx), k, _ptr(sink), _ptr(gate), float(sm_scale),
+                              B, H, od, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                              _stream_ptr(stream))
+    return out, lse
+
+
+class LayerStack:
+    """Holds the per-layer pointer table, the shape struct, the index buffer
+    and the workspace of one decode stack, so that a step is one C call."""
+
+    def __init__(self, layers: Sequence, schedule: str, B: int, N: int, H_I: int, d_I: int, topk: int, H: int,
+                 k_fp8: bool = False, shared_keys: bool = True, shared_kv: bool = True,
+                 n_valid: Optional[torch.Tensor] = None, sm_scale: Optional[float] = None,
+                 out_dtype: torch.dtype = torch.bfloat16, trace: bool = False, device="cuda",
+                 want_lse: bool = False):
+        self.L = len(schedule)
+        self.schedule = schedule.encode()
+        self.layers = layers
+        self.B, self.topk, self.H = B, topk, H
+        dev = torch.device(device)
+        self.outs: List[torch.Tensor] = [torch.empty((B, H, D_V), dtype=out_dtype, device=dev)
+                                         for _ in range(self.L)]
+        self.lses = [torch.empty((B, H), dtype=torch.float32, device=dev) if want_lse else None
+                     for _ in range(self.L)]
+        first_f = next(l for l in layers if l.k_idx is not None)
+        first_kv = layers[0].kv
+        sh = _abi.ic_stack_shape_t()
+        sh.B, sh.N, sh.H_I, sh.d_I = B, N, H_I, d_I
+        sh.k_dtype = _abi.IC_FP8_E4M3 if k_fp8 else _abi.IC_BF16
+        sh.topk, sh.H = topk, H
+        sh.sm_scale = float(sm_scale if sm_scale is not None else 1.0 / math.sqrt(D_QK))
+        sh.out_dtype = _abi.IC_F32 if out_dtype == torch.float32 else _abi.IC_BF16
+        sh.k_batch_stride = 0 if (shared_keys or B == 1) else first_f.k_idx.stride(0)
+        sh.scale_batch_stride = 0 if (shared_keys or B == 1 or first_f.k_scale is None) else first_f.k_scale.stride(0)
+        sh.kv_batch_stride = 0 if (shared_kv or B == 1) else first_kv.stride(0)
+        sh.n_valid = None if n_valid is None else n_valid.data_ptr()
+        self.n_valid = n_valid
+        self.shape = sh
+        table = (_abi.ic_layer_t * self.L)()
+        for l, lay in enumerate(layers):
+            t = table[l]
+            if schedule[l] == "F":
+                t.q_idx, t.w, t.k_idx = lay.q_idx.data_ptr(), lay.w.data_ptr(), lay.k_idx.data_ptr()
+                t.k_scale = None if lay.k_scale is None else lay.k_scale.data_ptr()
+            t.q, t.kv, t.sink = lay.q.data_ptr(), lay.kv.data_ptr(), lay.sink.data_ptr()
+            t.gate = None if lay.gate is None else lay.gate.data_ptr()
+            t.out = self.outs[l].data_ptr()
+            t.lse = None if self.lses[l] is None else self.lses[l].data_ptr()
+        self.table = table
+        self.index_buf = torch.empty((B, topk), dtype=torch.int32, device=dev)
+        self.trace = torch.empty((self.L, B, topk), dtype=torch.int32, device=dev) if trace else None
+        self.ws = new_workspace(_abi.ic_layer_stack_workspace_size(sh), dev)
+
+    def step(self, stream=None) -> int:
+        """Enqueue one decode step; returns the number of kernels enqueued."""
+        _abi.ic_layer_stack(self.table, self.L, self.schedule, self.shape, _ptr(self.index_buf), _ptr(self.trace),
+                            _ptr(self.ws), self.ws.numel(), _stream_ptr(stream))
+        return _abi.ic_last_launch_count()
+
+    def device_status(self, stream=None) -> int:
+        return _abi.ic_last_device_status(_ptr(self.ws), _stream_ptr(stream))
+
+
+def stack_from_workload(wl, trace: bool = False, out_dtype=torch.bfloat16, want_lse: bool = False) -> LayerStack:
+    return LayerStack(wl.layers, wl.schedule, wl.B, wl.N, wl.H_I, wl.d_I, wl.topk, wl.H, k_fp8=wl.k_fp8,
+                      shared_keys=wl.shared_keys, shared_kv=wl.shared_kv, n_valid=wl.n_valid,
+                      sm_scale=wl.sm_scale, out_dtype=out_dtype, trace=trace,
+                      device=wl.layers[0].q.device, want_lse=want_lse)

@@ -1,0 +1,129 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+the header declares, and rejects bad arguments on the host before launching
+anything. No compute calls are made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from lightning_indexer_cross_b200 import build
+    build.build()
+    from lightning_indexer_cross_b200 import _abi
+    return _abi
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "indexcache.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ic_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree(abi):
+    assert _declared_symbols() == sorted(abi.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(abi):
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(abi):
+    for code in range(6):
+        assert abi.ic_status_string(code).startswith("IC_")
+    assert "unknown" in abi.ic_status_string(77)
+
+
+def _fake(n=1 << 20):
+    # host memory stands in for device pointers: validation must reject before any use
+    buf = (ctypes.c_uint8 * n)()
+    return ctypes.c_void_p(ctypes.addressof(buf) + (-ctypes.addressof(buf)) % 256), buf
+
+
+def test_indexer_rejects_bad_arguments(abi):
+    p, keep = _fake()
+    ws = p
+    call = lambda **kw: abi._indexer(*[kw.get(n, d) for n, d in [
+        ("q", p), ("w", p), ("k", p), ("ks", None), ("dt", abi.IC_BF16), ("B", 2), ("H", 64), ("d", 128),
+        ("N", 1000), ("kbs", 0), ("sbs", 0), ("nv", None), ("s", p), ("ws", ws), ("wsb", 256), ("st", None)]])
+    assert call(q=None) == abi.IC_ERR_INVALID_ARG
+    assert call(B=0) == abi.IC_ERR_INVALID_ARG
+    assert call(N=0) == abi.IC_ERR_INVALID_ARG
+    assert call(d=96) == abi.IC_ERR_UNSUPPORTED
+    assert call(H=129) == abi.IC_ERR_UNSUPPORTED
+    assert call(dt=abi.IC_F32) == abi.IC_ERR_UNSUPPORTED
+    assert call(dt=abi.IC_FP8_E4M3) == abi.IC_ERR_INVALID_ARG  # e4m3 keys need scales
+    assert call(q=ctypes.c_void_p(p.value + 4)) == abi.IC_ERR_INVALID_ARG  # misaligned
+    assert call(kbs=100) == abi.IC_ERR_INVALID_ARG  # stride shorter than a cache
+    assert call(wsb=16) == abi.IC_ERR_INVALID_ARG
+    assert call(ws=None) == abi.IC_ERR_INVALID_ARG
+
+
+def test_topk_rejects_bad_arguments(abi):
+    p, keep = _fake()
+    call = lambda **kw: abi._topk(*[kw.get(n, d) for n, d in [
+        ("s", p), ("B", 2), ("N", 1000), ("nv", None), ("k", 64), ("idx", p), ("ws", p), ("wsb", 1 << 20),
+        ("st", None)]])
+    assert call(k=0) == abi.IC_ERR_INVALID_ARG
+    assert call(k=20000) == abi.IC_ERR_INVALID_ARG
+    assert call(s=None) == abi.IC_ERR_INVALID_ARG
+    assert call(wsb=300) == abi.IC_ERR_INVALID_ARG  # too small for the histograms
+    need = abi.ic_topk_workspace_size(2, 1000, 64)
+    assert need > 3 * 2 * 2048 * 4
+
+
+def test_sparse_mla_rejects_bad_arguments(abi):
+    p, keep = _fake()
+    call = lambda **kw: abi._mla(*[kw.get(n, d) for n, d in [
+        ("q", p), ("kv", p), ("kvs", 0), ("N", 100), ("idx", p), ("k", 16), ("sink", p), ("gate", None),
+        ("sc", 0.04), ("B", 1), ("H", 8), ("od", abi.IC_BF16), ("out", p), ("lse", None), ("ws", p),
+        ("wsb", 1 << 20), ("st", None)]])
+    assert call(sc=0.0) == abi.IC_ERR_INVALID_ARG
+    assert call(sc=-1.0) == abi.IC_ERR_INVALID_ARG
+    assert call(sc=float("nan")) == abi.IC_ERR_INVALID_ARG
+    assert call(od=abi.IC_FP8_E4M3) == abi.IC_ERR_UNSUPPORTED
+    assert call(kvs=10) == abi.IC_ERR_INVALID_ARG
+    assert call(sink=None) == abi.IC_ERR_INVALID_ARG
+    assert call(wsb=64) == abi.IC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("sched", [b"SFFF", b"FXSS", b"FS", b"FSSSS", b"", b"fsss"])
+def test_stack_rejects_bad_schedules(abi, sched):
+    p, keep = _fake()
+    L = 4
+    table = (abi.ic_layer_t * L)()
+    for l in range(L):
+        for f in ("q_idx", "w", "k_idx", "q", "kv", "sink", "out"):
+            setattr(table[l], f, p.value)
+    sh = abi.ic_stack_shape_t()
+    sh.B, sh.N, sh.H_I, sh.d_I, sh.topk, sh.H, sh.sm_scale = 1, 4096, 4, 64, 256, 8, 0.04
+    r = abi._stack(table, L, sched, ctypes.byref(sh), p, None, p, 1 << 20, None)
+    assert r == abi.IC_ERR_INVALID_ARG
+
+
+def test_stack_rejects_missing_indexer_inputs_on_f_layers(abi):
+    p, keep = _fake()
+    L = 3
+    table = (abi.ic_layer_t * L)()
+    for l in range(L):
+        for f in ("q", "kv", "sink", "out"):
+            setattr(table[l], f, p.value)
+    table[0].q_idx, table[0].w, table[0].k_idx = p.value, p.value, p.value
+    sh = abi.ic_stack_shape_t()
+    sh.B, sh.N, sh.H_I, sh.d_I, sh.topk, sh.H, sh.sm_scale = 1, 4096, 4, 64, 256, 8, 0.04
+    # layer 2 is F but has no indexer inputs
+    assert abi._stack(table, L, b"FSF", ctypes.byref(sh), p, None, p, 1 << 30, None) == abi.IC_ERR_INVALID_ARG
+
+
+def test_ops_refuse_cpu_tensors(abi):
+    import torch
+    from lightning_indexer_cross_b200 import ops
+    q = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.indexer_score(q, torch.zeros(1, 4), torch.zeros(1, 10, 64, dtype=torch.bfloat16))

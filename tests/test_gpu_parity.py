@@ -1,0 +1,225 @@
+"""Parity of the CUDA path (through the C ABI) against the float64 oracle,
+at sizes the oracle finishes in seconds that still span several tiles and a
+ragged tail. Every test here needs a B200."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lightning_indexer_cross_b200 import workloads as W
+from tests._helpers import ATTN_TOL, SCORE_TOL, attn_row_error, index_sets_match
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from lightning_indexer_cross_b200 import ops
+    return ops
+
+
+# ------------------------------------------------------------------ indexer
+INDEXER_CASES = [
+    # B, N, H_I, d_I, shared, fp8, causal
+    (1, 4096, 4, 64, False, False, False),
+    (3, 1000, 64, 128, False, False, False),
+    (2, 777, 64, 128, True, False, False),
+    (9, 2500, 64, 128, True, False, True),
+    (5, 1300, 32, 64, True, False, False),
+    (2, 3000, 128, 128, False, False, False),
+    (3, 1500, 64, 128, False, True, False),
+    (6, 1100, 64, 128, True, True, True),
+    (2, 640, 20, 64, False, True, False),
+    (1, 1, 64, 128, False, False, False),
+]
+
+
+@pytest.mark.parametrize("B,N,H_I,d_I,shared,fp8,causal", INDEXER_CASES)
+def test_indexer_matches_oracle(cuda_dev, B, N, H_I, d_I, shared, fp8, causal):
+    q, w, k, ks, nv = W.indexer_case(B, N, H_I, d_I, shared=shared, fp8=fp8, causal=causal, seed=B * 7 + N,
+                                     device=cuda_dev)
+    got = _ops().indexer_score(q, w, k, ks, nv)
+    torch.cuda.synchronize()
+    ref = oracle.indexer_scores(q, w, k, ks, nv, keys_are_e4m3=fp8)
+    g = got.double().cpu().numpy()
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(g), fin), "masking differs"
+    assert np.all(g[~fin] == -np.inf)
+    scale = np.abs(np.where(fin, ref, 0)).max(axis=1, keepdims=True)
+    scale = np.where(scale == 0, 1.0, scale)
+    err = np.abs(np.where(fin, g, 0) - np.where(fin, ref, 0)) / scale
+    assert err.max() <= SCORE_TOL, f"max scaled error {err.max():.3e}"
+
+
+# ------------------------------------------------------------------ top-k
+TOPK_CASES = [
+    # B, N, k, ties, neg_inf_frac, causal
+    (1, 4096, 256, False, 0.0, False),
+    (3, 10000, 2048, False, 0.0, False),
+    (2, 5000, 100, True, 0.0, False),
+    (4, 3001, 64, False, 0.3, False),
+    (5, 20000, 2048, False, 0.0, True),
+    (2, 100, 256, False, 0.0, False),
+    (2, 2048, 2048, False, 0.0, False),
+    (1, 70001, 1, False, 0.0, False),
+    (3, 9000, 500, True, 0.5, True),
+]
+
+
+@pytest.mark.parametrize("B,N,k,ties,ninf,causal", TOPK_CASES)
+def test_topk_is_exact(cuda_dev, B, N, k, ties, ninf, causal):
+    s = W.scores_case(B, N, seed=N + k, ties=ties, neg_inf_frac=ninf, device=cuda_dev)
+    nv = None
+    if causal:
+        g = torch.Generator(device=cuda_dev).manual_seed(3)
+        nv = torch.randint(0, N + 1, (B,), generator=g, device=cuda_dev, dtype=torch.int64)
+        nv[0] = min(k // 2, N)
+    idx = _ops().topk(s, k, nv)
+    torch.cuda.synchronize()
+    ref = oracle.topk_indices(s, k, nv)
+    gi = idx.cpu().numpy()
+    # same fp32 scores on both sides and the same tie rule: the sets are equal
+    for b in range(B):
+        assert set(gi[b][gi[b] >= 0].tolist()) == set(ref[b][ref[b] >= 0].tolist()), f"row {b}"
+        assert (gi[b] == -1).sum() == (ref[b] == -1).sum()
+
+
+def test_topk_all_equal_scores_take_lowest_indices(cuda_dev):
+    s = torch.full((2, 9000), 0.5, device=cuda_dev)
+    idx = _ops().topk(s, 300)
+    torch.cuda.synchronize()
+    for b in range(2):
+        assert sorted(idx[b].tolist()) == list(range(300))
+
+
+def test_topk_deterministic_set(cuda_dev):
+    s = W.scores_case(4, 50000, seed=99, ties=True, device=cuda_dev)
+    a = _ops().topk(s, 2048).sort(dim=1).values
+    b = _ops().topk(s, 2048).sort(dim=1).values
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ sparse MLA
+MLA_CASES = [
+    # B, N, H, k, shared, gate, n_invalid, out dtype
+    (1, 4096, 8, 256, False, False, 0, torch.bfloat16),
+    (2, 3000, 128, 300, False, True, 0, torch.bfloat16),
+    (3, 5000, 128, 2048, True, True, 37, torch.float32),
+    (2, 2500, 16, 64, False, True, 10, torch.float32),
+    (1, 9000, 130, 700, True, False, 0, torch.bfloat16),
+    (8, 4000, 128, 2048, False, True, 0, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("B,N,H,k,shared,gate,n_invalid,odt", MLA_CASES)
+def test_sparse_mla_matches_oracle(cuda_dev, B, N, H, k, shared, gate, n_invalid, odt):
+    q, kv, idx, sink, g = W.attention_case(B, N, H, k, shared=shared, gate=gate, n_invalid=n_invalid,
+                                           seed=B + N + k, device=cuda_dev)
+    out, lse = _ops().sparse_mla_decode(q, kv, idx, sink, g, out_dtype=odt)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.sparse_mla(q, kv, idx, sink, g)
+    err = attn_row_error(out, ref)
+    assert err <= ATTN_TOL[odt], f"attention row error {err:.3e}"
+    np.testing.assert_allclose(lse.double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-3)
+
+
+def test_sparse_mla_all_padding_gives_zero_and_sink_lse(cuda_dev):
+    q, kv, idx, sink, _ = W.attention_case(2, 500, 128, 64, gate=False, seed=5, device=cuda_dev)
+    idx.fill_(-1)
+    out, lse = _ops().sparse_mla_decode(q, kv, idx, sink, None, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+    torch.testing.assert_close(lse, sink.unsqueeze(0).expand(2, -1).contiguous(), rtol=1e-5, atol=1e-5)
+
+
+def test_sparse_mla_bad_index_is_reported_and_skipped(cuda_dev):
+    from lightning_indexer_cross_b200 import _abi
+    ops = _ops()
+    q, kv, idx, sink, _ = W.attention_case(1, 400, 128, 64, gate=False, seed=6, device=cuda_dev)
+    ws = ops.new_workspace(_abi.ic_sparse_mla_workspace_size(1, 128, 64), cuda_dev)
+    good = idx.clone()
+    good[0, 5] = -1
+    bad = idx.clone()
+    bad[0, 5] = 400  # == N: out of range
+    ref_out, _ = ops.sparse_mla_decode(q, kv, good, sink, None, out_dtype=torch.float32, workspace=ws)
+    assert _abi.ic_last_device_status(ops._ptr(ws), ops._stream_ptr()) == _abi.IC_OK
+    out, _ = ops.sparse_mla_decode(q, kv, bad, sink, None, out_dtype=torch.float32, workspace=ws)
+    assert _abi.ic_last_device_status(ops._ptr(ws), ops._stream_ptr()) == _abi.IC_ERR_BAD_INDEX
+    assert _abi.ic_last_device_status(ops._ptr(ws), ops._stream_ptr()) == _abi.IC_OK  # read clears it
+    torch.testing.assert_close(out, ref_out, rtol=0, atol=0)
+
+
+# ------------------------------------------------------------------ layer stack
+def _check_stack(wl, st, check_layers=None, rows=None):
+    """Compare a GPU stack run (with trace) to the oracle on sampled layers/rows."""
+    sched = wl.schedule
+    gov = oracle.governing_full_layer(sched)
+    trace = st.trace.cpu().numpy()
+    rows = list(range(wl.B)) if rows is None else rows
+    # S layers: byte-identical to their governing F layer's buffer
+    for l in range(wl.L):
+        assert trace[l].tobytes() == trace[gov[l]].tobytes(), f"layer {l} differs from layer {gov[l]}"
+    layers = range(wl.L) if check_layers is None else check_layers
+    for l in layers:
+        lay = wl.layers[l]
+        f = gov[l]
+        flay = wl.layers[f]
+        nv = None if wl.n_valid is None else wl.n_valid[rows]
+        kk = flay.k_idx if wl.shared_keys or flay.k_idx.shape[0] == 1 else flay.k_idx[rows]
+        ks = None if flay.k_scale is None else (flay.k_scale if flay.k_scale.shape[0] == 1 else flay.k_scale[rows])
+        sc = oracle.indexer_scores(flay.q_idx[rows], flay.w[rows], kk, ks, nv, keys_are_e4m3=wl.k_fp8)
+        ref_idx = oracle.topk_indices(sc, wl.topk, nv)
+        ok, msg = index_sets_match(trace[f][rows], ref_idx, sc, wl.topk, nv)
+        assert ok, f"layer {f}: {msg}"
+        kv = lay.kv if lay.kv.shape[0] == 1 else lay.kv[rows]
+        gate = None if lay.gate is None else lay.gate[rows]
+        ref, _ = oracle.sparse_mla(lay.q[rows], kv, trace[l][rows], lay.sink, gate, wl.sm_scale)
+        err = attn_row_error(st.outs[l][rows], ref)
+        assert err <= ATTN_TOL[st.outs[l].dtype], f"layer {l}: attention row error {err:.3e}"
+
+
+def test_stack_tiny_four_layers(cuda_dev):
+    wl = W.tiny(cuda_dev)
+    st = _ops().stack_from_workload(wl, trace=True)
+    n = st.step()
+    torch.cuda.synchronize()
+    assert st.device_status() == 0
+    assert n > 0
+    _check_stack(wl, st)
+    got = set(st.trace[0, 0].tolist())
+    assert set(wl.planted[0].tolist()) <= got  # planted tokens recovered
+
+
+def test_stack_small_hy4_like_schedule(cuda_dev):
+    sched = "FFFSSSFSSF"
+    wl = W.stack(cuda_dev, seed=21, L=len(sched), B=4, N=9000, topk=512, schedule=sched)
+    st = _ops().stack_from_workload(wl, trace=True, out_dtype=torch.float32)
+    st.step()
+    torch.cuda.synchronize()
+    assert st.device_status() == 0
+    _check_stack(wl, st)
+
+
+def test_stack_per_query_caches_fp8(cuda_dev):
+    wl = W.long_context(cuda_dev, N=20000, B=3, fp8=True, n_planted=16)
+    st = _ops().stack_from_workload(wl, trace=True)
+    st.step()
+    torch.cuda.synchronize()
+    assert st.device_status() == 0
+    _check_stack(wl, st)
+    for b in range(wl.B):
+        assert set(wl.planted[b].tolist()) <= set(st.trace[0, b].tolist())
+
+
+def test_stack_rerun_is_repeatable(cuda_dev):
+    wl = W.stack(cuda_dev, seed=22, L=4, B=2, N=5000, topk=256, schedule="FSFS")
+    st = _ops().stack_from_workload(wl, trace=True)
+    st.step()
+    a = [o.clone() for o in st.outs]
+    ta = st.trace.sort(dim=2).values.clone()
+    st.step()
+    torch.cuda.synchronize()
+    assert torch.equal(ta, st.trace.sort(dim=2).values)
+    for x, y in zip(a, st.outs):
+        torch.testing.assert_close(x.float(), y.float(), rtol=2e-2, atol=2e-2)
