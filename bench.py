@@ -356,16 +356,26 @@ def load_traffic(kernel):
         return None
 
 
-def _time_loop(fn, n, stream):
+def _time_loop(fn, n, stream, replays=3):
+    """Capture n calls of fn in a CUDA graph (so host launch cost cannot hide
+    in the number), replay it, and return the mean device time per call (us)
+    measured with events on the stream the kernels run on."""
     import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(n):
-        fn(i)
-    e1.record(stream)
+    e0.record(cur)
+    for _ in range(replays):
+        g.replay()
+    e1.record(cur)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) * 1000.0 / n  # us
+    return e0.elapsed_time(e1) * 1000.0 / (n * replays)  # us
 
 
 def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
@@ -373,7 +383,7 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
     the layers' own inputs (so each launch streams fresh data from HBM)."""
     import torch
     from lightning_indexer_cross_b200 import _abi, ops
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.Stream(device=dev)
     f_layers = [l for l in range(wl.L) if wl.schedule[l] == "F"]
     scores = torch.empty((B, N), dtype=torch.float32, device=dev)
     ws_i = ops.new_workspace(_abi.ic_indexer_workspace_size(), dev)
@@ -381,7 +391,7 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
     ws_m = ops.new_workspace(_abi.ic_sparse_mla_workspace_size(B, H, TOPK), dev)
     idx = torch.empty((B, TOPK), dtype=torch.int32, device=dev)
     out = torch.empty((B, H, D_V), dtype=torch.bfloat16, device=dev)
-    reps = max(3 * len(f_layers), min(args.steps, 200))
+    reps = 2 * len(f_layers)
 
     def ind(i):
         lay = wl.layers[f_layers[i % len(f_layers)]]
@@ -411,7 +421,7 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
     t_ind = _time_loop(ind, reps, stream)
     # top-k reads scores written just before (as in the stack); time it alone
     t_tk = _time_loop(tk, reps, stream)
-    t_mla = _time_loop(mla, max(reps, wl.L), stream)
+    t_mla = _time_loop(mla, wl.L, stream)
 
     # algorithmic work per launch
     ind_bytes = N * D_I * 2 + B * H_I * D_I * 2 + B * H_I * 4 + B * N * 4
@@ -437,7 +447,7 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
                     "roofline": roofline(ind_bytes, ind_flops, t_ind)},
         "topk": {"us": t_tk, "launches": reps, "elems_per_s": B * N / (t_tk * 1e-6),
                  "roofline": roofline(tk_bytes, 0.0, t_tk)},
-        "sparse_mla": {"us": t_mla, "launches": max(reps, wl.L), "gbs": mla_bytes / (t_mla * 1e-6) / 1e9,
+        "sparse_mla": {"us": t_mla, "launches": wl.L, "gbs": mla_bytes / (t_mla * 1e-6) / 1e9,
                        "distinct_rows_per_layer": mla_rows,
                        "roofline": roofline(mla_bytes, mla_flops, t_mla)},
     }

@@ -10,6 +10,20 @@
 
 namespace ic {
 
+// Raise a kernel's dynamic shared-memory limit once per device (never again
+// afterwards, so later calls are safe inside CUDA-graph capture).
+template <typename Kernel>
+inline cudaError_t set_smem_once(Kernel kern, int bytes) {
+  static bool done[64] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
+
 struct IndexerArgs {
   const __nv_bfloat16* q;      // [B, H_I, d_I]
   const float* w;              // [B, H_I]
