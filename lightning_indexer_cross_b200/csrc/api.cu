@@ -121,13 +121,11 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   return IC_OK;
 }
 
-// ------------------------------------------------------------------ top-k
-struct TopkLayout {
-  int cpr;
-  int64_t slice;
-  size_t hist_off, tie_off, cnt_off, total;
-};
+}  // namespace
 
+namespace ic {
+
+// ------------------------------------------------------------------ top-k
 TopkLayout topk_layout(int B, int64_t N) {
   TopkLayout L{};
   const int64_t target = std::max<int64_t>(1, 592 / std::max(B, 1));
@@ -172,6 +170,14 @@ ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_va
   g_launches += launches + 1;  // + the memset
   return IC_OK;
 }
+
+}  // namespace ic
+
+namespace {
+
+using ic::TopkLayout;
+using ic::topk_layout;
+using ic::topk_impl;
 
 // ------------------------------------------------------------------ sparse MLA
 int mla_ts(int B, int H, int k) {

@@ -327,7 +327,8 @@ template <int D_I, int HP, bool FP8>
 cudaError_t launch_indexer_inst(const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t stream) {
   using C = IdxCfg<D_I, FP8>;
   auto kern = indexer_tc_kernel<D_I, HP, FP8>;
-  cudaError_t e = set_smem_once(kern, C::kSmemBytes);
+  static bool done[64] = {false};  // one flag set per template instance
+  cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, a);
   return cudaGetLastError();

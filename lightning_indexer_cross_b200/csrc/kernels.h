@@ -8,13 +8,16 @@
 
 #include <cuda_bf16.h>
 
+#include "../../include/indexcache.h"
+
 namespace ic {
 
 // Raise a kernel's dynamic shared-memory limit once per device (never again
-// afterwards, so later calls are safe inside CUDA-graph capture).
+// afterwards, so later calls are safe inside CUDA-graph capture). `done` is
+// the caller's per-kernel flag array: kernels of one signature share a
+// function type, so the flag cannot live in this template.
 template <typename Kernel>
-inline cudaError_t set_smem_once(Kernel kern, int bytes) {
-  static bool done[64] = {false};
+inline cudaError_t set_smem_once(Kernel kern, int bytes, bool (&done)[64]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -59,6 +62,18 @@ struct TopkArgs {
   int64_t slice;            // elements per CTA slice
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches);
+
+// Scratch layout of the top-k passes for B rows of N scores (byte offsets
+// from the start of the scratch region, which follows the status word).
+struct TopkLayout {
+  int cpr;
+  int64_t slice;
+  size_t hist_off, tie_off, cnt_off, total;
+};
+TopkLayout topk_layout(int B, int64_t N);
+// Validate, clear the scratch region and enqueue the top-k passes.
+ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_valid, int k, int32_t* idx,
+                      uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream);
 
 struct MlaArgs {
   const __nv_bfloat16* q;    // [B, H, 576]

@@ -366,7 +366,8 @@ template <int TS>
 cudaError_t launch_ts(const MlaArgs& a, cudaStream_t stream) {
   using C = MlaCfg<TS>;
   auto kern = sparse_mla_kernel<TS>;
-  cudaError_t e = set_smem_once(kern, C::kSmemBytes);
+  static bool done[64] = {false};  // one flag set per template instance
+  cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.B, (a.H + kHeads - 1) / kHeads);
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(a);
