@@ -102,6 +102,25 @@ ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_vali
 size_t ic_topk_workspace_size(int B, int64_t N, int k);
 
 /* ---------------------------------------------------------------------------
+ * ic_topk_noalloc -- ic_topk for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is an interface choice of the library.
+ *
+ * Same result and limits as ic_topk, but takes no workspace: its scratch is
+ * a fixed array inside the library (about 1.6 MB on every GPU that loads
+ * it, held until exit). Meant for code that cannot call cudaMalloc, e.g.
+ * enqueueing inside a CUDA-graph capture that forbids allocation, or engine
+ * plugins that only receive their input and output buffers.
+ *   - At most IC_TOPK_NOALLOC_MAX_ROWS rows; more returns IC_ERR_UNSUPPORTED
+ *     with nothing launched.
+ *   - All calls share the one array; calls that overlap on the GPU race.
+ *   - The first call on a device looks up the array's address; make it
+ *     before any stream capture. Device-side status is not reported.
+ * ------------------------------------------------------------------------- */
+#define IC_TOPK_NOALLOC_MAX_ROWS 64
+ic_status_t ic_topk_noalloc(const float* scores, int B, int64_t N, const int64_t* n_valid, int k,
+                            int32_t* idx, ic_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * ic_sparse_mla_decode -- DSA token-level sparse attention, MLA shape,
  * with a per-head sink and a sigmoid output gate (Hy4 IndexCache explainer,
  * Jargon "DSA"; Hy4-preview porting issue: head 576 = 512 latent + 64 RoPE,

@@ -30,6 +30,7 @@ EXPORTED = [
     "ic_indexer_workspace_size",
     "ic_topk",
     "ic_topk_workspace_size",
+    "ic_topk_noalloc",
     "ic_sparse_mla_decode",
     "ic_sparse_mla_workspace_size",
     "ic_layer_stack",
@@ -86,6 +87,7 @@ _indexer = _sig("ic_indexer_score", _i, [_p, _p, _p, _p, _i, _i, _i, _i, _i64, _
 _indexer_ws = _sig("ic_indexer_workspace_size", _sz, [])
 _topk = _sig("ic_topk", _i, [_p, _i, _i64, _p, _i, _p, _p, _sz, _p])
 _topk_ws = _sig("ic_topk_workspace_size", _sz, [_i, _i64, _i])
+_topk_noalloc = _sig("ic_topk_noalloc", _i, [_p, _i, _i64, _p, _i, _p, _p])
 _mla = _sig("ic_sparse_mla_decode", _i,
             [_p, _p, _i64, _i64, _p, _i, _p, _p, _f, _i, _i, _i, _p, _p, _p, _sz, _p])
 _mla_ws = _sig("ic_sparse_mla_workspace_size", _sz, [_i, _i, _i])
@@ -118,6 +120,14 @@ def ic_indexer_workspace_size() -> int:
 
 def ic_topk(scores, B, N, n_valid, k, idx, workspace, ws_bytes, stream) -> None:
     _check(_topk(scores, B, N, n_valid, k, idx, workspace, ws_bytes, stream), "ic_topk")
+
+
+def ic_topk_noalloc(scores, B, N, n_valid, k, idx, stream) -> None:
+    """Top-k with the library's built-in scratch (no workspace argument)."""
+    _check(_topk_noalloc(scores, B, N, n_valid, k, idx, stream), "ic_topk_noalloc")
+
+
+IC_TOPK_NOALLOC_MAX_ROWS = 64
 
 
 def ic_topk_workspace_size(B, N, k) -> int:
