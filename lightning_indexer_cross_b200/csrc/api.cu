@@ -128,7 +128,8 @@ namespace ic {
 // ------------------------------------------------------------------ top-k
 TopkLayout topk_layout(int B, int64_t N) {
   TopkLayout L{};
-  const int64_t target = std::max<int64_t>(1, 592 / std::max(B, 1));
+  // about four 512-thread CTAs per SM in total, and at least 4096 scores per CTA
+  const int64_t target = std::max<int64_t>(1, 4 * num_sms() / std::max(B, 1));
   int64_t cpr = std::min<int64_t>(ceil_div<int64_t>(N, 4096), target);
   cpr = std::max<int64_t>(cpr, 1);
   int64_t slice = ceil_div<int64_t>(N, cpr);
@@ -139,7 +140,7 @@ TopkLayout topk_layout(int B, int64_t N) {
   L.hist_off = 0;
   L.tie_off = align256(L.hist_off + size_t(3) * B * 2048 * 4);
   L.cnt_off = align256(L.tie_off + size_t(B) * L.cpr * 4);
-  L.total = align256(L.cnt_off + size_t(B) * 2 * 4);
+  L.total = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
   return L;
 }
 
@@ -218,6 +219,20 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
     return IC_ERR_INVALID_ARG;
   MlaLayout L = mla_layout(B, H, k);
   if (ws_bytes < L.total) return IC_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * H >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return IC_ERR_CUDA;
+  CUtensorMap qmap;
+  {
+    const cuuint64_t dims[2] = {576, static_cast<cuuint64_t>(B) * H};
+    const cuuint64_t strides[1] = {576 * 2};
+    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return IC_ERR_INVALID_ARG;
+  }
   ic::MlaArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.kv = static_cast<const __nv_bfloat16*>(kv);
@@ -232,14 +247,14 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
   a.H = H;
   a.splits = L.splits;
   a.ts = L.ts;
-  a.part_o = reinterpret_cast<float*>(ws + L.o_off);
+  a.part_o = ws + L.o_off;
   a.part_ml = reinterpret_cast<float*>(ws + L.ml_off);
   a.out = out;
   a.out_f32 = out_dtype == IC_F32 ? 1 : 0;
   a.lse = lse;
   a.status = status;
   int launches = 0;
-  cudaError_t e = ic::launch_sparse_mla(a, stream, &launches);
+  cudaError_t e = ic::launch_sparse_mla(qmap, a, stream, &launches);
   if (e != cudaSuccess) return IC_ERR_CUDA;
   g_launches += launches;
   return IC_OK;

@@ -28,6 +28,8 @@
 //               head sum, since ReLU(c x) = c ReLU(x) for c >= 0.
 #include <cuda_fp8.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,7 +40,6 @@ namespace {
 constexpr int kTileKeys = 128;
 constexpr int kMaxCols = 256;  // MMA N limit for M = 128
 constexpr int kEpiWarp0 = 2;
-constexpr int kNumEpiThreads = 128;
 
 template <int D_I, bool FP8>
 struct IdxCfg {
@@ -48,6 +49,12 @@ struct IdxCfg {
   static constexpr int kStages = FP8 ? 2 : (D_I == 128 ? 4 : 6);  // bf16 stages
   static constexpr int kRawStages = FP8 ? 4 : 0;
   static constexpr int kQBytes = kMaxCols * D_I * 2;
+  // 4 epilogue warps (one per TMEM lane quadrant); e4m3 keys add 4 converter
+  // warps. With 6 warps every thread may hold up to 255 registers, which the
+  // epilogue's 128-register TMEM payload needs.
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kHalves = 1;
+  static constexpr int kEpiThreads = kEpiWarps * 32;
   static constexpr int kThreads = FP8 ? 320 : 192;
   // smem layout offsets (from a 1024-aligned base)
   static constexpr int kOffStages = 0;
@@ -104,7 +111,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], kNumEpiThreads);
+      mbar_init(&acc_empty[i], C::kEpiThreads);
     }
     mbar_init(q_ready, 1);
     *abort_flag = 0;
@@ -192,11 +199,13 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
       mma_commit(q_ready);
       mbar_drain(q_ready, q_phase);
     }
-  } else if (warp < kEpiWarp0 + 4) {
+  } else if (warp < kEpiWarp0 + C::kEpiWarps) {
     // ------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - kEpiWarp0 * 32;  // 0..127
-    const int quad = warp & 3;                     // TMEM lane quadrant this warp may access
-    const int row = quad * 32 + lane;              // key row inside the tile
+    constexpr int kNumEpiThreads = C::kEpiThreads;
+    const int et = threadIdx.x - kEpiWarp0 * 32;    // 0 .. kNumEpiThreads-1
+    const int quad = warp & 3;                       // TMEM lane quadrant this warp may access
+    const int half = (warp - kEpiWarp0) >> 2;        // which half of the columns
+    const int row = quad * 32 + lane;                // key row inside the tile
     int cur_grp = -1;
     int64_t it = 0;
     for (int64_t wi = lo; wi < hi; ++wi, ++it) {
@@ -237,39 +246,79 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
       __syncwarp();  // tcgen05.ld below is warp-collective
       if (!got) break;
       tc_fence_after();
-      float sum[GMAX];
-#pragma unroll
-      for (int g = 0; g < GMAX; ++g) sum[g] = 0.f;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256;
-#pragma unroll
-      for (int c0 = 0; c0 < kMaxCols; c0 += 32) {
-        if (c0 < ncols) {
-          float v[32];
-          tmem_ld32(taddr + c0, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int col = c0 + j;
-            sum[col / HP] = fmaf(ws[col], fmaxf(v[j], 0.f), sum[col / HP]);
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      const int b0 = grp * a.G;
       const int64_t s = static_cast<int64_t>(t) * kTileKeys + row;
-      if (s < a.N) {
-        float scale = 1.f;
-        if constexpr (FP8) {
-          const int64_t zb = a.per_query ? grp : 0;
-          scale = a.k_scale[zb * a.scale_batch_stride + s];
-        }
-        const int b0 = grp * a.G;
+      // One half of the columns = a contiguous run of whole queries.
+      auto tile_half = [&](auto half_c) {
+        constexpr int H = decltype(half_c)::value;
+        constexpr int kChunks = kMaxCols / 32 / C::kHalves;  // 32-column chunks of this half
+        constexpr int kC0 = H * kChunks;
+        constexpr int kQ = GMAX / C::kHalves;                 // queries of this half
+        constexpr int kQ0 = H * kQ;
+        // NP partial sums per query keep the FMA dependency chains short
+        constexpr int NP = HP >= 64 ? 4 : (HP == 32 ? 2 : 1);
+        float sum[kQ][NP];
 #pragma unroll
-        for (int g = 0; g < GMAX; ++g) {
-          if (g < a.G && b0 + g < a.B) {
-            const float val = (s < nvs[g]) ? sum[g] * scale : -INFINITY;
-            a.scores[static_cast<int64_t>(b0 + g) * a.N + s] = val;
+        for (int g = 0; g < kQ; ++g)
+#pragma unroll
+          for (int p = 0; p < NP; ++p) sum[g][p] = 0.f;
+        // The half's columns come in as two 64-column TMEM loads issued back
+        // to back with a single wait: one load latency per tile, not one per
+        // 32 columns.
+        static_assert(kChunks == 4 || kChunks == 8, "half = 128 or 256 columns");
+        constexpr int kLoads = kChunks / 2;  // 64-column loads of this half
+#pragma unroll
+        for (int pass = 0; pass < kLoads; pass += 2) {
+          const int cA = (kC0 + 2 * pass) * 32, cB = cA + 64;
+          const bool haveA = cA < ncols, haveB = cB < ncols && pass + 1 < kLoads;
+          uint32_t ra[64], rb[64];
+          if (haveA) tmem_ld64_issue(taddr + cA, ra);
+          if (haveB) tmem_ld64_issue(taddr + cB, rb);
+          if (haveA) tmem_ld_wait64(ra);
+          if (haveB) tmem_ld_wait64(rb);
+          auto reduce64 = [&](const uint32_t (&rv)[64], int cbase) {
+#pragma unroll
+            for (int j4 = 0; j4 < 16; ++j4) {
+              const float4 wv = ld_shared_v4f(ws + cbase + 4 * j4);
+              const float wj[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int j = j4 * 4 + e;
+                float& acc_ref = sum[(cbase + j) / HP - kQ0][j % NP];
+                acc_ref = fmaf(wj[e], fmaxf(__uint_as_float(rv[j]), 0.f), acc_ref);
+              }
+            }
+          };
+          if (haveA) reduce64(ra, (kC0 + 2 * pass) * 32);
+          if (haveB) reduce64(rb, (kC0 + 2 * pass) * 32 + 64);
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[acc]);
+        if (s < a.N) {
+          float scale = 1.f;
+          if constexpr (FP8) {
+            const int64_t zb = a.per_query ? grp : 0;
+            scale = a.k_scale[zb * a.scale_batch_stride + s];
+          }
+#pragma unroll
+          for (int g = 0; g < kQ; ++g) {
+            const int gg = kQ0 + g;
+            if (gg < a.G && b0 + gg < a.B) {
+              float tot = 0.f;
+#pragma unroll
+              for (int p = 0; p < NP; ++p) tot += sum[g][p];
+              const float val = (s < nvs[gg]) ? tot * scale : -INFINITY;
+              a.scores[static_cast<int64_t>(b0 + gg) * a.N + s] = val;
+            }
           }
         }
+      };
+      if constexpr (C::kHalves == 2) {
+        if (half == 0) tile_half(std::integral_constant<int, 0>{});
+        else tile_half(std::integral_constant<int, 1>{});
+      } else {
+        tile_half(std::integral_constant<int, 0>{});
       }
     }
   } else if constexpr (FP8) {

@@ -47,13 +47,17 @@ int indexer_smem_bytes(int d_I, bool fp8);
 cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
                            cudaStream_t stream);
 
+// 32-bit words of per-row top-k control state (one 128-byte line per row,
+// so rows do not contend for the same line in L2).
+constexpr int kCtrlWords = 32;
+
 struct TopkArgs {
   const float* scores;      // [B, N]
   const int64_t* n_valid;   // [B] or null
   int32_t* idx;             // [B, k]
   uint32_t* hist;           // [3][B][2048]
   uint32_t* tie_counts;     // [B][cpr]
-  uint32_t* counters;       // [B][2]: emitted-above count, done CTAs
+  uint32_t* counters;       // [B][kCtrlWords] per-row control state
   int* status;
   int B;
   int64_t N;
@@ -88,14 +92,16 @@ struct MlaArgs {
   int B, H;
   int splits;                // ceil(k / TS)
   int ts;                    // tokens per CTA
-  float* part_o;             // [B, H, splits, 512]
-  float* part_ml;            // [B, H, splits, 2]  (running max in log2 units, sum)
+  void* part_o;              // [B, H, splits, 512] normalised O/l: bf16 if out is bf16, else fp32
+  float* part_ml;            // [B, H, splits, 2]  (max in log2 units, sum)
   void* out;                 // [B, H, 512]
   int out_f32;
   float* lse;                // [B, H] or null
   int* status;
 };
 int mla_smem_bytes(int ts);
-cudaError_t launch_sparse_mla(const MlaArgs& a, cudaStream_t stream, int* launches);
+// qmap: 2-D tensor map over q viewed as [B*H rows, 576] bf16, box 64 x 128,
+// 128-byte swizzle (one 64-dim slice of a 128-head block per load).
+cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const MlaArgs& a, cudaStream_t stream, int* launches);
 
 }  // namespace ic

@@ -38,11 +38,13 @@ constexpr int kDv = 512;
 constexpr int kHeads = 128;      // heads per CTA (MMA M)
 constexpr int kQKChunks = kD / 64;
 constexpr int kStages = 3;
+// 8 warps (two per SM sub-partition, so up to 255 registers per thread):
+// three gather warps, the MMA issuer, four epilogue warps (TMEM lane quadrants)
+constexpr int kProdThreads = 96;   // warps 0..2
+constexpr int kMmaWarp = 3;
+constexpr int kEpiWarp0 = 4;       // warps 4..7
+constexpr int kThreads = 256;
 constexpr int kLookahead = kStages - 1;
-constexpr int kProdThreads = 128;  // warps 0..3
-constexpr int kMmaWarp = 4;
-constexpr int kEpiWarp0 = 5;       // warps 5..8
-constexpr int kThreads = 288;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int TS>
@@ -54,7 +56,8 @@ struct MlaCfg {
   static constexpr int kOffStages = 0;
   static constexpr int kOffP = kStages * kStageBytes;
   static constexpr int kOffIdx = kOffP + kPBytes;
-  static constexpr int kOffBar = kOffIdx + TS * 4;
+  static constexpr int kOffMask = kOffIdx + TS * 4;
+  static constexpr int kOffBar = kOffMask + (TS / 32) * 4 + 8;
   static constexpr int kNumBars = 2 * kStages + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
@@ -62,13 +65,15 @@ struct MlaCfg {
 };
 
 template <int TS>
-__global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                   const MlaArgs a) {
   using C = MlaCfg<TS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem + C::kOffStages;
   uint8_t* ps = smem + C::kOffP;
   int32_t* idx_s = reinterpret_cast<int32_t*>(smem + C::kOffIdx);
+  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + C::kOffMask);  // bit j of word w: token 32w+j valid
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;
@@ -90,13 +95,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a
       mbar_init(&empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_ready, 128);
+    mbar_init(p_ready, 128);  // the four epilogue warps
     mbar_init(o_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   // selected rows of this split; anything outside [0, N) is treated as -1
-  for (int j = threadIdx.x; j < TS; j += kThreads) {
+  static_assert(TS % 32 == 0, "whole warps of selected rows");
+  for (int j0 = warp * 32; j0 < TS; j0 += kThreads) {  // warp-uniform
+    const int j = j0 + lane;
     int v = -1;
     if (tok0 + j < a.k) {
       v = a.idx[static_cast<int64_t>(b) * a.k + tok0 + j];
@@ -106,6 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a
       }
     }
     idx_s[j] = v;
+    const uint32_t bal = __ballot_sync(0xffffffffu, v >= 0);
+    if (lane == 0) vmask[j0 >> 5] = bal;
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_holder, 512);
@@ -117,10 +126,38 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp < kMmaWarp) {
-    // ------------------------------------------------------------ producers
+    // ------------------------------------------------------------ gather warps
+    // QK stage c: the 64-dim slice c of the 128-head Q block by one TMA load,
+    // and slice c of every selected row by cp.async. PV stage: 64 selected
+    // rows x 256 latent dims by cp.async. Rows land in 128-byte-swizzled
+    // operand layouts; -1 slots are zero-filled (their logits are masked).
+    // (Measured on B200: 16-byte cp.async gathers sustain more bytes in
+    // flight per SM than 512-byte tile::gather4 TMA operations here.)
     const int pt = threadIdx.x;
     const __nv_bfloat16* kvb = a.kv + static_cast<int64_t>(b) * a.kv_batch_stride;
-    const __nv_bfloat16* qb = a.q + (static_cast<int64_t>(b) * a.H) * kD;
+    if (pt == 0) tma_prefetch_desc(&qmap);
+    // stage r's copies are in place: every gather thread arrives once; for
+    // QK stages thread 0's arrival also books the TMA bytes of the Q slice
+    auto arrive_stage = [&](int r) {
+      if (pt == 0 && r < kQKChunks) mbar_arrive_expect_tx(&full[r % kStages], kHeads * 128);
+      else mbar_arrive(&full[r % kStages]);
+    };
+    // Copy i of a stage is row i/8 (QK) or row-block i/8 (PV), 16-byte chunk
+    // i%8. Thread pt takes i = pt + kProdThreads*n, so its chunk column
+    // cc = pt % 8 is fixed and its QK rows (pt/8 + kRowStep*n) are the same
+    // in all nine QK stages: they are loaded into registers once.
+    constexpr int kNQ = (TS * 8 + kProdThreads - 1) / kProdThreads;
+    constexpr int kNP = (64 * 32 + kProdThreads - 1) / kProdThreads;
+    static_assert(kProdThreads % 8 == 0, "chunk column fixed per thread");
+    constexpr int kRowStep = kProdThreads / 8;
+    const int cc = pt & 7;
+    const int q0 = pt >> 3;  // 0 .. kRowStep-1
+    int qk_tok[kNQ];
+#pragma unroll
+    for (int n = 0; n < kNQ; ++n) {
+      const int j = q0 + kRowStep * n;
+      qk_tok[n] = j < TS ? idx_s[j] : -1;
+    }
     int s = 0;
     bool ok = true;
     for (; s < C::kNumSt; ++s) {
@@ -134,42 +171,57 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a
       const uint32_t base_u = smem_u32(base);
       if (s < kQKChunks) {
         const int c = s;
-        for (int i = pt; i < kHeads * 8; i += kProdThreads) {
-          const int r = i >> 3, cc = i & 7;
-          const int head = hb * kHeads + r;
-          const bool v = head < a.H;
-          const __nv_bfloat16* src = v ? qb + static_cast<int64_t>(head) * kD + c * 64 + cc * 8 : a.q;
-          cp_async16(base_u + sw128_offset(r, cc), src, v ? 16u : 0u);
-        }
-        for (int i = pt; i < TS * 8; i += kProdThreads) {
-          const int j = i >> 3, cc = i & 7;
-          const int tok = idx_s[j];
-          const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + c * 64 + cc * 8 : a.kv;
-          cp_async16(base_u + kHeads * 128 + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
+        // rows past the last query read zeros; rows of a neighbouring query
+        // are never written out
+        if (pt == 0) tma_load_2d(base, &qmap, &full[st], c * 64, b * a.H + hb * kHeads);
+        const uint32_t kv_u = base_u + kHeads * 128;
+#pragma unroll
+        for (int n = 0; n < kNQ; ++n) {
+          const int j = q0 + kRowStep * n;
+          if (j < TS) {
+            const int tok = qk_tok[n];
+            const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + c * 64 + cc * 8 : a.kv;
+            cp_async16(kv_u + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
+          }
         }
       } else {
         const int p = s - kQKChunks;
         const int jh = p / (TS / 64), tc = p % (TS / 64);
-        for (int i = pt; i < 64 * 32; i += kProdThreads) {
-          const int j = i >> 5, bb = (i >> 3) & 3, cc = i & 7;
-          const int tok = idx_s[tc * 64 + j];
-          const __nv_bfloat16* src =
-              tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + jh * 256 + bb * 64 + cc * 8 : a.kv;
-          cp_async16(base_u + bb * 8192 + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
+        int pv_tok[kNP];
+#pragma unroll
+        for (int n = 0; n < kNP; ++n) {
+          const int q = q0 + kRowStep * n;  // (token in chunk) * 4 + 64-dim block
+          pv_tok[n] = q < 256 ? idx_s[tc * 64 + (q >> 2)] : -1;
+        }
+#pragma unroll
+        for (int n = 0; n < kNP; ++n) {
+          const int q = q0 + kRowStep * n;
+          if (q < 256) {
+            const int j = q >> 2, bb = q & 3;
+            const int tok = pv_tok[n];
+            const __nv_bfloat16* src =
+                tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + jh * 256 + bb * 64 + cc * 8 : a.kv;
+            cp_async16(base_u + bb * 8192 + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
+          }
         }
       }
       cp_async_commit();
       if (s >= kLookahead) {
         cp_async_wait<kLookahead>();
         fence_proxy_async_smem();
-        mbar_arrive(&full[(s - kLookahead) % kStages]);
+        arrive_stage(s - kLookahead);
       }
     }
     // land everything still in flight (also on the abort path)
     cp_async_wait<0>();
     fence_proxy_async_smem();
     if (ok)
-      for (int r = (s > kLookahead ? s - kLookahead : 0); r < s; ++r) mbar_arrive(&full[r % kStages]);
+      for (int r = (s > kLookahead ? s - kLookahead : 0); r < s; ++r) arrive_stage(r);
+    if (!ok && pt == 0) {
+      // wind down: the Q loads issued for QK stages still pending must land
+      for (int r = (s > kStages ? s - kStages : 0); r < s && r < kQKChunks; ++r)
+        mbar_drain(&full[r % kStages], static_cast<uint32_t>((r / kStages) & 1));
+    }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -226,27 +278,45 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a
     __syncwarp();  // tcgen05.ld is warp-collective
     if (ok) {
       tc_fence_after();
-      float m = -INFINITY;
-#pragma unroll 1
-      for (int c0 = 0; c0 < TS; c0 += 32) {
-        float v[32];
-        tmem_ld32(taddr + c0, v);
+      constexpr int kChunks = TS / 32;  // even: TS is a multiple of 64
+      uint32_t rb0[32], rb1[32];
+      // pass 1: row max over valid tokens. Two register buffers: the load of
+      // chunk c+1 is in flight while chunk c is reduced; four partial maxima
+      // keep the dependency chains short.
+      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      auto max_chunk = [&](const uint32_t (&rv)[32], uint32_t vm) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (idx_s[c0 + j] >= 0) m = fmaxf(m, v[j]);
-      }
-      mx = m * c2;
+        for (int j = 0; j < 32; ++j) {
+          const float x = ((vm >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
+          mp[j & 3] = fmaxf(mp[j & 3], x);
+        }
+      };
+      tmem_ld32_issue(taddr, rb0);
+      tmem_ld_wait(rb0);
 #pragma unroll 1
-      for (int c0 = 0; c0 < TS; c0 += 32) {
-        float v[32];
-        tmem_ld32(taddr + c0, v);
+      for (int c = 0; c < kChunks; c += 2) {
+        tmem_ld32_issue(taddr + (c + 1) * 32, rb1);
+        max_chunk(rb0, vmask[c]);
+        tmem_ld_wait(rb1);
+        if (c + 2 < kChunks) tmem_ld32_issue(taddr + (c + 2) * 32, rb0);
+        max_chunk(rb1, vmask[c + 1]);
+        if (c + 2 < kChunks) tmem_ld_wait(rb0);
+      }
+      const float m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+      mx = m * c2;
+      const float mxe = m == -INFINITY ? 0.f : mx;  // every token invalid: all p = 0
+      // pass 2: P = 2^(z log2e - max) as bf16 into the A-operand layout; row
+      // sum of the rounded values
+      float lp[4] = {0.f, 0.f, 0.f, 0.f};
+      auto p_chunk = [&](const uint32_t (&rv)[32], uint32_t vm, int c0) {
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float p0 = idx_s[c0 + j] >= 0 ? exp2f(fmaf(v[j], c2, -mx)) : 0.f;
-          const float p1 = idx_s[c0 + j + 1] >= 0 ? exp2f(fmaf(v[j + 1], c2, -mx)) : 0.f;
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          l += __low2float(pb) + __high2float(pb);
+          const float x0 = ((vm >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
+          const float x1 = ((vm >> (j + 1)) & 1u) ? __uint_as_float(rv[j + 1]) : -INFINITY;
+          const __nv_bfloat162 pb =
+              __floats2bfloat162_rn(ex2_approx(fmaf(x0, c2, -mxe)), ex2_approx(fmaf(x1, c2, -mxe)));
+          lp[(j >> 1) & 3] += __low2float(pb) + __high2float(pb);
           pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
         }
         const uint32_t blk = smem_u32(ps + (c0 >> 6) * (kHeads * 128));
@@ -255,7 +325,19 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a
         for (int q4 = 0; q4 < 4; ++q4)
           st_shared_v4(blk + sw128_offset(r, ch0 + q4),
                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]));
+      };
+      tmem_ld32_issue(taddr, rb0);
+      tmem_ld_wait(rb0);
+#pragma unroll 1
+      for (int c = 0; c < kChunks; c += 2) {
+        tmem_ld32_issue(taddr + (c + 1) * 32, rb1);
+        p_chunk(rb0, vmask[c], c * 32);
+        tmem_ld_wait(rb1);
+        if (c + 2 < kChunks) tmem_ld32_issue(taddr + (c + 2) * 32, rb0);
+        p_chunk(rb1, vmask[c + 1], (c + 1) * 32);
+        if (c + 2 < kChunks) tmem_ld_wait(rb0);
       }
+      l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(p_ready);
@@ -265,21 +347,50 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const MlaArgs a
     if (ok) {
       tc_fence_after();
       const int64_t row = (static_cast<int64_t>(b) * a.H + head) * a.splits + sp;
-      float* po = a.part_o + row * kDv;
-#pragma unroll 1
-      for (int jh = 0; jh < 2; ++jh) {
-        const uint32_t colbase = jh == 0 ? 256u : 0u;
-#pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
-          float v[32];
-          tmem_ld32(taddr + colbase + c0, v);
-          if (head < a.H) {
-            float4* dst = reinterpret_cast<float4*>(po + jh * 256 + c0);
+      // O / l (0 when no token was valid), transposed through shared memory
+      // in 32-dim chunks (the stage ring is idle once every MMA has retired)
+      // so each warp store writes whole rows segments.
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      uint32_t* tile = reinterpret_cast<uint32_t*>(stages) + quad * (32 * 33);
+      const int64_t row0 = (static_cast<int64_t>(b) * a.H + hb * kHeads + quad * 32) * a.splits + sp;
+      const int nrows = min(32, a.H - (hb * kHeads + quad * 32));
+      const int64_t rstride = static_cast<int64_t>(a.splits) * kDv;  // elements between heads' rows
+      // O_lo sits in TMEM columns [256, 512), O_hi in [0, 256); 16 chunks of 32 dims
+      uint32_t rb0[32], rb1[32];
+      auto col_of = [](int c) { return c < 8 ? 256u + 32u * c : 32u * (c - 8); };
+      auto out_chunk = [&](const uint32_t (&rv)[32], int c) {
+        if (a.out_f32) {
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-          }
+          for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = __float_as_uint(__uint_as_float(rv[j]) * inv_l);
+          __syncwarp();
+          float* dst = static_cast<float*>(a.part_o) + row0 * kDv + c * 32 + lane;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nrows) dst[i * rstride] = __uint_as_float(tile[i * 33 + lane]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            tile[lane * 17 + j] = pack_bf16x2(__uint_as_float(rv[2 * j]) * inv_l, __uint_as_float(rv[2 * j + 1]) * inv_l);
+          __syncwarp();
+          // lanes 0-15 write row i, lanes 16-31 row i+1 (64 bytes each)
+          uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(a.part_o) + row0 * kDv + c * 32);
+          const int half = lane >> 4, w = lane & 15;
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            if (i + half < nrows) dst[(i + half) * (rstride / 2) + w] = tile[(i + half) * 17 + w];
         }
+        __syncwarp();
+      };
+      tmem_ld32_issue(taddr + col_of(0), rb0);
+      tmem_ld_wait(rb0);
+#pragma unroll 1
+      for (int c = 0; c < 16; c += 2) {
+        tmem_ld32_issue(taddr + col_of(c + 1), rb1);
+        out_chunk(rb0, c);
+        tmem_ld_wait(rb1);
+        if (c + 2 < 16) tmem_ld32_issue(taddr + col_of(c + 2), rb0);
+        out_chunk(rb1, c + 1);
+        if (c + 2 < 16) tmem_ld_wait(rb0);
       }
       if (head < a.H) {
         a.part_ml[row * 2 + 0] = mx;
@@ -305,7 +416,7 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
   if (gw >= static_cast<int64_t>(a.B) * a.H) return;
   const int h = static_cast<int>(gw % a.H);
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + gw * a.splits;
-  const float* po = a.part_o + gw * a.splits * kDv;
+  const int64_t pbase = gw * a.splits * kDv;
   const float sink2 = a.sink[h] * kLog2e;
   float M = sink2;
   for (int s = lane; s < a.splits; s += 32) M = fmaxf(M, ml[s].x);
@@ -325,14 +436,21 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
   for (int s = 0; s < a.splits; ++s) {
     const float ms = ml[s].x;
     if (ms == -INFINITY) continue;
-    const float wgt = exp2f(ms - M);
+    const float wgt = exp2f(ms - M) * ml[s].y;  // partials hold O / l
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 o = *reinterpret_cast<const float4*>(po + s * kDv + i * 128 + lane * 4);
-      acc[4 * i] = fmaf(wgt, o.x, acc[4 * i]);
-      acc[4 * i + 1] = fmaf(wgt, o.y, acc[4 * i + 1]);
-      acc[4 * i + 2] = fmaf(wgt, o.z, acc[4 * i + 2]);
-      acc[4 * i + 3] = fmaf(wgt, o.w, acc[4 * i + 3]);
+      float o[4];
+      if (a.out_f32) {
+        const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.part_o) + pbase + s * kDv + i * 128 + lane * 4);
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.part_o) + pbase + s * kDv + i * 128 + lane * 4);
+        const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+        const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+        o[0] = __low2float(v01); o[1] = __high2float(v01); o[2] = __low2float(v23); o[3] = __high2float(v23);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[4 * i + e] = fmaf(wgt, o[e], acc[4 * i + e]);
     }
   }
   const float inv = 1.f / den;
@@ -363,14 +481,14 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
 }
 
 template <int TS>
-cudaError_t launch_ts(const MlaArgs& a, cudaStream_t stream) {
+cudaError_t launch_ts(const CUtensorMap& qmap, const MlaArgs& a, cudaStream_t stream) {
   using C = MlaCfg<TS>;
   auto kern = sparse_mla_kernel<TS>;
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.B, (a.H + kHeads - 1) / kHeads);
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(a);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(qmap, a);
   return cudaGetLastError();
 }
 
@@ -384,12 +502,12 @@ int mla_smem_bytes(int ts) {
   }
 }
 
-cudaError_t launch_sparse_mla(const MlaArgs& a, cudaStream_t stream, int* launches) {
+cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const MlaArgs& a, cudaStream_t stream, int* launches) {
   cudaError_t e;
   switch (a.ts) {
-    case 64: e = launch_ts<64>(a, stream); break;
-    case 128: e = launch_ts<128>(a, stream); break;
-    case 256: e = launch_ts<256>(a, stream); break;
+    case 64: e = launch_ts<64>(qmap, a, stream); break;
+    case 128: e = launch_ts<128>(qmap, a, stream); break;
+    case 256: e = launch_ts<256>(qmap, a, stream); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

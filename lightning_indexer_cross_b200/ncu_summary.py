@@ -1,5 +1,5 @@
 """Summarise an ncu launch list (gpu__time_duration.sum CSV) per kernel:
-launches, total time, mean, share. Usage: python profiles/summarize_launches.py launches.csv"""
+launches, total time, mean, share. Usage: python -m lightning_indexer_cross_b200.ncu_summary launches.csv"""
 import collections
 import csv
 import sys
