@@ -1,0 +1,114 @@
+"""Parity at the five workloads' full sizes, through the same C-ABI calls the
+benchmark makes (ic_layer_stack). The oracle checks sampled queries and
+layers one by one; properties that hold at any size (S-layer byte identity,
+planted-token recovery, index range and uniqueness) are checked everywhere.
+Every test here needs a B200 and a few GB of device memory."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from lightning_indexer_cross_b200 import workloads as W
+from tests._helpers import ATTN_TOL, attn_row_error, index_sets_match
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from lightning_indexer_cross_b200 import ops
+    return ops
+
+
+def _run(wl, out_dtype=torch.bfloat16):
+    st = _ops().stack_from_workload(wl, trace=True, out_dtype=out_dtype)
+    st.step()
+    torch.cuda.synchronize()
+    assert st.device_status() == 0
+    return st
+
+
+def _check_layer(wl, st, l, rows):
+    """Oracle indexer + top-k for `rows` of the layer governing l, and oracle
+    attention of layer l on the GPU's own index set (reported with the
+    oracle's own set too)."""
+    gov = oracle.governing_full_layer(wl.schedule)[l]
+    f = wl.layers[gov]
+    lay = wl.layers[l]
+    trace = st.trace[l].cpu().numpy()
+    nv = None if wl.n_valid is None else wl.n_valid[rows]
+    kk = f.k_idx if f.k_idx.shape[0] == 1 else f.k_idx[rows]
+    ks = None if f.k_scale is None else (f.k_scale if f.k_scale.shape[0] == 1 else f.k_scale[rows])
+    sc = oracle.indexer_scores(f.q_idx[rows], f.w[rows], kk, ks, nv, keys_are_e4m3=wl.k_fp8)
+    ref_idx = oracle.topk_indices(sc, wl.topk, nv)
+    ok, msg = index_sets_match(trace[rows], ref_idx, sc, wl.topk, nv)
+    assert ok, f"layer {gov}: {msg}"
+    # gather only the selected rows before handing them to the float64 oracle
+    # (a whole 1M-token cache would not fit in host memory as float64)
+    idx = torch.as_tensor(trace[rows], device=lay.kv.device, dtype=torch.int64)
+    cache = lay.kv[0] if lay.kv.shape[0] == 1 else None
+    sel = []
+    for i, b in enumerate(rows):
+        src = cache if cache is not None else lay.kv[b]
+        sel.append(src[idx[i].clamp_min(0)])
+    kv_sel = torch.stack(sel)                               # [R, k, 576]
+    idx_sel = torch.where(idx >= 0, torch.arange(idx.shape[1], device=idx.device), -1)
+    gate = None if lay.gate is None else lay.gate[rows]
+    ref, _ = oracle.sparse_mla(lay.q[rows], kv_sel, idx_sel, lay.sink, gate, wl.sm_scale)
+    err = attn_row_error(st.outs[l][rows], ref)
+    assert err <= ATTN_TOL[st.outs[l].dtype], f"layer {l}: attention row error {err:.3e}"
+
+
+def _check_indices_valid(wl, st):
+    tr = st.trace
+    nv = torch.full((wl.B,), wl.N, device=tr.device) if wl.n_valid is None else wl.n_valid
+    assert bool(((tr >= -1) & (tr < nv.view(1, -1, 1))).all())
+    srt = tr.sort(dim=2).values
+    dup = (srt[:, :, 1:] == srt[:, :, :-1]) & (srt[:, :, 1:] >= 0)
+    assert not bool(dup.any())
+
+
+def test_single_f_layer_model_shape(cuda_dev):
+    """N=131072, 8 queries with their own caches, 64x128 indexer, k=2048,
+    128 heads, gate: every query checked."""
+    wl = W.single_f(cuda_dev)
+    st = _run(wl)
+    _check_indices_valid(wl, st)
+    _check_layer(wl, st, 0, list(range(wl.B)))
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_long_context_1m(cuda_dev, fp8):
+    """N=1,048,576, 4 queries with their own caches, bf16 and e4m3 keys:
+    planted tokens recovered for every query, full oracle check of query 0."""
+    wl = W.long_context(cuda_dev, fp8=fp8)
+    st = _run(wl)
+    _check_indices_valid(wl, st)
+    for b in range(wl.B):
+        assert set(wl.planted[b].tolist()) <= set(st.trace[0, b].tolist())
+    _check_layer(wl, st, 0, [0])
+
+
+def test_prefill_chunk_causal(cuda_dev):
+    """2048 causal queries over 264192 tokens: sampled rows against the oracle."""
+    wl = W.prefill(cuda_dev)
+    st = _run(wl)
+    _check_indices_valid(wl, st)
+    rows = [0, 1, 777, 1500, 2046, 2047]
+    _check_layer(wl, st, 0, rows)
+
+
+def test_stack78_decode(cuda_dev):
+    """The 78-layer F/S stack the benchmark runs (B=32, N=131072): every S
+    layer byte-identical to its governing F layer; sampled F layers and
+    queries against the oracle; attention on sampled S layers."""
+    wl = W.stack(cuda_dev)
+    st = _run(wl)
+    _check_indices_valid(wl, st)
+    gov = oracle.governing_full_layer(wl.schedule)
+    tr = st.trace.cpu().numpy()
+    for l in range(wl.L):
+        assert tr[l].tobytes() == tr[gov[l]].tobytes(), f"layer {l}"
+    f_layers = [l for l in range(wl.L) if wl.schedule[l] == "F"]
+    s_layers = [l for l in range(wl.L) if wl.schedule[l] == "S"]
+    for l in (f_layers[0], f_layers[len(f_layers) // 2], f_layers[-1], s_layers[0], s_layers[-1]):
+        _check_layer(wl, st, l, [0, 31])
