@@ -106,12 +106,13 @@ size_t ic_topk_workspace_size(int B, int64_t N, int k);
  * The pages have no counterpart: this is an interface choice of the library.
  *
  * Same result and limits as ic_topk, but takes no workspace: its scratch is
- * a fixed array inside the library (about 1.6 MB on every GPU that loads
- * it, held until exit). Meant for code that cannot call cudaMalloc, e.g.
+ * a fixed array inside the library (4 MB on every GPU that loads it, held
+ * until exit). Meant for code that cannot call cudaMalloc, e.g.
  * enqueueing inside a CUDA-graph capture that forbids allocation, or engine
  * plugins that only receive their input and output buffers.
- *   - At most IC_TOPK_NOALLOC_MAX_ROWS rows; more returns IC_ERR_UNSUPPORTED
- *     with nothing launched.
+ *   - At most IC_TOPK_NOALLOC_MAX_ROWS rows, and the per-row histograms and
+ *     candidate buffers must fit the array (64 rows of up to 131072 scores
+ *     do); otherwise IC_ERR_UNSUPPORTED with nothing launched.
  *   - All calls share the one array; calls that overlap on the GPU race.
  *   - The first call on a device looks up the array's address; make it
  *     before any stream capture. Device-side status is not reported.

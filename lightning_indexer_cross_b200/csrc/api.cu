@@ -128,8 +128,8 @@ namespace ic {
 // ------------------------------------------------------------------ top-k
 TopkLayout topk_layout(int B, int64_t N) {
   TopkLayout L{};
-  // about four 512-thread CTAs per SM in total, and at least 4096 scores per CTA
-  const int64_t target = std::max<int64_t>(1, 4 * num_sms() / std::max(B, 1));
+  // one wave: two 512-thread CTAs per SM in total, at least 4096 scores per CTA
+  const int64_t target = std::max<int64_t>(1, 2 * num_sms() / std::max(B, 1));
   int64_t cpr = std::min<int64_t>(ceil_div<int64_t>(N, 4096), target);
   cpr = std::max<int64_t>(cpr, 1);
   int64_t slice = ceil_div<int64_t>(N, cpr);
@@ -137,10 +137,14 @@ TopkLayout topk_layout(int B, int64_t N) {
   cpr = ceil_div<int64_t>(N, slice);
   L.cpr = static_cast<int>(cpr);
   L.slice = slice;
+  // the k-th key's 1/16-octave bin rarely holds more than a few percent of a
+  // row; bigger bins fall back to passes over the row itself
+  L.cand_cap = static_cast<int>(std::min<int64_t>(N, std::max<int64_t>(4096, N / 16)));
+  // histograms and control words first, so one memset clears both
   L.hist_off = 0;
-  L.tie_off = align256(L.hist_off + size_t(3) * B * 2048 * 4);
-  L.cnt_off = align256(L.tie_off + size_t(B) * L.cpr * 4);
-  L.total = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
+  L.cnt_off = align256(L.hist_off + size_t(B) * 4096 * 4);
+  L.cand_off = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
+  L.total = align256(L.cand_off + size_t(B) * L.cand_cap * 4);
   return L;
 }
 
@@ -151,14 +155,15 @@ ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_va
   if (!aligned16(scores) || !aligned16(idx)) return IC_ERR_INVALID_ARG;
   TopkLayout L = topk_layout(B, N);
   if (ws_bytes < L.total) return IC_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(ws, 0, L.total, stream) != cudaSuccess) return IC_ERR_CUDA;
+  if (cudaMemsetAsync(ws + L.hist_off, 0, L.cand_off - L.hist_off, stream) != cudaSuccess) return IC_ERR_CUDA;
   ic::TopkArgs a{};
   a.scores = scores;
   a.n_valid = n_valid;
   a.idx = idx;
   a.hist = reinterpret_cast<uint32_t*>(ws + L.hist_off);
-  a.tie_counts = reinterpret_cast<uint32_t*>(ws + L.tie_off);
+  a.cand = reinterpret_cast<int32_t*>(ws + L.cand_off);
   a.counters = reinterpret_cast<uint32_t*>(ws + L.cnt_off);
+  a.cand_cap = L.cand_cap;
   a.status = status;
   a.B = B;
   a.N = N;

@@ -55,8 +55,8 @@ struct TopkArgs {
   const float* scores;      // [B, N]
   const int64_t* n_valid;   // [B] or null
   int32_t* idx;             // [B, k]
-  uint32_t* hist;           // [3][B][2048]
-  uint32_t* tie_counts;     // [B][cpr]
+  uint32_t* hist;           // [B][4096] histogram of the top 12 key bits
+  int32_t* cand;            // [B][cand_cap] candidate positions (the k-th key's bin)
   uint32_t* counters;       // [B][kCtrlWords] per-row control state
   int* status;
   int B;
@@ -64,6 +64,7 @@ struct TopkArgs {
   int k;
   int cpr;                  // CTAs per row
   int64_t slice;            // elements per CTA slice
+  int cand_cap;             // candidate buffer entries per row
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches);
 
@@ -72,7 +73,8 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches);
 struct TopkLayout {
   int cpr;
   int64_t slice;
-  size_t hist_off, tie_off, cnt_off, total;
+  int cand_cap;
+  size_t hist_off, cand_off, cnt_off, total;
 };
 TopkLayout topk_layout(int B, int64_t N);
 // Validate, clear the scratch region and enqueue the top-k passes.

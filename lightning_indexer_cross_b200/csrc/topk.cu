@@ -2,20 +2,22 @@
 // "Top-k selection": keep the k highest-scoring cached tokens).
 //
 // Radix select on the order-preserving 32-bit key of each fp32 score
-// (negative floats: all bits flipped; others: sign bit set), in digits of
-// 11, 11 and 10 bits, most significant first. Each row is split across
-// `cpr` CTAs; every pass is its own launch, so no CTA ever waits on another:
-//   pass 1  histogram of key[31:21] over the row's valid positions
-//   pass 2  histogram of key[20:10] over keys whose top digit is the k-th's
-//   pass 3  histogram of key[9:0]  over keys whose top 22 bits match
-//   emit    keys > T (T = the exact k-th key) are compacted per CTA in
-//           shared memory and written with one atomic reservation per CTA;
-//           the last CTA of the row (atomic ticket) writes the r lowest-index
-//           keys equal to T, so ties resolve toward the lower index and the
-//           selected set is deterministic.
-// After each histogram pass the last CTA of the row (atomic ticket) turns the
-// row's global histogram into the chosen digit and the remaining rank, kept
-// in a per-row state word that the next pass reads once.
+// (negative floats: all bits flipped; others: sign bit set). Two launches,
+// neither of which ever waits on another CTA:
+//   histogram  a 12-bit histogram of key[31:20] over each row's valid
+//              positions (several CTAs per row, merged with atomics).
+//   filter     every CTA finds the bin d1 holding the k-th key from the
+//              row's histogram; keys in bins above d1 are final and are
+//              written straight to the output (compacted per CTA, one atomic
+//              reservation per CTA); keys in bin d1 are candidates, appended
+//              to a per-row buffer. The last CTA of the row (atomic ticket)
+//              resolves the exact k-th key T among the candidates (two more
+//              10-bit digits), writes the candidates above T, and then the
+//              r keys equal to T with the lowest indices -- ties resolve
+//              toward the lower index, so the selected set is deterministic.
+// If bin d1 holds more candidates than the buffer, the last CTA runs the same
+// two digits over the row itself (correct, slower; only for rows whose scores
+// crowd into one 1/16-octave bin).
 // Rows with n_valid <= k take every valid index and pad with -1.
 #include "common.cuh"
 #include "kernels.h"
@@ -26,16 +28,22 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 2048;
+constexpr int kBins1 = 4096;      // first digit: key[31:20]
+constexpr int kBins2 = 1024;      // second and third digits: key[19:10], key[9:0]
 constexpr int kUnroll = 4;        // float4 loads in flight per lane
-constexpr int kLocalCap = 4096;   // per-CTA shared buffer of selected indices
+constexpr int kLocalCap = 2048;   // per-CTA shared buffer of indices (each list)
+constexpr int kTieCap = 2048;     // ties resolved in shared memory up to this many
+constexpr int kRegCand = 16;      // candidates per thread held in registers by the last CTA
 
 // per-row control block (kCtrlWords 32-bit words, one 128-byte line per row)
 enum : int {
-  kAboveCount = 0,  // emitted keys > T
-  kTicket0 = 1,     // tickets of pass 1..3 and emit: kTicket0 + p
-  kPrefix = 8,      // digits chosen so far (key bits above the current digit)
-  kRank = 9,        // remaining rank within the keys matching the prefix
+  kAboveCount = 0,  // keys written above bin d1
+  kCandCount = 1,   // candidates appended (may exceed the capacity)
+  kTicket = 2,      // CTAs of the filter pass finished
+  kHistTicket = 3,  // CTAs of the histogram pass finished
+  kBin = 4,         // d1: the first-digit bin of the k-th key
+  kBinRank = 5,     // rank of the k-th key inside bin d1
+  kBinCount = 6,    // keys in bin d1 over the whole row
 };
 
 IC_DEV uint32_t score_key(float f) {
@@ -89,7 +97,7 @@ IC_DEV void select_digit(const uint32_t* counts, int nbins, uint32_t kr, int* d_
   __syncthreads();
 }
 
-// Visit this CTA's slice of row b: f(i, key, valid) for every position, in
+// Visit positions [lo, hi) of row b: f(i, key, valid) for every position, in
 // warp-uniform steps (all 32 lanes call f together), with kUnroll
 // independent 16-byte loads in flight per lane.
 template <typename F>
@@ -139,69 +147,166 @@ IC_DEV void for_slice(const TopkArgs& a, int b, int64_t lo, int64_t hi, F&& f) {
   }
 }
 
-// Warp-aggregated shared-memory histogram increment; all 32 lanes call.
+// Shared-memory histogram increment (native shared atomics; measured faster
+// on B200 than grouping equal bins with __match_any_sync first).
 IC_DEV void hist_add(uint32_t* h, uint32_t bin, bool take) {
-  if (__ballot_sync(0xffffffffu, take) == 0u) return;  // common in passes 2 and 3
-  const uint32_t b = take ? bin : 0xFFFFFFFFu;
-  const uint32_t peers = __match_any_sync(0xffffffffu, b);
-  const int leader = __ffs(peers) - 1;
-  if (take && (threadIdx.x & 31) == leader) atomicAdd(&h[bin], __popc(peers));
+  if (take) atomicAdd(&h[bin], 1u);
 }
 
-template <int PASS>
+// Append i to a shared list when `take` (warp-aggregated; all 32 lanes call).
+// Entries past `cap` are not stored but still counted.
+IC_DEV void list_push(int32_t* list, uint32_t* count, uint32_t cap, int64_t i, bool take) {
+  const uint32_t bal = __ballot_sync(0xffffffffu, take);
+  if (!bal) return;
+  const int lane = threadIdx.x & 31;
+  uint32_t base = 0;
+  if (lane == 0) base = atomicAdd(count, static_cast<uint32_t>(__popc(bal)));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  if (take) {
+    const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
+    if (pos < cap) list[pos] = static_cast<int32_t>(i);
+  }
+}
+
+// ------------------------------------------------------------------ pass 1
 __global__ void __launch_bounds__(kThreads) topk_hist_kernel(const TopkArgs a) {
-  __shared__ uint32_t sh_hist[kBins];
+  __shared__ uint32_t sh_hist[kBins1];
   __shared__ uint32_t warp_tot[kWarps];
   __shared__ int sh_d;
   __shared__ uint32_t sh_kr;
   __shared__ int sh_last;
   const int b = blockIdx.y, c = blockIdx.x;
   const int64_t nv = row_valid(a, b);
-  if (nv <= a.k) return;  // the emit pass takes every valid index
-  uint32_t* ctrl = row_ctrl(a, b);
+  if (nv <= a.k) return;  // the filter pass takes every valid index
   const int64_t lo = static_cast<int64_t>(c) * a.slice;
   const int64_t hi = lo + a.slice < nv ? lo + a.slice : nv;
-  const uint32_t prefix = PASS > 1 ? __ldcg(&ctrl[kPrefix]) : 0u;
-  const uint32_t kr = PASS > 1 ? __ldcg(&ctrl[kRank]) : static_cast<uint32_t>(a.k);
-  for (int j = threadIdx.x; j < kBins; j += kThreads) sh_hist[j] = 0;
+  for (int j = threadIdx.x; j < kBins1; j += kThreads) sh_hist[j] = 0;
   __syncthreads();
-  if (lo < hi) {
-    for_slice(a, b, lo, hi, [&](int64_t, uint32_t key, bool valid) {
-      if (PASS == 1) hist_add(sh_hist, key >> 21, valid);
-      if (PASS == 2) hist_add(sh_hist, (key >> 10) & 0x7FFu, valid && (key >> 21) == prefix);
-      if (PASS == 3) hist_add(sh_hist, key & 0x3FFu, valid && (key >> 10) == prefix);
-    });
-  }
+  if (lo < hi)
+    for_slice(a, b, lo, hi, [&](int64_t, uint32_t key, bool valid) { hist_add(sh_hist, key >> 20, valid); });
   __syncthreads();
-  uint32_t* g = a.hist + (static_cast<int64_t>(PASS - 1) * a.B + b) * kBins;
-  for (int j = threadIdx.x; j < kBins; j += kThreads)
+  uint32_t* g = a.hist + static_cast<int64_t>(b) * kBins1;
+  for (int j = threadIdx.x; j < kBins1; j += kThreads)
     if (sh_hist[j]) atomicAdd(g + j, sh_hist[j]);
-  // last CTA of the row: choose this pass's digit once for everyone
+  // the last CTA of the row picks the bin of the k-th key once for everyone
+  uint32_t* ctrl = row_ctrl(a, b);
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) sh_last = atomicAdd(&ctrl[kTicket0 + PASS - 1], 1u) == static_cast<uint32_t>(a.cpr) - 1;
+  if (threadIdx.x == 0) sh_last = atomicAdd(&ctrl[kHistTicket], 1u) == static_cast<uint32_t>(a.cpr) - 1;
   __syncthreads();
   if (!sh_last) return;
   __threadfence();
-  const int nb = PASS == 3 ? 1024 : kBins;
-  for (int j = threadIdx.x; j < nb; j += kThreads) sh_hist[j] = __ldcg(g + j);
+  for (int j = threadIdx.x; j < kBins1; j += kThreads) sh_hist[j] = __ldcg(g + j);
   __syncthreads();
-  select_digit(sh_hist, nb, kr, &sh_d, &sh_kr, warp_tot);
+  select_digit(sh_hist, kBins1, static_cast<uint32_t>(a.k), &sh_d, &sh_kr, warp_tot);
   if (threadIdx.x == 0) {
-    const int shift = PASS == 3 ? 10 : 11;
-    ctrl[kPrefix] = (prefix << shift) | static_cast<uint32_t>(sh_d);
-    ctrl[kRank] = sh_kr;
+    ctrl[kBin] = static_cast<uint32_t>(sh_d);
+    ctrl[kBinRank] = sh_kr;
+    ctrl[kBinCount] = sh_hist[sh_d];
   }
 }
 
-__global__ void __launch_bounds__(kThreads) topk_emit_kernel(const TopkArgs a) {
-  __shared__ int32_t sh_sel[kLocalCap];
-  __shared__ uint32_t sh_n;
-  __shared__ uint32_t sh_base;
-  __shared__ uint32_t warp_cnt[kWarps];
-  __shared__ int sh_last;
+// ------------------------------------------------------------------ pass 2
+struct FilterShared {
+  uint32_t hist[kBins1];
+  int32_t above[kLocalCap];
+  int32_t cand[kLocalCap];
+  uint32_t warp_tot[kWarps];
+  uint32_t n_above, n_cand, base_above, base_cand;
+  int d;
+  uint32_t kr;
+  int last;
+};
+
+// Exact resolution of the k-th key within bin d1 by the last CTA of the row.
+// `visit(f)` enumerates (index, key, valid) for a superset of the keys of bin
+// d1 (the candidate buffer, or the whole row when the buffer overflowed).
+template <typename Visit>
+IC_DEV void resolve_bin(const TopkArgs& a, int b, int64_t nv, uint32_t d1, uint32_t kr1, uint32_t n_above,
+                        FilterShared& sh, Visit&& visit) {
+  int32_t* out = a.idx + static_cast<int64_t>(b) * a.k;
+  uint32_t* h = sh.hist;
+  // digit 2: key[19:10]
+  for (int j = threadIdx.x; j < kBins2; j += kThreads) h[j] = 0;
+  __syncthreads();
+  visit([&](int64_t, uint32_t key, bool ok) { hist_add(h, (key >> 10) & 0x3FFu, ok && (key >> 20) == d1); });
+  __syncthreads();
+  select_digit(h, kBins2, kr1, &sh.d, &sh.kr, sh.warp_tot);
+  const uint32_t p2 = (d1 << 10) | static_cast<uint32_t>(sh.d);
+  const uint32_t kr2 = sh.kr;
+  __syncthreads();
+  // digit 3: key[9:0]
+  for (int j = threadIdx.x; j < kBins2; j += kThreads) h[j] = 0;
+  __syncthreads();
+  visit([&](int64_t, uint32_t key, bool ok) { hist_add(h, key & 0x3FFu, ok && (key >> 10) == p2); });
+  __syncthreads();
+  select_digit(h, kBins2, kr2, &sh.d, &sh.kr, sh.warp_tot);
+  const uint32_t T = (p2 << 10) | static_cast<uint32_t>(sh.d);
+  const uint32_t r = sh.kr;                      // keys equal to T to take (>= 1)
+  const uint32_t n_ties = h[sh.d];               // keys equal to T
+  const uint32_t n_hi = kr1 - r;                 // keys of bin d1 above T
+  __syncthreads();
+  // keys of bin d1 above T
+  if (threadIdx.x == 0) sh.n_above = 0;
+  __syncthreads();
+  visit([&](int64_t i, uint32_t key, bool ok) {
+    const bool take = ok && (key >> 20) == d1 && key > T;
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    if (!bal) return;
+    const int lane = threadIdx.x & 31;
+    uint32_t base = 0;
+    if (lane == 0) base = atomicAdd(&sh.n_above, static_cast<uint32_t>(__popc(bal)));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (take) {
+      const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
+      if (pos < n_hi) out[n_above + pos] = static_cast<int32_t>(i);
+      else record_status(a.status, IC_ERR_BAD_INDEX);  // cannot happen with consistent counts
+    }
+  });
+  __syncthreads();
+  // the r lowest-index keys equal to T
+  int32_t* tie_out = out + (a.k - r);
+  if (n_ties <= static_cast<uint32_t>(kTieCap)) {
+    if (threadIdx.x == 0) sh.n_cand = 0;
+    __syncthreads();
+    visit([&](int64_t i, uint32_t key, bool ok) { list_push(sh.cand, &sh.n_cand, kTieCap, i, ok && key == T); });
+    __syncthreads();
+    const uint32_t n = sh.n_cand;
+    for (uint32_t x = threadIdx.x; x < n; x += kThreads) {
+      const int32_t me = sh.cand[x];
+      uint32_t rank = 0;  // ties with a lower index
+      for (uint32_t y = 0; y < n; ++y) rank += sh.cand[y] < me;
+      if (rank < r) tie_out[rank] = me;
+    }
+  } else {
+    // many exact ties: scan the row in index order
+    const float* row = a.scores + static_cast<int64_t>(b) * a.N;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t taken = 0;
+    for (int64_t base = 0; base < nv && taken < r; base += kThreads) {
+      const int64_t i = base + threadIdx.x;
+      const bool tie = (i < nv) && score_key(__ldcg(row + i)) == T;
+      const uint32_t bal = __ballot_sync(0xffffffffu, tie);
+      if (lane == 0) sh.warp_tot[warp] = __popc(bal);
+      __syncthreads();
+      uint32_t before = 0, total = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        if (w < warp) before += sh.warp_tot[w];
+        total += sh.warp_tot[w];
+      }
+      const uint32_t pos = taken + before + __popc(bal & ((1u << lane) - 1u));
+      if (tie && pos < r) tie_out[pos] = static_cast<int32_t>(i);
+      taken += total;
+      __syncthreads();
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  FilterShared& sh = *reinterpret_cast<FilterShared*>(smem_raw);
   const int b = blockIdx.y, c = blockIdx.x;
-  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int t = threadIdx.x;
   int32_t* out = a.idx + static_cast<int64_t>(b) * a.k;
   const int64_t nv = row_valid(a, b);
   if (nv <= a.k) {
@@ -210,97 +315,150 @@ __global__ void __launch_bounds__(kThreads) topk_emit_kernel(const TopkArgs a) {
     return;
   }
   uint32_t* ctrl = row_ctrl(a, b);
-  const uint32_t T = __ldcg(&ctrl[kPrefix]);  // the exact k-th key
-  const uint32_t r = __ldcg(&ctrl[kRank]);    // keys equal to T to take, >= 1
-  const uint32_t n_above = static_cast<uint32_t>(a.k) - r;
-  if (t == 0) sh_n = 0;
+  // the bin of the k-th key, chosen by the histogram pass
+  const uint32_t d1 = __ldcg(&ctrl[kBin]);
+  const uint32_t kr1 = __ldcg(&ctrl[kBinRank]);        // rank of the k-th key inside bin d1
+  const uint32_t n_cand_row = __ldcg(&ctrl[kBinCount]); // keys in bin d1 (whole row)
+  const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
+  if (t == 0) {
+    sh.n_above = 0;
+    sh.n_cand = 0;
+  }
   __syncthreads();
 
   const int64_t lo = static_cast<int64_t>(c) * a.slice;
   const int64_t hi = lo + a.slice < nv ? lo + a.slice : nv;
-  uint32_t my_ties = 0;
   if (lo < hi) {
     for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
-      const bool above = valid && key > T;
-      const uint32_t bal = __ballot_sync(0xffffffffu, above);
-      if (bal) {
-        uint32_t base = 0;
-        if (lane == 0) base = atomicAdd(&sh_n, static_cast<uint32_t>(__popc(bal)));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (above) {
-          const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
-          if (pos < kLocalCap) {
-            sh_sel[pos] = static_cast<int32_t>(i);
-          } else {  // shared buffer full: reserve globally, one at a time
-            const uint32_t gp = atomicAdd(&ctrl[kAboveCount], 1u);
-            if (gp < n_above) out[gp] = static_cast<int32_t>(i);
-            else record_status(a.status, IC_ERR_BAD_INDEX);
-          }
-        }
-      }
-      if (valid && key == T) ++my_ties;
+      const uint32_t bin = key >> 20;
+      // a few percent of the keys reach bin d1: one vote skips the rest
+      if (__ballot_sync(0xffffffffu, valid && bin >= d1) == 0u) return;
+      list_push(sh.above, &sh.n_above, kLocalCap, i, valid && bin > d1);
+      list_push(sh.cand, &sh.n_cand, kLocalCap, i, valid && bin == d1);
     });
   }
   __syncthreads();
-  const uint32_t n_local = sh_n < kLocalCap ? sh_n : kLocalCap;
-  if (t == 0) sh_base = n_local ? atomicAdd(&ctrl[kAboveCount], n_local) : 0u;
-  __syncthreads();
-  for (uint32_t j = t; j < n_local; j += kThreads) {
-    const uint32_t gp = sh_base + j;
-    if (gp < n_above) out[gp] = sh_sel[j];
-    else record_status(a.status, IC_ERR_BAD_INDEX);  // cannot happen with consistent histograms
-  }
-  // CTA total of ties
-#pragma unroll
-  for (int off = 16; off; off >>= 1) my_ties += __shfl_down_sync(0xffffffffu, my_ties, off);
-  if (lane == 0) warp_cnt[warp] = my_ties;
-  __syncthreads();
+  // flush: one reservation per list per CTA; if a shared list overflowed,
+  // the slice is scanned again and written through the reserved ranges
+  const uint32_t na = sh.n_above, nc = sh.n_cand;
   if (t == 0) {
-    uint32_t tot = 0;
-    for (int w = 0; w < kWarps; ++w) tot += warp_cnt[w];
-    a.tie_counts[static_cast<int64_t>(b) * a.cpr + c] = tot;
-    __threadfence();
-    sh_last = atomicAdd(&ctrl[kTicket0 + 3], 1u) == static_cast<uint32_t>(a.cpr) - 1;
+    sh.base_above = na ? atomicAdd(&ctrl[kAboveCount], na) : 0u;
+    sh.base_cand = nc ? atomicAdd(&ctrl[kCandCount], nc) : 0u;
   }
   __syncthreads();
-  if (!sh_last) return;
-  __threadfence();
-
-  // Last CTA of the row: the r lowest-index ties, slice by slice in order.
-  uint32_t taken = 0;
-  const float* row = a.scores + static_cast<int64_t>(b) * a.N;
-  for (int j = 0; j < a.cpr && taken < r; ++j) {
-    const uint32_t cnt = __ldcg(&a.tie_counts[static_cast<int64_t>(b) * a.cpr + j]);
-    if (cnt == 0) continue;
-    const int64_t slo = static_cast<int64_t>(j) * a.slice;
-    const int64_t shi = slo + a.slice < nv ? slo + a.slice : nv;
-    for (int64_t base = slo; base < shi && taken < r; base += kThreads) {
-      const int64_t i = base + t;
-      const bool tie = (i < shi) && score_key(__ldcg(row + i)) == T;
-      const uint32_t bal = __ballot_sync(0xffffffffu, tie);
-      if (lane == 0) warp_cnt[warp] = __popc(bal);
-      __syncthreads();
-      uint32_t before = 0;
-      for (int w = 0; w < warp; ++w) before += warp_cnt[w];
-      uint32_t total = 0;
-      for (int w = 0; w < kWarps; ++w) total += warp_cnt[w];
-      const uint32_t pos = taken + before + __popc(bal & ((1u << lane) - 1u));
-      if (tie && pos < r) out[n_above + pos] = static_cast<int32_t>(i);
-      taken += total;
-      __syncthreads();
+  int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
+  if (na <= static_cast<uint32_t>(kLocalCap) && nc <= static_cast<uint32_t>(kLocalCap)) {
+    for (uint32_t j = t; j < na; j += kThreads) {
+      const uint32_t gp = sh.base_above + j;
+      if (gp < n_above) out[gp] = sh.above[j];
+      else record_status(a.status, IC_ERR_BAD_INDEX);
     }
+    for (uint32_t j = t; j < nc; j += kThreads) {
+      const uint32_t gp = sh.base_cand + j;
+      if (gp < static_cast<uint32_t>(a.cand_cap)) cbuf[gp] = sh.cand[j];
+    }
+  } else {
+    __syncthreads();
+    if (t == 0) {
+      sh.n_above = 0;
+      sh.n_cand = 0;
+    }
+    __syncthreads();
+    for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
+      const uint32_t bin = key >> 20;
+      const bool ta = valid && bin > d1, tc = valid && bin == d1;
+      const int lane = threadIdx.x & 31;
+      const uint32_t ba = __ballot_sync(0xffffffffu, ta), bc = __ballot_sync(0xffffffffu, tc);
+      uint32_t oa = 0, oc = 0;
+      if (lane == 0) {
+        if (ba) oa = atomicAdd(&sh.n_above, static_cast<uint32_t>(__popc(ba)));
+        if (bc) oc = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bc)));
+      }
+      oa = __shfl_sync(0xffffffffu, oa, 0);
+      oc = __shfl_sync(0xffffffffu, oc, 0);
+      const uint32_t lt = (1u << lane) - 1u;
+      if (ta) {
+        const uint32_t gp = sh.base_above + oa + __popc(ba & lt);
+        if (gp < n_above) out[gp] = static_cast<int32_t>(i);
+        else record_status(a.status, IC_ERR_BAD_INDEX);
+      }
+      if (tc) {
+        const uint32_t gp = sh.base_cand + oc + __popc(bc & lt);
+        if (gp < static_cast<uint32_t>(a.cand_cap)) cbuf[gp] = static_cast<int32_t>(i);
+      }
+    });
+  }
+  // the last CTA of the row resolves bin d1
+  __threadfence();
+  __syncthreads();
+  if (t == 0) sh.last = atomicAdd(&ctrl[kTicket], 1u) == static_cast<uint32_t>(a.cpr) - 1;
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();
+  const float* row = a.scores + static_cast<int64_t>(b) * a.N;
+  if (n_cand_row <= static_cast<uint32_t>(kRegCand * kThreads) &&
+      n_cand_row <= static_cast<uint32_t>(a.cand_cap)) {
+    // up to kRegCand candidates per thread, fetched once into registers
+    // (keys re-read from the score row); every digit pass then runs on them
+    const uint32_t n = n_cand_row;
+    int32_t ci[kRegCand];
+    uint32_t ck[kRegCand];
+#pragma unroll
+    for (int u = 0; u < kRegCand; ++u) {
+      const uint32_t x = static_cast<uint32_t>(u) * kThreads + t;
+      ci[u] = x < n ? __ldcg(cbuf + x) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < kRegCand; ++u) {
+      const uint32_t x = static_cast<uint32_t>(u) * kThreads + t;
+      ck[u] = x < n ? score_key(__ldcg(row + ci[u])) : 0u;
+    }
+    resolve_bin(a, b, nv, d1, kr1, n_above, sh, [&](auto&& f) {
+#pragma unroll
+      for (int u = 0; u < kRegCand; ++u) {
+        const uint32_t x = static_cast<uint32_t>(u) * kThreads + t;
+        f(static_cast<int64_t>(ci[u]), ck[u], x < n);
+      }
+    });
+  } else if (n_cand_row <= static_cast<uint32_t>(a.cand_cap)) {
+    // a larger bin: batches of 8 candidates per thread per round trip
+    const uint32_t n = n_cand_row;
+    resolve_bin(a, b, nv, d1, kr1, n_above, sh, [&](auto&& f) {
+      for (uint32_t base = 0; base < n; base += 8 * kThreads) {  // warp-uniform bound
+        int32_t bi[8];
+        uint32_t bk[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t x = base + static_cast<uint32_t>(u) * kThreads + t;
+          bi[u] = x < n ? __ldcg(cbuf + x) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t x = base + static_cast<uint32_t>(u) * kThreads + t;
+          bk[u] = x < n ? score_key(__ldcg(row + bi[u])) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t x = base + static_cast<uint32_t>(u) * kThreads + t;
+          f(static_cast<int64_t>(bi[u]), bk[u], x < n);
+        }
+      }
+    });
+  } else {
+    resolve_bin(a, b, nv, d1, kr1, n_above, sh, [&](auto&& f) { for_slice(a, b, 0, nv, f); });
   }
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches) {
+  static bool done[64] = {false};  // one flag set per device
+  cudaError_t e = set_smem_once(topk_filter_kernel, static_cast<int>(sizeof(FilterShared)), done);
+  if (e != cudaSuccess) return e;
   dim3 grid(a.cpr, a.B);
-  topk_hist_kernel<1><<<grid, kThreads, 0, stream>>>(a);
-  topk_hist_kernel<2><<<grid, kThreads, 0, stream>>>(a);
-  topk_hist_kernel<3><<<grid, kThreads, 0, stream>>>(a);
-  topk_emit_kernel<<<grid, kThreads, 0, stream>>>(a);
-  *launches += 4;
+  topk_hist_kernel<<<grid, kThreads, 0, stream>>>(a);
+  topk_filter_kernel<<<grid, kThreads, sizeof(FilterShared), stream>>>(a);
+  *launches += 2;
   return cudaGetLastError();
 }
 

@@ -13,11 +13,12 @@
 // For them this entry point allocates nothing: it needs only the scores and
 // the output index buffer. Its scratch is g_topk_scratch below, a
 // __device__ array that every GPU which loads this library holds until the
-// process exits (kScratchBytes, about 1.6 MB).
+// process exits (kScratchBytes, 4 MB).
 //
-// Limits. At most IC_TOPK_NOALLOC_MAX_ROWS rows per call (64); larger calls
-// return IC_ERR_UNSUPPORTED and launch nothing. The other limits are those
-// of ic_topk (k <= 16384, N < 2^31).
+// Limits. At most IC_TOPK_NOALLOC_MAX_ROWS rows per call (64), and the
+// call's histograms and candidate buffers must fit the array (64 rows of up
+// to 131072 scores do); larger calls return IC_ERR_UNSUPPORTED and launch
+// nothing. The other limits are those of ic_topk (k <= 16384, N < 2^31).
 //
 // Sharing. Every call, from every stream and thread, uses the same array and
 // each call starts by clearing the part it uses (including its status word).
@@ -38,7 +39,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = 1600 * 1024;
+constexpr size_t kScratchBytes = 4 * 1024 * 1024;
 constexpr size_t kStatusBytes = 256;
 
 static __device__ __align__(256) unsigned char g_topk_scratch[kScratchBytes];
