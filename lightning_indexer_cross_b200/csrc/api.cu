@@ -238,6 +238,20 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return IC_ERR_INVALID_ARG;
   }
+  CUtensorMap omap;
+  {
+    const bool f32 = out_dtype == IC_F32;
+    const cuuint64_t es = f32 ? 4 : 2;
+    const cuuint64_t dims[4] = {512, static_cast<cuuint64_t>(L.splits), static_cast<cuuint64_t>(H),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {512 * es, 512 * es * L.splits, 512 * es * L.splits * H};
+    const cuuint32_t box[4] = {f32 ? 32u : 64u, 1, 32, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(&omap, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ws + L.o_off, dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return IC_ERR_INVALID_ARG;
+  }
   ic::MlaArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.kv = static_cast<const __nv_bfloat16*>(kv);
@@ -259,7 +273,7 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
   a.lse = lse;
   a.status = status;
   int launches = 0;
-  cudaError_t e = ic::launch_sparse_mla(qmap, a, stream, &launches);
+  cudaError_t e = ic::launch_sparse_mla(qmap, omap, a, stream, &launches);
   if (e != cudaSuccess) return IC_ERR_CUDA;
   g_launches += launches;
   return IC_OK;

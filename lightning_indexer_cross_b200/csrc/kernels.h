@@ -104,6 +104,10 @@ struct MlaArgs {
 int mla_smem_bytes(int ts);
 // qmap: 2-D tensor map over q viewed as [B*H rows, 576] bf16, box 64 x 128,
 // 128-byte swizzle (one 64-dim slice of a 128-head block per load).
-cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const MlaArgs& a, cudaStream_t stream, int* launches);
+// omap: 4-D tensor map over part_o as [B][H][splits][512] (innermost first:
+// 512, splits, H, B), box 128 bytes x 1 x 32 x 1, 128-byte swizzle (32 heads'
+// rows of one 64-dim (bf16) or 32-dim (fp32) block per store).
+cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a,
+                              cudaStream_t stream, int* launches);
 
 }  // namespace ic

@@ -20,12 +20,15 @@
 //        O_hi = P . V[:, 256:512] into columns [0, 256) (S is dead by then);
 //        V rows are the same gathered 576-d rows, read as an MN-major B
 //        operand (64 tokens x 256 dims per stage).
-// It writes an unnormalised partial (m, l, O) per split. The combine kernel
-// merges the splits, adds e^{sink} once to the denominator, applies the gate
-// and writes out / lse.
+// It writes a normalised partial (m, l, O / l) per split: O / l as 32-head x
+// 128-byte tiles staged in swizzled shared memory and written by TMA stores.
+// The combine kernel merges the splits, adds e^{sink} once to the
+// denominator, applies the gate and writes out / lse.
 //
-// Gathers are cp.async (16 B, zero fill for -1 rows) into 128-byte-swizzled
-// stages; producer threads fence the async proxy before signalling the MMA.
+// Warp roles (8 warps): 0-2 gather every stage, 3 issues the MMAs, 4-7 run the
+// softmax and the output and gather the stages in between. Gathers are
+// cp.async (16 B, zero fill for -1 rows) into 128-byte-swizzled stages; the
+// gathering threads fence the async proxy before signalling the MMA.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -44,6 +47,9 @@ constexpr int kProdThreads = 96;   // warps 0..2
 constexpr int kMmaWarp = 3;
 constexpr int kEpiWarp0 = 4;       // warps 4..7
 constexpr int kThreads = 256;
+constexpr int kGather = 224;       // gather threads: warps 0-2 and 4-7
+constexpr int kPvSolo = kStages;   // first PV stages: warps 0-2 alone, during the softmax
+constexpr int kOutSlots = 4;       // 4 KB output tiles per epilogue warp
 constexpr int kLookahead = kStages - 1;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -64,8 +70,38 @@ struct MlaCfg {
   static constexpr int kNumSt = kQKChunks + 2 * (TS / 64);
 };
 
+// PV stage p (64 selected rows x 256 latent dims) gathered by NT threads:
+// copy i is 16-byte chunk i % 8 of (row, 64-dim block) pair i / 8; thread gt
+// takes i = gt + NT n, so its chunk column is fixed.
+template <int TS, int NT>
+IC_DEV void gather_pv_stage(uint32_t base_u, const int32_t* idx_s, const __nv_bfloat16* kvb,
+                            const __nv_bfloat16* zero_src, int gt, int p) {
+  constexpr int kRowStep = NT / 8;
+  constexpr int kNP = (64 * 32 + NT - 1) / NT;
+  static_assert(NT % 8 == 0, "chunk column fixed per thread");
+  const int cc = gt & 7, q0 = gt >> 3;
+  const int jh = p / (TS / 64), tc = p % (TS / 64);
+  int tok[kNP];
+#pragma unroll
+  for (int n = 0; n < kNP; ++n) {
+    const int q = q0 + kRowStep * n;  // (row in chunk) * 4 + 64-dim block
+    tok[n] = q < 256 ? idx_s[tc * 64 + (q >> 2)] : -1;
+  }
+#pragma unroll
+  for (int n = 0; n < kNP; ++n) {
+    const int q = q0 + kRowStep * n;
+    if (q < 256) {
+      const int j = q >> 2, bb = q & 3;
+      const __nv_bfloat16* src =
+          tok[n] >= 0 ? kvb + static_cast<int64_t>(tok[n]) * kD + jh * 256 + bb * 64 + cc * 8 : zero_src;
+      cp_async16(base_u + bb * 8192 + sw128_offset(j, cc), src, tok[n] >= 0 ? 16u : 0u);
+    }
+  }
+}
+
 template <int TS>
 __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                   const __grid_constant__ CUtensorMap omap,
                                                                    const MlaArgs a) {
   using C = MlaCfg<TS>;
   extern __shared__ uint8_t smem_raw[];
@@ -91,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], kProdThreads);
+      mbar_init(&full[i], kGather);
       mbar_init(&empty[i], 1);
     }
     mbar_init(s_full, 1);
@@ -125,88 +161,70 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp < kMmaWarp) {
-    // ------------------------------------------------------------ gather warps
-    // QK stage c: the 64-dim slice c of the 128-head Q block by one TMA load,
-    // and slice c of every selected row by cp.async. PV stage: 64 selected
-    // rows x 256 latent dims by cp.async. Rows land in 128-byte-swizzled
-    // operand layouts; -1 slots are zero-filled (their logits are masked).
-    // (Measured on B200: 16-byte cp.async gathers sustain more bytes in
-    // flight per SM than 512-byte tile::gather4 TMA operations here.)
-    const int pt = threadIdx.x;
-    const __nv_bfloat16* kvb = a.kv + static_cast<int64_t>(b) * a.kv_batch_stride;
-    if (pt == 0) tma_prefetch_desc(&qmap);
-    // stage r's copies are in place: every gather thread arrives once; for
-    // QK stages thread 0's arrival also books the TMA bytes of the Q slice
-    auto arrive_stage = [&](int r) {
-      if (pt == 0 && r < kQKChunks) mbar_arrive_expect_tx(&full[r % kStages], kHeads * 128);
-      else mbar_arrive(&full[r % kStages]);
-    };
-    // Copy i of a stage is row i/8 (QK) or row-block i/8 (PV), 16-byte chunk
-    // i%8. Thread pt takes i = pt + kProdThreads*n, so its chunk column
-    // cc = pt % 8 is fixed and its QK rows (pt/8 + kRowStep*n) are the same
-    // in all nine QK stages: they are loaded into registers once.
-    constexpr int kNQ = (TS * 8 + kProdThreads - 1) / kProdThreads;
-    constexpr int kNP = (64 * 32 + kProdThreads - 1) / kProdThreads;
-    static_assert(kProdThreads % 8 == 0, "chunk column fixed per thread");
-    constexpr int kRowStep = kProdThreads / 8;
-    const int cc = pt & 7;
-    const int q0 = pt >> 3;  // 0 .. kRowStep-1
-    int qk_tok[kNQ];
+  // ---------------------------------------------------------------- gather
+  // Warps 0-2 gather every stage; the epilogue warps 4-7 gather too except
+  // while they run the softmax (the first kPvSolo PV stages, which warps 0-2
+  // take alone) and the output. QK stage c: the 64-dim slice c of the
+  // 128-head Q block by one TMA load, and slice c of every selected row by
+  // cp.async. PV stage: 64 selected rows x 256 latent dims by cp.async. Rows
+  // land in 128-byte-swizzled operand layouts; -1 slots are zero-filled (their
+  // logits are masked). (Measured on B200: the random 16-byte gathers of one
+  // SM scale with the number of threads issuing them, about 33 GB/s from 96
+  // threads and 62 GB/s from 256, while tile::gather4 and per-row bulk copies
+  // are limited by their issue rate.)
+  const bool producer = warp < kMmaWarp;
+  const int gt = producer ? static_cast<int>(threadIdx.x) : static_cast<int>(threadIdx.x) - 32;
+  const __nv_bfloat16* kvb = a.kv + static_cast<int64_t>(b) * a.kv_batch_stride;
+  constexpr int kQRowStep = kGather / 8;
+  constexpr int kNQ = (TS + kQRowStep - 1) / kQRowStep;
+  const int gcc = gt & 7, gq0 = gt >> 3;
+  int qk_tok[kNQ];  // this thread's QK rows, the same in all nine QK stages
+  if (warp != kMmaWarp) {
 #pragma unroll
     for (int n = 0; n < kNQ; ++n) {
-      const int j = q0 + kRowStep * n;
+      const int j = gq0 + kQRowStep * n;
       qk_tok[n] = j < TS ? idx_s[j] : -1;
     }
-    int s = 0;
+  }
+  // stage r's copies are in place: every gather thread arrives once; for QK
+  // stages thread 0's arrival also books the TMA bytes of the Q slice
+  auto arrive_stage = [&](int r) {
+    if (gt == 0 && producer && r < kQKChunks) mbar_arrive_expect_tx(&full[r % kStages], kHeads * 128);
+    else mbar_arrive(&full[r % kStages]);
+  };
+  // Gather stages [s0, s1); false if a wait gave up.
+  auto gather = [&](int s0, int s1) -> bool {
+    int s = s0;
     bool ok = true;
-    for (; s < C::kNumSt; ++s) {
+    for (; s < s1; ++s) {
       const int st = s % kStages;
-      const uint32_t ph = static_cast<uint32_t>((s / kStages) & 1);
-      if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status)) {
+      if (!mbar_wait(&empty[st], static_cast<uint32_t>((s / kStages) & 1) ^ 1u, abort_flag, a.status)) {
         ok = false;
         break;
       }
       uint8_t* base = stages + st * C::kStageBytes;
       const uint32_t base_u = smem_u32(base);
       if (s < kQKChunks) {
-        const int c = s;
         // rows past the last query read zeros; rows of a neighbouring query
         // are never written out
-        if (pt == 0) tma_load_2d(base, &qmap, &full[st], c * 64, b * a.H + hb * kHeads);
+        if (gt == 0 && producer) tma_load_2d(base, &qmap, &full[st], s * 64, b * a.H + hb * kHeads);
         const uint32_t kv_u = base_u + kHeads * 128;
 #pragma unroll
         for (int n = 0; n < kNQ; ++n) {
-          const int j = q0 + kRowStep * n;
+          const int j = gq0 + kQRowStep * n;
           if (j < TS) {
             const int tok = qk_tok[n];
-            const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + c * 64 + cc * 8 : a.kv;
-            cp_async16(kv_u + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
+            const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + s * 64 + gcc * 8 : a.kv;
+            cp_async16(kv_u + sw128_offset(j, gcc), src, tok >= 0 ? 16u : 0u);
           }
         }
       } else {
         const int p = s - kQKChunks;
-        const int jh = p / (TS / 64), tc = p % (TS / 64);
-        int pv_tok[kNP];
-#pragma unroll
-        for (int n = 0; n < kNP; ++n) {
-          const int q = q0 + kRowStep * n;  // (token in chunk) * 4 + 64-dim block
-          pv_tok[n] = q < 256 ? idx_s[tc * 64 + (q >> 2)] : -1;
-        }
-#pragma unroll
-        for (int n = 0; n < kNP; ++n) {
-          const int q = q0 + kRowStep * n;
-          if (q < 256) {
-            const int j = q >> 2, bb = q & 3;
-            const int tok = pv_tok[n];
-            const __nv_bfloat16* src =
-                tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + jh * 256 + bb * 64 + cc * 8 : a.kv;
-            cp_async16(base_u + bb * 8192 + sw128_offset(j, cc), src, tok >= 0 ? 16u : 0u);
-          }
-        }
+        if (p >= kPvSolo) gather_pv_stage<TS, kGather>(base_u, idx_s, kvb, a.kv, gt, p);
+        else if (producer) gather_pv_stage<TS, kProdThreads>(base_u, idx_s, kvb, a.kv, gt, p);
       }
       cp_async_commit();
-      if (s >= kLookahead) {
+      if (s - s0 >= kLookahead) {
         cp_async_wait<kLookahead>();
         fence_proxy_async_smem();
         arrive_stage(s - kLookahead);
@@ -215,13 +233,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     // land everything still in flight (also on the abort path)
     cp_async_wait<0>();
     fence_proxy_async_smem();
-    if (ok)
-      for (int r = (s > kLookahead ? s - kLookahead : 0); r < s; ++r) arrive_stage(r);
-    if (!ok && pt == 0) {
+    if (ok) {
+      for (int r = (s - kLookahead > s0 ? s - kLookahead : s0); r < s; ++r) arrive_stage(r);
+    } else if (gt == 0 && producer) {
       // wind down: the Q loads issued for QK stages still pending must land
-      for (int r = (s > kStages ? s - kStages : 0); r < s && r < kQKChunks; ++r)
+      for (int r = (s - kStages > s0 ? s - kStages : s0); r < s && r < kQKChunks; ++r)
         mbar_drain(&full[r % kStages], static_cast<uint32_t>((r / kStages) & 1));
     }
+    return ok;
+  };
+
+  if (producer) {
+    gather(0, C::kNumSt);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -274,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const float c2 = a.sm_scale * kLog2e;
     float mx = -INFINITY, l = 0.f;
-    bool ok = mbar_wait(s_full, 0, abort_flag, a.status);
+    bool ok = gather(0, kQKChunks);
+    ok = ok && mbar_wait(s_full, 0, abort_flag, a.status);
     __syncwarp();  // tcgen05.ld is warp-collective
     if (ok) {
       tc_fence_after();
@@ -341,58 +365,66 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(p_ready);
-      ok = mbar_wait(o_full, 0, abort_flag, a.status);
+      // the PV stages after the first kPvSolo are gathered by all seven warps
+      ok = gather(kQKChunks, C::kNumSt);
+      ok = ok && mbar_wait(o_full, 0, abort_flag, a.status);
       __syncwarp();
     }
     if (ok) {
       tc_fence_after();
-      const int64_t row = (static_cast<int64_t>(b) * a.H + head) * a.splits + sp;
-      // O / l (0 when no token was valid), transposed through shared memory
-      // in 32-dim chunks (the stage ring is idle once every MMA has retired)
-      // so each warp store writes whole rows segments.
+      // O / l (0 when no token was valid) as 32-row x 128-byte tiles in
+      // 128-byte-swizzled shared memory (the stage ring is idle once every
+      // MMA has retired), each written out by one TMA store; heads past H
+      // fall outside the map and are not written. O_lo sits in TMEM columns
+      // [256, 512), O_hi in [0, 256).
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      uint32_t* tile = reinterpret_cast<uint32_t*>(stages) + quad * (32 * 33);
-      const int64_t row0 = (static_cast<int64_t>(b) * a.H + hb * kHeads + quad * 32) * a.splits + sp;
-      const int nrows = min(32, a.H - (hb * kHeads + quad * 32));
-      const int64_t rstride = static_cast<int64_t>(a.splits) * kDv;  // elements between heads' rows
-      // O_lo sits in TMEM columns [256, 512), O_hi in [0, 256); 16 chunks of 32 dims
-      uint32_t rb0[32], rb1[32];
-      auto col_of = [](int c) { return c < 8 ? 256u + 32u * c : 32u * (c - 8); };
-      auto out_chunk = [&](const uint32_t (&rv)[32], int c) {
-        if (a.out_f32) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) tile[lane * 33 + j] = __float_as_uint(__uint_as_float(rv[j]) * inv_l);
+      uint8_t* tiles = stages + quad * (kOutSlots * 4096);
+      const int head0 = hb * kHeads + quad * 32;
+      auto put_tile = [&](int t, const uint32_t (&w)[32], int x) {
+        const int slot = t % kOutSlots;
+        if (t >= kOutSlots) {
+          if (lane == 0) bulk_wait_read<kOutSlots - 1>();  // the slot's previous store has read it
           __syncwarp();
-          float* dst = static_cast<float*>(a.part_o) + row0 * kDv + c * 32 + lane;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < nrows) dst[i * rstride] = __uint_as_float(tile[i * 33 + lane]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            tile[lane * 17 + j] = pack_bf16x2(__uint_as_float(rv[2 * j]) * inv_l, __uint_as_float(rv[2 * j + 1]) * inv_l);
-          __syncwarp();
-          // lanes 0-15 write row i, lanes 16-31 row i+1 (64 bytes each)
-          uint32_t* dst = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(a.part_o) + row0 * kDv + c * 32);
-          const int half = lane >> 4, w = lane & 15;
-#pragma unroll
-          for (int i = 0; i < 32; i += 2)
-            if (i + half < nrows) dst[(i + half) * (rstride / 2) + w] = tile[(i + half) * 17 + w];
         }
+        uint8_t* tile = tiles + slot * 4096;
+        const uint32_t tb = smem_u32(tile);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          st_shared_v4(tb + sw128_offset(lane, k), make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]));
+        fence_proxy_async_smem();
         __syncwarp();
+        if (lane == 0 && head0 < a.H) {
+          tma_store_4d(&omap, tile, x, sp, head0, b);
+          bulk_commit();
+        }
       };
-      tmem_ld32_issue(taddr + col_of(0), rb0);
-      tmem_ld_wait(rb0);
+      if (a.out_f32) {
 #pragma unroll 1
-      for (int c = 0; c < 16; c += 2) {
-        tmem_ld32_issue(taddr + col_of(c + 1), rb1);
-        out_chunk(rb0, c);
-        tmem_ld_wait(rb1);
-        if (c + 2 < 16) tmem_ld32_issue(taddr + col_of(c + 2), rb0);
-        out_chunk(rb1, c + 1);
-        if (c + 2 < 16) tmem_ld_wait(rb0);
+        for (int t = 0; t < 16; ++t) {  // 32 dims per tile
+          uint32_t rv[32];
+          tmem_ld32_issue(taddr + (t < 8 ? 256u + 32u * t : 32u * (t - 8)), rv);
+          tmem_ld_wait(rv);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) rv[j] = __float_as_uint(__uint_as_float(rv[j]) * inv_l);
+          put_tile(t, rv, 32 * t);
+        }
+      } else {
+#pragma unroll 1
+        for (int t = 0; t < 8; ++t) {  // 64 dims per tile
+          uint32_t rv[64];
+          tmem_ld64_issue(taddr + (t < 4 ? 256u + 64u * t : 64u * (t - 4)), rv);
+          tmem_ld_wait64(rv);
+          uint32_t w[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            w[j] = pack_bf16x2(__uint_as_float(rv[2 * j]) * inv_l, __uint_as_float(rv[2 * j + 1]) * inv_l);
+          put_tile(t, w, 64 * t);
+        }
       }
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
       if (head < a.H) {
+        const int64_t row = (static_cast<int64_t>(b) * a.H + head) * a.splits + sp;
         a.part_ml[row * 2 + 0] = mx;
         a.part_ml[row * 2 + 1] = l;
       }
@@ -410,6 +442,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
 
 // One warp per (query, head): merge the splits' (m, l, O), add the sink to
 // the denominator once, normalise, gate, write out and lse.
+// One partial row chunk (4 dims at i*128 + lane*4 of split s) as floats.
+IC_DEV void load_part4(const MlaArgs& a, int64_t off, float (&o)[4]) {
+  if (a.out_f32) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(static_cast<const float*>(a.part_o) + off));
+    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+  } else {
+    const uint2 v = __ldcg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.part_o) + off));
+    const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+    const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+    o[0] = __low2float(v01); o[1] = __high2float(v01); o[2] = __low2float(v23); o[3] = __high2float(v23);
+  }
+}
+
+// One warp per (query, head): merge the splits' (m, l, O/l), add the sink to
+// the denominator once, normalise, gate, write out and lse. Lane s holds
+// split s's (m, l); every split's partial row is requested before it is
+// reduced, so the loads of a head overlap.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * 4 + warp;
@@ -417,14 +466,30 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
   const int h = static_cast<int>(gw % a.H);
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + gw * a.splits;
   const int64_t pbase = gw * a.splits * kDv;
+  // gate logits first: independent of the partials
+  float gs[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) gs[4 * i + e] = 1.f;
+    if (a.gate) {
+      const uint2 graw = *reinterpret_cast<const uint2*>(a.gate + gw * kDv + i * 128 + lane * 4);
+      const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&graw.x);
+      const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&graw.y);
+      gs[4 * i] = __low2float(g01);
+      gs[4 * i + 1] = __high2float(g01);
+      gs[4 * i + 2] = __low2float(g23);
+      gs[4 * i + 3] = __high2float(g23);
+    }
+  }
   const float sink2 = a.sink[h] * kLog2e;
   float M = sink2;
-  for (int s = lane; s < a.splits; s += 32) M = fmaxf(M, ml[s].x);
+  for (int s = lane; s < a.splits; s += 32) M = fmaxf(M, __ldcg(&ml[s].x));
 #pragma unroll
   for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float den = 0.f;
   for (int s = lane; s < a.splits; s += 32) {
-    const float2 v = ml[s];
+    const float2 v = __ldcg(&ml[s]);
     den += v.x == -INFINITY ? 0.f : exp2f(v.x - M) * v.y;
   }
 #pragma unroll
@@ -433,24 +498,33 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int s = 0; s < a.splits; ++s) {
-    const float ms = ml[s].x;
-    if (ms == -INFINITY) continue;
-    const float wgt = exp2f(ms - M) * ml[s].y;  // partials hold O / l
+  for (int s0 = 0; s0 < a.splits; s0 += 32) {
+    // weight of split s0 + lane (partials hold O / l)
+    float wl = 0.f;
+    if (s0 + lane < a.splits) {
+      const float2 v = __ldcg(&ml[s0 + lane]);
+      wl = v.x == -INFINITY ? 0.f : exp2f(v.x - M) * v.y;
+    }
+    const int ns = min(32, a.splits - s0);
+    for (int j = 0; j < ns; j += 4) {
+      float o[4][16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float o[4];
-      if (a.out_f32) {
-        const float4 v = *reinterpret_cast<const float4*>(static_cast<const float*>(a.part_o) + pbase + s * kDv + i * 128 + lane * 4);
-        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-      } else {
-        const uint2 v = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.part_o) + pbase + s * kDv + i * 128 + lane * 4);
-        const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-        const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-        o[0] = __low2float(v01); o[1] = __high2float(v01); o[2] = __low2float(v23); o[3] = __high2float(v23);
+      for (int u = 0; u < 4; ++u)
+        if (j + u < ns)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float t4[4];
+            load_part4(a, pbase + static_cast<int64_t>(s0 + j + u) * kDv + i * 128 + lane * 4, t4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[u][4 * i + e] = t4[e];
+          }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float wgt = __shfl_sync(0xffffffffu, wl, (j + u) & 31);
+        if (j + u < ns && wgt != 0.f)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[e] = fmaf(wgt, o[u][e], acc[e]);
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[4 * i + e] = fmaf(wgt, o[e], acc[4 * i + e]);
     }
   }
   const float inv = 1.f / den;
@@ -459,14 +533,9 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
     const int d0 = i * 128 + lane * 4;
     float o[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = acc[4 * i + e] * inv;
-    if (a.gate) {
-      const uint2 graw = *reinterpret_cast<const uint2*>(a.gate + gw * kDv + d0);
-      const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&graw.x);
-      const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&graw.y);
-      const float g[4] = {__low2float(g01), __high2float(g01), __low2float(g23), __high2float(g23)};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] *= 1.f / (1.f + __expf(-g[e]));
+    for (int e = 0; e < 4; ++e) {
+      o[e] = acc[4 * i + e] * inv;
+      if (a.gate) o[e] *= 1.f / (1.f + __expf(-gs[4 * i + e]));
     }
     if (a.out_f32) {
       *reinterpret_cast<float4*>(static_cast<float*>(a.out) + gw * kDv + d0) = make_float4(o[0], o[1], o[2], o[3]);
@@ -481,14 +550,14 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
 }
 
 template <int TS>
-cudaError_t launch_ts(const CUtensorMap& qmap, const MlaArgs& a, cudaStream_t stream) {
+cudaError_t launch_ts(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a, cudaStream_t stream) {
   using C = MlaCfg<TS>;
   auto kern = sparse_mla_kernel<TS>;
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.B, (a.H + kHeads - 1) / kHeads);
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(qmap, a);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(qmap, omap, a);
   return cudaGetLastError();
 }
 
@@ -502,12 +571,13 @@ int mla_smem_bytes(int ts) {
   }
 }
 
-cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const MlaArgs& a, cudaStream_t stream, int* launches) {
+cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a, cudaStream_t stream,
+                              int* launches) {
   cudaError_t e;
   switch (a.ts) {
-    case 64: e = launch_ts<64>(qmap, a, stream); break;
-    case 128: e = launch_ts<128>(qmap, a, stream); break;
-    case 256: e = launch_ts<256>(qmap, a, stream); break;
+    case 64: e = launch_ts<64>(qmap, omap, a, stream); break;
+    case 128: e = launch_ts<128>(qmap, omap, a, stream); break;
+    case 256: e = launch_ts<256>(qmap, omap, a, stream); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
