@@ -66,7 +66,7 @@ int indexer_hp(int H_I) {
 
 ic_status_t indexer_impl(const void* q, const float* w, const void* k, const float* k_scale, ic_dtype_t k_dtype,
                          int B, int H_I, int d_I, int64_t N, int64_t k_batch_stride, int64_t scale_batch_stride,
-                         const int64_t* n_valid, float* scores, int* status, cudaStream_t stream) {
+                         const int64_t* n_valid, float* scores, int* status, cudaStream_t stream, bool pdl) {
   if (!q || !w || !k || !scores) return IC_ERR_INVALID_ARG;
   if (B < 1 || N < 1 || H_I < 1 || N >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
   if (k_dtype != IC_BF16 && k_dtype != IC_FP8_E4M3) return IC_ERR_UNSUPPORTED;
@@ -115,7 +115,7 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   a.total_items = groups * a.tiles;
   a.per_query = per_query ? 1 : 0;
   const int grid = static_cast<int>(std::min<int64_t>(num_sms(), a.total_items));
-  cudaError_t e = ic::launch_indexer(map, a, HP, d_I, fp8, grid, stream);
+  cudaError_t e = ic::launch_indexer(map, a, HP, d_I, fp8, grid, stream, pdl);
   if (e != cudaSuccess) return IC_ERR_CUDA;
   g_launches += 1;
   return IC_OK;
@@ -213,7 +213,8 @@ MlaLayout mla_layout(int B, int H, int k) {
 
 ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int64_t N, const int32_t* idx, int k,
                      const float* sink, const void* gate, float sm_scale, int B, int H, ic_dtype_t out_dtype,
-                     void* out, float* lse, uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream) {
+                     void* out, float* lse, uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream,
+                     bool pdl) {
   if (!q || !kv || !idx || !sink || !out || !ws) return IC_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || k < 1 || N < 1 || N >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || sm_scale == INFINITY) return IC_ERR_INVALID_ARG;
@@ -273,7 +274,7 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
   a.lse = lse;
   a.status = status;
   int launches = 0;
-  cudaError_t e = ic::launch_sparse_mla(qmap, omap, a, stream, &launches);
+  cudaError_t e = ic::launch_sparse_mla(qmap, omap, a, stream, pdl, &launches);
   if (e != cudaSuccess) return IC_ERR_CUDA;
   g_launches += launches;
   return IC_OK;
@@ -324,7 +325,7 @@ ic_status_t ic_indexer_score(const void* q, const float* w, const void* k, const
   g_launches = 0;
   if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
   return indexer_impl(q, w, k, k_scale, k_dtype, B, H_I, d_I, N, k_batch_stride, scale_batch_stride, n_valid,
-                      scores, static_cast<int*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+                      scores, static_cast<int*>(workspace), reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 size_t ic_topk_workspace_size(int B, int64_t N, int k) {
@@ -356,7 +357,7 @@ ic_status_t ic_sparse_mla_decode(const void* q, const void* kv, int64_t kv_batch
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return mla_impl(q, kv, kv_batch_stride, N, idx, k, sink, gate, sm_scale, B, H, out_dtype, out, lse,
                   ws + kStatusBytes, ws_bytes - kStatusBytes, reinterpret_cast<int*>(ws),
-                  reinterpret_cast<cudaStream_t>(stream));
+                  reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 size_t ic_layer_stack_workspace_size(const ic_stack_shape_t* shape) {
@@ -390,29 +391,39 @@ ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule
   float* scores = reinterpret_cast<float*>(ws + SL.scores_off);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int total = 0;
+  // Consecutive kernels of the stack overlap their launch and prologue with
+  // the previous kernel's tail (programmatic dependent launch). The first
+  // kernel of the call, and any kernel after a copy or memset, launches
+  // normally.
+  bool after_kernel = false;
   for (int l = 0; l < L; ++l) {
     const ic_layer_t& y = layers[l];
     if (schedule[l] == 'F') {
       g_launches = 0;
       ic_status_t r = indexer_impl(y.q_idx, y.w, y.k_idx, y.k_scale, s.k_dtype, s.B, s.H_I, s.d_I, s.N,
-                                   s.k_batch_stride, s.scale_batch_stride, s.n_valid, scores, status, st);
+                                   s.k_batch_stride, s.scale_batch_stride, s.n_valid, scores, status, st,
+                                   after_kernel);
       if (r != IC_OK) return r;
       total += g_launches;
       g_launches = 0;
       r = topk_impl(scores, s.B, s.N, s.n_valid, s.topk, index_buf, ws + SL.topk_off, SL.tk.total, status, st);
       if (r != IC_OK) return r;
       total += g_launches;
+      after_kernel = true;
     }
     g_launches = 0;
     ic_status_t r = mla_impl(y.q, y.kv, s.kv_batch_stride, s.N, index_buf, s.topk, y.sink, y.gate, s.sm_scale,
-                             s.B, s.H, s.out_dtype, y.out, y.lse, ws + SL.mla_off, SL.ml.total, status, st);
+                             s.B, s.H, s.out_dtype, y.out, y.lse, ws + SL.mla_off, SL.ml.total, status, st,
+                             after_kernel);
     if (r != IC_OK) return r;
     total += g_launches;
+    after_kernel = true;
     if (idx_trace) {
       const size_t n = size_t(s.B) * s.topk;
       if (cudaMemcpyAsync(idx_trace + size_t(l) * n, index_buf, n * 4, cudaMemcpyDeviceToDevice, st) !=
           cudaSuccess)
         return IC_ERR_CUDA;
+      after_kernel = false;
     }
   }
   g_launches = total;

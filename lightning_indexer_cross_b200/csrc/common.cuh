@@ -36,6 +36,16 @@ IC_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// pdl_trigger lets the next kernel of the stream (if launched with
+// programmatic serialisation) be scheduled while this one runs; pdl_wait
+// blocks until the previous kernel of the stream has completed and its
+// memory is visible. Every kernel of this library calls pdl_wait before its
+// first global-memory access and before allocating tensor memory. Both are
+// no-ops for kernels launched without the attribute.
+IC_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+IC_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 IC_DEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -296,6 +306,8 @@ IC_DEV float4 ld_shared_v4f(const void* p) {
   return v;
 }
 
+// Element e (0 = low half, 1 = high half) of a packed bf16 pair, as float.
+IC_DEV float bf16_lane(uint32_t w, int e) { return __uint_as_float(e ? (w & 0xffff0000u) : (w << 16)); }
 IC_DEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
 
   // This CTA's contiguous share of the (group, tile) work list.
   const int64_t total = a.total_items;
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&kmap);
+  pdl_wait();
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
@@ -373,23 +375,24 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
 }
 
 template <int D_I, int HP, bool FP8>
-cudaError_t launch_indexer_inst(const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t stream) {
+cudaError_t launch_indexer_inst(const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t stream,
+                                bool pdl) {
   using C = IdxCfg<D_I, FP8>;
   auto kern = indexer_tc_kernel<D_I, HP, FP8>;
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, a);
-  return cudaGetLastError();
+  e = launch_kernel(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, pdl, map, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D_I, bool FP8>
-cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t s) {
+cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t s, bool pdl) {
   switch (HP) {
-    case 16: return launch_indexer_inst<D_I, 16, FP8>(map, a, grid, s);
-    case 32: return launch_indexer_inst<D_I, 32, FP8>(map, a, grid, s);
-    case 64: return launch_indexer_inst<D_I, 64, FP8>(map, a, grid, s);
-    case 128: return launch_indexer_inst<D_I, 128, FP8>(map, a, grid, s);
+    case 16: return launch_indexer_inst<D_I, 16, FP8>(map, a, grid, s, pdl);
+    case 32: return launch_indexer_inst<D_I, 32, FP8>(map, a, grid, s, pdl);
+    case 64: return launch_indexer_inst<D_I, 64, FP8>(map, a, grid, s, pdl);
+    case 128: return launch_indexer_inst<D_I, 128, FP8>(map, a, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -402,9 +405,13 @@ int indexer_smem_bytes(int d_I, bool fp8) {
 }
 
 cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
-                           cudaStream_t stream) {
-  if (d_I == 64) return fp8 ? dispatch_hp<64, true>(HP, map, a, grid, stream) : dispatch_hp<64, false>(HP, map, a, grid, stream);
-  if (d_I == 128) return fp8 ? dispatch_hp<128, true>(HP, map, a, grid, stream) : dispatch_hp<128, false>(HP, map, a, grid, stream);
+                           cudaStream_t stream, bool pdl) {
+  if (d_I == 64)
+    return fp8 ? dispatch_hp<64, true>(HP, map, a, grid, stream, pdl)
+               : dispatch_hp<64, false>(HP, map, a, grid, stream, pdl);
+  if (d_I == 128)
+    return fp8 ? dispatch_hp<128, true>(HP, map, a, grid, stream, pdl)
+               : dispatch_hp<128, false>(HP, map, a, grid, stream, pdl);
   return cudaErrorInvalidValue;
 }
 

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include <cuda_bf16.h>
 
 #include "../../include/indexcache.h"
@@ -27,6 +29,26 @@ inline cudaError_t set_smem_once(Kernel kern, int bytes, bool (&done)[64]) {
   return e;
 }
 
+// Launch a kernel; with pdl set, with programmatic stream serialisation, so
+// it may start while the previous kernel in the stream (one of this library's,
+// which all wait with griddepcontrol.wait before touching global memory)
+// finishes. Only set pdl when the previous stream operation is such a kernel.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                 bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 struct IndexerArgs {
   const __nv_bfloat16* q;      // [B, H_I, d_I]
   const float* w;              // [B, H_I]
@@ -45,7 +67,7 @@ struct IndexerArgs {
 
 int indexer_smem_bytes(int d_I, bool fp8);
 cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
-                           cudaStream_t stream);
+                           cudaStream_t stream, bool pdl);
 
 // 32-bit words of per-row top-k control state (one 128-byte line per row,
 // so rows do not contend for the same line in L2).
@@ -108,6 +130,6 @@ int mla_smem_bytes(int ts);
 // 512, splits, H, B), box 128 bytes x 1 x 32 x 1, 128-byte swizzle (32 heads'
 // rows of one 64-dim (bf16) or 32-dim (fp32) block per store).
 cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a,
-                              cudaStream_t stream, int* launches);
+                              cudaStream_t stream, bool pdl, int* launches);
 
 }  // namespace ic

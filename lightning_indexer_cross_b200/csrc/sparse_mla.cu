@@ -124,8 +124,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   const int hb = blockIdx.z;   // head block
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok0 = sp * TS;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&omap);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], kGather);
       mbar_init(&empty[i], 1);
@@ -136,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     *abort_flag = 0;
     fence_mbar_init();
   }
+  pdl_wait();
   // selected rows of this split; anything outside [0, N) is treated as -1
   static_assert(TS % 32 == 0, "whole warps of selected rows");
   for (int j0 = warp * 32; j0 < TS; j0 += kThreads) {  // warp-uniform
@@ -440,125 +444,140 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   }
 }
 
-// One warp per (query, head): merge the splits' (m, l, O), add the sink to
-// the denominator once, normalise, gate, write out and lse.
-// One partial row chunk (4 dims at i*128 + lane*4 of split s) as floats.
-IC_DEV void load_part4(const MlaArgs& a, int64_t off, float (&o)[4]) {
-  if (a.out_f32) {
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(static_cast<const float*>(a.part_o) + off));
-    o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-  } else {
-    const uint2 v = __ldcg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.part_o) + off));
-    const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-    const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-    o[0] = __low2float(v01); o[1] = __high2float(v01); o[2] = __low2float(v23); o[3] = __high2float(v23);
-  }
+// One warp per (query, head): merge the splits' normalised partials
+// (m, l, O / l), add e^{sink} once to the denominator, normalise, gate, write
+// out and lse. Lane `lane` owns 16 of the 512 output dims: with bf16 partials
+// dims [8 lane, 8 lane + 8) and [256 + 8 lane, 256 + 8 lane + 8) (two 16-byte
+// loads per split), with fp32 partials dims 128 i + 4 lane + [0, 4) for
+// i < 4. Every split of a chunk of CH splits is requested before any is
+// reduced, so one memory latency covers a whole chunk; chunks are merged with
+// a running maximum.
+template <bool F32>
+IC_DEV int comb_dim(int lane, int e) {
+  if constexpr (F32) return (e >> 2) * 128 + lane * 4 + (e & 3);
+  else return (e >> 3) * 256 + lane * 8 + (e & 7);
 }
 
-// One warp per (query, head): merge the splits' (m, l, O/l), add the sink to
-// the denominator once, normalise, gate, write out and lse. Lane s holds
-// split s's (m, l); every split's partial row is requested before it is
-// reduced, so the loads of a head overlap.
+template <bool F32>
 __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
+  constexpr int CH = F32 ? 4 : 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * 4 + warp;
+  pdl_trigger();
+  pdl_wait();
   if (gw >= static_cast<int64_t>(a.B) * a.H) return;
   const int h = static_cast<int>(gw % a.H);
-  const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + gw * a.splits;
-  const int64_t pbase = gw * a.splits * kDv;
-  // gate logits first: independent of the partials
-  float gs[16];
+  const int S = a.splits;
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + gw * S;
+  // gate logits (independent of the partials)
+  float g[16];
+  if (a.gate) {
+    const __nv_bfloat16* gp = a.gate + gw * kDv;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+    for (int r = 0; r < (F32 ? 4 : 2); ++r) {
+      const int d0 = comb_dim<F32>(lane, r * (F32 ? 4 : 8));
+      if constexpr (F32) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(gp + d0));
+        const uint32_t w[2] = {v.x, v.y};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) gs[4 * i + e] = 1.f;
-    if (a.gate) {
-      const uint2 graw = *reinterpret_cast<const uint2*>(a.gate + gw * kDv + i * 128 + lane * 4);
-      const __nv_bfloat162 g01 = *reinterpret_cast<const __nv_bfloat162*>(&graw.x);
-      const __nv_bfloat162 g23 = *reinterpret_cast<const __nv_bfloat162*>(&graw.y);
-      gs[4 * i] = __low2float(g01);
-      gs[4 * i + 1] = __high2float(g01);
-      gs[4 * i + 2] = __low2float(g23);
-      gs[4 * i + 3] = __high2float(g23);
+        for (int e = 0; e < 4; ++e) g[4 * r + e] = bf16_lane(w[e >> 1], e & 1);
+      } else {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(gp + d0));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[8 * r + e] = bf16_lane(w[e >> 1], e & 1);
+      }
     }
   }
   const float sink2 = a.sink[h] * kLog2e;
-  float M = sink2;
-  for (int s = lane; s < a.splits; s += 32) M = fmaxf(M, __ldcg(&ml[s].x));
-#pragma unroll
-  for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float den = 0.f;
-  for (int s = lane; s < a.splits; s += 32) {
-    const float2 v = __ldcg(&ml[s]);
-    den += v.x == -INFINITY ? 0.f : exp2f(v.x - M) * v.y;
-  }
-#pragma unroll
-  for (int off = 16; off; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-  den += exp2f(sink2 - M);
+  float M = sink2, den = 1.f;  // the sink's term e^{sink - M}, M = sink so far
   float acc[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (int s0 = 0; s0 < a.splits; s0 += 32) {
-    // weight of split s0 + lane (partials hold O / l)
-    float wl = 0.f;
-    if (s0 + lane < a.splits) {
-      const float2 v = __ldcg(&ml[s0 + lane]);
-      wl = v.x == -INFINITY ? 0.f : exp2f(v.x - M) * v.y;
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  for (int s0 = 0; s0 < S; s0 += CH) {
+    float2 mlv[CH];
+    uint4 raw[CH][F32 ? 4 : 2];
+#pragma unroll
+    for (int u = 0; u < CH; ++u) {
+      if (s0 + u < S) {
+        mlv[u] = __ldcg(&ml[s0 + u]);
+        const int64_t rowoff = (gw * S + s0 + u) * kDv;
+#pragma unroll
+        for (int r = 0; r < (F32 ? 4 : 2); ++r) {
+          const int d0 = comb_dim<F32>(lane, r * (F32 ? 4 : 8));
+          raw[u][r] = F32 ? __ldcg(reinterpret_cast<const uint4*>(static_cast<const float*>(a.part_o) + rowoff + d0))
+                          : __ldcg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.part_o) +
+                                                                  rowoff + d0));
+        }
+      } else {
+        mlv[u] = make_float2(-INFINITY, 0.f);
+      }
     }
-    const int ns = min(32, a.splits - s0);
-    for (int j = 0; j < ns; j += 4) {
-      float o[4][16];
+    float Mc = M;
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (j + u < ns)
+    for (int u = 0; u < CH; ++u) Mc = fmaxf(Mc, mlv[u].x);
+    const float sc = exp2f(M - Mc);
+    den *= sc;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            float t4[4];
-            load_part4(a, pbase + static_cast<int64_t>(s0 + j + u) * kDv + i * 128 + lane * 4, t4);
+    for (int e = 0; e < 16; ++e) acc[e] *= sc;
+    M = Mc;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) o[u][4 * i + e] = t4[e];
-          }
+    for (int u = 0; u < CH; ++u) {
+      if (mlv[u].x == -INFINITY) continue;  // no valid token in that split
+      const float wgt = exp2f(mlv[u].x - Mc) * mlv[u].y;
+      den += wgt;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float wgt = __shfl_sync(0xffffffffu, wl, (j + u) & 31);
-        if (j + u < ns && wgt != 0.f)
+      for (int r = 0; r < (F32 ? 4 : 2); ++r) {
+        const uint32_t w[4] = {raw[u][r].x, raw[u][r].y, raw[u][r].z, raw[u][r].w};
+        if constexpr (F32) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) acc[e] = fmaf(wgt, o[u][e], acc[e]);
+          for (int e = 0; e < 4; ++e) acc[4 * r + e] = fmaf(wgt, __uint_as_float(w[e]), acc[4 * r + e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[8 * r + e] = fmaf(wgt, bf16_lane(w[e >> 1], e & 1), acc[8 * r + e]);
+        }
       }
     }
   }
   const float inv = 1.f / den;
+  float o[16];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int d0 = i * 128 + lane * 4;
-    float o[4];
+  for (int e = 0; e < 16; ++e) {
+    o[e] = acc[e] * inv;
+    if (a.gate) o[e] *= 1.f / (1.f + __expf(-g[e]));
+  }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      o[e] = acc[4 * i + e] * inv;
-      if (a.gate) o[e] *= 1.f / (1.f + __expf(-gs[4 * i + e]));
-    }
+  for (int r = 0; r < (F32 ? 4 : 2); ++r) {
+    const int d0 = comb_dim<F32>(lane, r * (F32 ? 4 : 8));
     if (a.out_f32) {
-      *reinterpret_cast<float4*>(static_cast<float*>(a.out) + gw * kDv + d0) = make_float4(o[0], o[1], o[2], o[3]);
+      float* dst = static_cast<float*>(a.out) + gw * kDv + d0;
+      if constexpr (F32) {
+        *reinterpret_cast<float4*>(dst) = make_float4(o[4 * r], o[4 * r + 1], o[4 * r + 2], o[4 * r + 3]);
+      }
     } else {
-      uint2 pk;
-      pk.x = pack_bf16x2(o[0], o[1]);
-      pk.y = pack_bf16x2(o[2], o[3]);
-      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + d0) = pk;
+      if constexpr (!F32) {
+        uint4 pk;
+        pk.x = pack_bf16x2(o[8 * r], o[8 * r + 1]);
+        pk.y = pack_bf16x2(o[8 * r + 2], o[8 * r + 3]);
+        pk.z = pack_bf16x2(o[8 * r + 4], o[8 * r + 5]);
+        pk.w = pack_bf16x2(o[8 * r + 6], o[8 * r + 7]);
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + d0) = pk;
+      }
     }
   }
   if (a.lse && lane == 0) a.lse[gw] = (M + log2f(den)) / kLog2e;
 }
 
 template <int TS>
-cudaError_t launch_ts(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a, cudaStream_t stream) {
+cudaError_t launch_ts(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a, cudaStream_t stream,
+                      bool pdl) {
   using C = MlaCfg<TS>;
   auto kern = sparse_mla_kernel<TS>;
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   dim3 grid(a.splits, a.B, (a.H + kHeads - 1) / kHeads);
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(qmap, omap, a);
-  return cudaGetLastError();
+  return launch_kernel(kern, grid, dim3(kThreads), C::kSmemBytes, stream, pdl, qmap, omap, a);
 }
 
 }  // namespace
@@ -572,17 +591,20 @@ int mla_smem_bytes(int ts) {
 }
 
 cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a, cudaStream_t stream,
-                              int* launches) {
+                              bool pdl, int* launches) {
   cudaError_t e;
   switch (a.ts) {
-    case 64: e = launch_ts<64>(qmap, omap, a, stream); break;
-    case 128: e = launch_ts<128>(qmap, omap, a, stream); break;
-    case 256: e = launch_ts<256>(qmap, omap, a, stream); break;
+    case 64: e = launch_ts<64>(qmap, omap, a, stream, pdl); break;
+    case 128: e = launch_ts<128>(qmap, omap, a, stream, pdl); break;
+    case 256: e = launch_ts<256>(qmap, omap, a, stream, pdl); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
   const int64_t warps = static_cast<int64_t>(a.B) * a.H;
-  mla_combine_kernel<<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(a);
+  const dim3 grid(static_cast<unsigned>((warps + 3) / 4));
+  e = a.out_f32 ? launch_kernel(mla_combine_kernel<true>, grid, dim3(128), 0, stream, true, a)
+                : launch_kernel(mla_combine_kernel<false>, grid, dim3(128), 0, stream, true, a);
+  if (e != cudaSuccess) return e;
   *launches += 2;
   return cudaGetLastError();
 }

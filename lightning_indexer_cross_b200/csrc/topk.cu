@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(kThreads) topk_hist_kernel(const TopkArgs a) {
   __shared__ uint32_t sh_kr;
   __shared__ int sh_last;
   const int b = blockIdx.y, c = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();
   const int64_t nv = row_valid(a, b);
   if (nv <= a.k) return;  // the filter pass takes every valid index
   const int64_t lo = static_cast<int64_t>(c) * a.slice;
@@ -307,6 +309,8 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
   FilterShared& sh = *reinterpret_cast<FilterShared*>(smem_raw);
   const int b = blockIdx.y, c = blockIdx.x;
   const int t = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   int32_t* out = a.idx + static_cast<int64_t>(b) * a.k;
   const int64_t nv = row_valid(a, b);
   if (nv <= a.k) {
@@ -456,8 +460,12 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches) {
   cudaError_t e = set_smem_once(topk_filter_kernel, static_cast<int>(sizeof(FilterShared)), done);
   if (e != cudaSuccess) return e;
   dim3 grid(a.cpr, a.B);
-  topk_hist_kernel<<<grid, kThreads, 0, stream>>>(a);
-  topk_filter_kernel<<<grid, kThreads, sizeof(FilterShared), stream>>>(a);
+  // the histogram pass follows the caller's memset of its counters (no
+  // programmatic overlap); the filter pass overlaps the histogram pass's tail
+  e = launch_kernel(topk_hist_kernel, grid, dim3(kThreads), 0, stream, false, a);
+  if (e != cudaSuccess) return e;
+  e = launch_kernel(topk_filter_kernel, grid, dim3(kThreads), sizeof(FilterShared), stream, true, a);
+  if (e != cudaSuccess) return e;
   *launches += 2;
   return cudaGetLastError();
 }
