@@ -186,12 +186,14 @@ using ic::topk_layout;
 using ic::topk_impl;
 
 // ------------------------------------------------------------------ sparse MLA
+// Selected rows per work unit: the largest of 256, 128 that still gives at
+// least 4/5 of a work unit per SM, else 64.
 int mla_ts(int B, int H, int k) {
   const int hb = (H + 127) / 128;
   const int sms = num_sms();
   for (int ts : {256, 128}) {
-    const int64_t ctas = ceil_div<int64_t>(k, ts) * B * hb;
-    if (ctas * 5 >= static_cast<int64_t>(sms) * 4) return ts;
+    const int64_t units = ceil_div<int64_t>(k, ts) * B * hb;
+    if (units * 5 >= static_cast<int64_t>(sms) * 4) return ts;
   }
   return 64;
 }
@@ -267,6 +269,12 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
   a.H = H;
   a.splits = L.splits;
   a.ts = L.ts;
+  {
+    const int64_t units = int64_t(L.splits) * B * ((H + 127) / 128);
+    if (units >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+    a.units = static_cast<int>(units);
+    a.ctas = static_cast<int>(std::min<int64_t>(units, num_sms()));
+  }
   a.part_o = ws + L.o_off;
   a.part_ml = reinterpret_cast<float*>(ws + L.ml_off);
   a.out = out;

@@ -115,7 +115,9 @@ struct MlaArgs {
   float sm_scale;
   int B, H;
   int splits;                // ceil(k / TS)
-  int ts;                    // tokens per CTA
+  int ts;                    // selected rows per work unit
+  int units;                 // splits * B * ceil(H / 128) work units
+  int ctas;                  // persistent CTAs (each takes units blockIdx.x + i * ctas)
   void* part_o;              // [B, H, splits, 512] normalised O/l: bf16 if out is bf16, else fp32
   float* part_ml;            // [B, H, splits, 2]  (max in log2 units, sum)
   void* out;                 // [B, H, 512]

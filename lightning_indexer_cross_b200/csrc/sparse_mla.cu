@@ -8,27 +8,30 @@
 //   o   = sum_j e^{z_j} kv[idx_j, :512] / (e^{sink_h} + sum_j e^{z_j})
 //   out = sigmoid(gate[b,h,:]) * o
 //
-// Main kernel: one CTA per (token split of TS <= 256 selected rows, query,
-// block of 128 heads). Tensor memory holds 512 fp32 columns per lane, and the
-// 128 x 512 output alone would fill it, so the CTA works in two phases:
+// Main kernel: persistent, one CTA per SM; a work unit is (split of TS <= 256
+// selected rows, query, block of 128 heads). Tensor memory holds 512 fp32
+// columns per lane, and the 128 x 512 output alone fills it, so each unit is
+// worked in two phases:
 //   QK   S[128 heads x TS] = Q . KV^T over 9 slices of 64 dims (tcgen05,
-//        M = 128 heads, N = TS tokens) into TMEM columns [0, TS);
+//        M = 128 heads, N = TS rows) into TMEM columns [0, TS);
 //   soft the epilogue warps read S (one head per TMEM lane), take the exact
-//        max over the CTA's tokens, write P = 2^{z log2e - m} as bf16 into
+//        max over the unit's rows, write P = 2^{z log2e - m} as bf16 into
 //        shared memory in the K-major layout of an MMA A operand;
 //   PV   O_lo = P . V[:, 0:256] into columns [256, 512), then
 //        O_hi = P . V[:, 256:512] into columns [0, 256) (S is dead by then);
-//        V rows are the same gathered 576-d rows, read as an MN-major B
-//        operand (64 tokens x 256 dims per stage).
-// It writes a normalised partial (m, l, O / l) per split: O / l as 32-head x
-// 128-byte tiles staged in swizzled shared memory and written by TMA stores.
-// The combine kernel merges the splits, adds e^{sink} once to the
-// denominator, applies the gate and writes out / lse.
+//        V rows are the same gathered rows, read again as an MN-major B
+//        operand (64 rows x 256 dims per stage).
+// Each unit writes a normalised partial (m, l, O / l): O / l as 32-head x
+// 128-byte tiles staged in swizzled shared memory and written by TMA stores,
+// O_hi first so the next unit's QK can start while O_lo is written. The
+// combine kernel merges the splits, adds e^{sink} once to the denominator,
+// applies the gate and writes out / lse.
 //
-// Warp roles (8 warps): 0-2 gather every stage, 3 issues the MMAs, 4-7 run the
-// softmax and the output and gather the stages in between. Gathers are
-// cp.async (16 B, zero fill for -1 rows) into 128-byte-swizzled stages; the
-// gathering threads fence the async proxy before signalling the MMA.
+// Warp roles (12 warps): 0-6 gather every stage of every unit (one ring of
+// three stages), 7 issues the MMAs, 8-11 run the softmax and the output.
+// Gathers are cp.async (16 B, zero fill for -1 rows) into 128-byte-swizzled
+// stages; the gathering threads fence the async proxy before signalling the
+// MMA. Each unit's row indices are loaded one unit ahead.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -40,16 +43,15 @@ constexpr int kD = 576;
 constexpr int kDv = 512;
 constexpr int kHeads = 128;      // heads per CTA (MMA M)
 constexpr int kQKChunks = kD / 64;
+// 12 warps (three per SM sub-partition, so at most 168 registers per thread):
+// seven gather warps, the MMA issuer, four softmax/output warps (one per TMEM
+// lane quadrant, quadrant = warp % 4)
+constexpr int kGatherWarps = 7;
+constexpr int kGather = kGatherWarps * 32;
+constexpr int kMmaWarp = 7;
+constexpr int kEpiWarp0 = 8;
+constexpr int kThreads = 384;
 constexpr int kStages = 3;
-// 8 warps (two per SM sub-partition, so up to 255 registers per thread):
-// three gather warps, the MMA issuer, four epilogue warps (TMEM lane quadrants)
-constexpr int kProdThreads = 96;   // warps 0..2
-constexpr int kMmaWarp = 3;
-constexpr int kEpiWarp0 = 4;       // warps 4..7
-constexpr int kThreads = 256;
-constexpr int kGather = 224;       // gather threads: warps 0-2 and 4-7
-constexpr int kPvSolo = kStages;   // first PV stages: warps 0-2 alone, during the softmax
-constexpr int kOutSlots = 4;       // 4 KB output tiles per epilogue warp
 constexpr int kLookahead = kStages - 1;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -59,15 +61,21 @@ struct MlaCfg {
   static constexpr int kPVStage = 64 * 256 * 2;
   static constexpr int kStageBytes = kQKStage > kPVStage ? kQKStage : kPVStage;
   static constexpr int kPBytes = kHeads * TS * 2;
+  // output tiles (4 KB) per epilogue warp, staged in the P buffer
+  static constexpr int kOutSlots = kPBytes / (4 * 4096) < 4 ? kPBytes / (4 * 4096) : 4;
   static constexpr int kOffStages = 0;
   static constexpr int kOffP = kStages * kStageBytes;
-  static constexpr int kOffIdx = kOffP + kPBytes;
-  static constexpr int kOffMask = kOffIdx + TS * 4;
-  static constexpr int kOffBar = kOffMask + (TS / 32) * 4 + 8;
-  static constexpr int kNumBars = 2 * kStages + 3;
+  static constexpr int kOffIdx = kOffP + kPBytes;         // [2][TS] selected rows, double-buffered
+  static constexpr int kOffMask = kOffIdx + 2 * TS * 4;   // [2][TS / 32] validity bits
+  static constexpr int kOffBar = kOffMask + 2 * (TS / 32) * 4;
+  // full[kStages], empty[kStages], s_full, p_ready, o_full, o_hi_free, retire, idx_ready[2], idx_free[2]
+  static constexpr int kNumBars = 2 * kStages + 9;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr int kNumSt = kQKChunks + 2 * (TS / 64);
+  static_assert(kOutSlots >= 1, "at least one output tile per warp");
+  static_assert(kOffBar % 8 == 0, "mbarrier alignment");
+  static_assert(kSmemBytes <= 232448, "fits one CTA per SM");
 };
 
 // PV stage p (64 selected rows x 256 latent dims) gathered by NT threads:
@@ -99,6 +107,24 @@ IC_DEV void gather_pv_stage(uint32_t base_u, const int32_t* idx_s, const __nv_bf
   }
 }
 
+// Work unit u -> (token split, query, head block); splits of one query are
+// adjacent, so the CTAs working at one time share each query's Q rows in L2.
+struct Unit {
+  int sp, b, hb;
+};
+IC_DEV Unit unit_of(const MlaArgs& a, int u) {
+  Unit w;
+  w.sp = u % a.splits;
+  const int r = u / a.splits;
+  w.b = r % a.B;
+  w.hb = r / a.B;
+  return w;
+}
+
+// Persistent: CTA c takes units c, c + ctas, c + 2 ctas, ... The gather warps
+// run continuously through the units' stages (a ring of kStages shared-memory
+// stages); the output of unit i (TMEM -> swizzled tiles -> TMA stores)
+// overlaps the QK gathers and MMAs of unit i + 1.
 template <int TS>
 __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap,
                                                                    const __grid_constant__ CUtensorMap omap,
@@ -109,21 +135,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   uint8_t* stages = smem + C::kOffStages;
   uint8_t* ps = smem + C::kOffP;
   int32_t* idx_s = reinterpret_cast<int32_t*>(smem + C::kOffIdx);
-  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + C::kOffMask);  // bit j of word w: token 32w+j valid
+  uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + C::kOffMask);  // bit j of word w: row 32w+j valid
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;
-  uint64_t* p_ready = s_full + 1;
-  uint64_t* o_full = p_ready + 1;
+  uint64_t* s_full = empty + kStages;  // S of the current unit in TMEM
+  uint64_t* p_ready = s_full + 1;      // P in shared memory, S read
+  uint64_t* o_full = p_ready + 1;      // O of the current unit in TMEM
+  uint64_t* o_hi_free = o_full + 1;    // TMEM columns [0, 256) read out
+  uint64_t* retire = o_hi_free + 1;    // every MMA of this CTA retired
+  uint64_t* idx_ready = retire + 1;    // [2] selected rows of a unit in shared memory
+  uint64_t* idx_free = idx_ready + 2;  // [2] the softmax is done with a unit's validity bits
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
-  const int sp = blockIdx.x;   // token split
-  const int b = blockIdx.y;    // query
-  const int hb = blockIdx.z;   // head block
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tok0 = sp * TS;
   pdl_trigger();
 
   if (threadIdx.x == 0) {
@@ -136,26 +162,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     mbar_init(s_full, 1);
     mbar_init(p_ready, 128);  // the four epilogue warps
     mbar_init(o_full, 1);
+    mbar_init(o_hi_free, 128);
+    mbar_init(retire, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&idx_ready[i], kGather);
+      mbar_init(&idx_free[i], 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
   pdl_wait();
-  // selected rows of this split; anything outside [0, N) is treated as -1
-  static_assert(TS % 32 == 0, "whole warps of selected rows");
-  for (int j0 = warp * 32; j0 < TS; j0 += kThreads) {  // warp-uniform
-    const int j = j0 + lane;
-    int v = -1;
-    if (tok0 + j < a.k) {
-      v = a.idx[static_cast<int64_t>(b) * a.k + tok0 + j];
-      if (v < -1 || static_cast<int64_t>(v) >= a.N) {
-        record_status(a.status, IC_ERR_BAD_INDEX);
-        v = -1;
-      }
-    }
-    idx_s[j] = v;
-    const uint32_t bal = __ballot_sync(0xffffffffu, v >= 0);
-    if (lane == 0) vmask[j0 >> 5] = bal;
-  }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
@@ -165,90 +181,125 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  // ---------------------------------------------------------------- gather
-  // Warps 0-2 gather every stage; the epilogue warps 4-7 gather too except
-  // while they run the softmax (the first kPvSolo PV stages, which warps 0-2
-  // take alone) and the output. QK stage c: the 64-dim slice c of the
-  // 128-head Q block by one TMA load, and slice c of every selected row by
-  // cp.async. PV stage: 64 selected rows x 256 latent dims by cp.async. Rows
-  // land in 128-byte-swizzled operand layouts; -1 slots are zero-filled (their
-  // logits are masked). (Measured on B200: the random 16-byte gathers of one
-  // SM scale with the number of threads issuing them, about 33 GB/s from 96
-  // threads and 62 GB/s from 256, while tile::gather4 and per-row bulk copies
-  // are limited by their issue rate.)
-  const bool producer = warp < kMmaWarp;
-  const int gt = producer ? static_cast<int>(threadIdx.x) : static_cast<int>(threadIdx.x) - 32;
-  const __nv_bfloat16* kvb = a.kv + static_cast<int64_t>(b) * a.kv_batch_stride;
-  constexpr int kQRowStep = kGather / 8;
-  constexpr int kNQ = (TS + kQRowStep - 1) / kQRowStep;
-  const int gcc = gt & 7, gq0 = gt >> 3;
-  int qk_tok[kNQ];  // this thread's QK rows, the same in all nine QK stages
-  if (warp != kMmaWarp) {
+  if (warp < kGatherWarps) {
+    // ------------------------------------------------------------ gather warps
+    // QK stage c: the 64-dim slice c of the unit's 128-head Q block by one TMA
+    // load, and slice c of every selected row by cp.async. PV stage: 64
+    // selected rows x 256 latent dims by cp.async. Rows land in
+    // 128-byte-swizzled operand layouts; -1 slots are zero-filled (their
+    // logits are masked). (Measured on B200: random 16-byte gathers of one
+    // SM scale with the number of threads issuing them and the bytes in
+    // flight, about 33 GB/s from 96 threads and 62 GB/s from 256, while
+    // tile::gather4 and per-row bulk copies are limited by their issue rate.)
+    const int gt = threadIdx.x;
+    constexpr int kQRowStep = kGather / 8;
+    constexpr int kNQ = (TS + kQRowStep - 1) / kQRowStep;
+    const int gcc = gt & 7, gq0 = gt >> 3;
+    // global stage r's copies are in place: every gather thread arrives once;
+    // for QK stages thread 0's arrival also books the TMA bytes of the Q slice
+    auto arrive_stage = [&](int r) {
+      if (gt == 0 && r % C::kNumSt < kQKChunks) mbar_arrive_expect_tx(&full[r % kStages], kHeads * 128);
+      else mbar_arrive(&full[r % kStages]);
+    };
+    // Thread gt holds rows gt and gt + kGather of a unit's selection in
+    // registers; the next unit's are loaded one unit ahead.
+    auto load_rows = [&](int u, int (&v)[2]) {
+      const Unit w = unit_of(a, u);
+      const int tok0 = w.sp * TS;
 #pragma unroll
-    for (int n = 0; n < kNQ; ++n) {
-      const int j = gq0 + kQRowStep * n;
-      qk_tok[n] = j < TS ? idx_s[j] : -1;
-    }
-  }
-  // stage r's copies are in place: every gather thread arrives once; for QK
-  // stages thread 0's arrival also books the TMA bytes of the Q slice
-  auto arrive_stage = [&](int r) {
-    if (gt == 0 && producer && r < kQKChunks) mbar_arrive_expect_tx(&full[r % kStages], kHeads * 128);
-    else mbar_arrive(&full[r % kStages]);
-  };
-  // Gather stages [s0, s1); false if a wait gave up.
-  auto gather = [&](int s0, int s1) -> bool {
-    int s = s0;
+      for (int e = 0; e < 2; ++e) {
+        const int j = gt + e * kGather;
+        int x = -1;
+        if (j < TS && tok0 + j < a.k) {
+          x = a.idx[static_cast<int64_t>(w.b) * a.k + tok0 + j];
+          if (x < -1 || static_cast<int64_t>(x) >= a.N) {  // anything outside [0, N) counts as -1
+            record_status(a.status, IC_ERR_BAD_INDEX);
+            x = -1;
+          }
+        }
+        v[e] = x;
+      }
+    };
+    int cur[2], nxt[2] = {-1, -1};
+    if (blockIdx.x < a.units) load_rows(blockIdx.x, cur);
     bool ok = true;
-    for (; s < s1; ++s) {
-      const int st = s % kStages;
-      if (!mbar_wait(&empty[st], static_cast<uint32_t>((s / kStages) & 1) ^ 1u, abort_flag, a.status)) {
+    int g = 0;  // global stage counter
+    for (int i = 0, u = blockIdx.x; u < a.units && ok; ++i, u += a.ctas) {
+      const Unit w = unit_of(a, u);
+      int32_t* ids = idx_s + (i & 1) * TS;
+      uint32_t* vm = vmask + (i & 1) * (TS / 32);
+      // the softmax of unit i - 2 is done with this buffer's validity bits
+      if (i >= 2 && !mbar_wait(&idx_free[i & 1], static_cast<uint32_t>(((i >> 1) - 1) & 1), abort_flag, a.status)) {
         ok = false;
         break;
       }
-      uint8_t* base = stages + st * C::kStageBytes;
-      const uint32_t base_u = smem_u32(base);
-      if (s < kQKChunks) {
-        // rows past the last query read zeros; rows of a neighbouring query
-        // are never written out
-        if (gt == 0 && producer) tma_load_2d(base, &qmap, &full[st], s * 64, b * a.H + hb * kHeads);
-        const uint32_t kv_u = base_u + kHeads * 128;
 #pragma unroll
-        for (int n = 0; n < kNQ; ++n) {
-          const int j = gq0 + kQRowStep * n;
-          if (j < TS) {
-            const int tok = qk_tok[n];
-            const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + s * 64 + gcc * 8 : a.kv;
-            cp_async16(kv_u + sw128_offset(j, gcc), src, tok >= 0 ? 16u : 0u);
-          }
+      for (int e = 0; e < 2; ++e) {
+        const int j0 = warp * 32 + e * kGather;  // warp-uniform
+        if (j0 < TS) {
+          ids[j0 + lane] = cur[e];
+          const uint32_t bal = __ballot_sync(0xffffffffu, cur[e] >= 0);
+          if (lane == 0) vm[j0 >> 5] = bal;
         }
-      } else {
-        const int p = s - kQKChunks;
-        if (p >= kPvSolo) gather_pv_stage<TS, kGather>(base_u, idx_s, kvb, a.kv, gt, p);
-        else if (producer) gather_pv_stage<TS, kProdThreads>(base_u, idx_s, kvb, a.kv, gt, p);
       }
-      cp_async_commit();
-      if (s - s0 >= kLookahead) {
-        cp_async_wait<kLookahead>();
-        fence_proxy_async_smem();
-        arrive_stage(s - kLookahead);
+      mbar_arrive(&idx_ready[i & 1]);
+      if (u + a.ctas < a.units) load_rows(u + a.ctas, nxt);
+      if (!mbar_wait(&idx_ready[i & 1], static_cast<uint32_t>((i >> 1) & 1), abort_flag, a.status)) {
+        ok = false;
+        break;
       }
+      int qk_tok[kNQ];  // this thread's QK rows, the same in all nine QK stages
+#pragma unroll
+      for (int n = 0; n < kNQ; ++n) {
+        const int j = gq0 + kQRowStep * n;
+        qk_tok[n] = j < TS ? ids[j] : -1;
+      }
+      const __nv_bfloat16* kvb = a.kv + static_cast<int64_t>(w.b) * a.kv_batch_stride;
+      for (int s = 0; s < C::kNumSt; ++s, ++g) {
+        const int st = g % kStages;
+        if (!mbar_wait(&empty[st], static_cast<uint32_t>((g / kStages) & 1) ^ 1u, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        uint8_t* base = stages + st * C::kStageBytes;
+        const uint32_t base_u = smem_u32(base);
+        if (s < kQKChunks) {
+          // rows past the last query read zeros; rows of a neighbouring query
+          // are never written out
+          if (gt == 0) tma_load_2d(base, &qmap, &full[st], s * 64, w.b * a.H + w.hb * kHeads);
+          const uint32_t kv_u = base_u + kHeads * 128;
+#pragma unroll
+          for (int n = 0; n < kNQ; ++n) {
+            const int j = gq0 + kQRowStep * n;
+            if (j < TS) {
+              const int tok = qk_tok[n];
+              const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + s * 64 + gcc * 8 : a.kv;
+              cp_async16(kv_u + sw128_offset(j, gcc), src, tok >= 0 ? 16u : 0u);
+            }
+          }
+        } else {
+          gather_pv_stage<TS, kGather>(base_u, ids, kvb, a.kv, gt, s - kQKChunks);
+        }
+        cp_async_commit();
+        if (g >= kLookahead) {
+          cp_async_wait<kLookahead>();
+          fence_proxy_async_smem();
+          arrive_stage(g - kLookahead);
+        }
+      }
+      cur[0] = nxt[0];
+      cur[1] = nxt[1];
     }
     // land everything still in flight (also on the abort path)
     cp_async_wait<0>();
     fence_proxy_async_smem();
     if (ok) {
-      for (int r = (s - kLookahead > s0 ? s - kLookahead : s0); r < s; ++r) arrive_stage(r);
-    } else if (gt == 0 && producer) {
-      // wind down: the Q loads issued for QK stages still pending must land
-      for (int r = (s - kStages > s0 ? s - kStages : s0); r < s && r < kQKChunks; ++r)
-        mbar_drain(&full[r % kStages], static_cast<uint32_t>((r / kStages) & 1));
+      for (int r = (g > kLookahead ? g - kLookahead : 0); r < g; ++r) arrive_stage(r);
+    } else if (gt == 0) {
+      // wind down: Q loads of QK stages still pending must land (bounded waits)
+      for (int r = (g > kStages ? g - kStages : 0); r < g; ++r)
+        if (r % C::kNumSt < kQKChunks) mbar_drain(&full[r % kStages], static_cast<uint32_t>((r / kStages) & 1));
     }
-    return ok;
-  };
-
-  if (producer) {
-    gather(0, C::kNumSt);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -256,66 +307,78 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
       const uint32_t p_addr = smem_u32(ps);
       bool ok = true;
-      int s = 0;
-      for (; s < kQKChunks && ok; ++s) {
-        const int st = s % kStages;
-        if (!mbar_wait(&full[st], (s / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
-        fence_proxy_async_smem();
+      int g = 0;
+      for (int i = 0, u = blockIdx.x; u < a.units && ok; ++i, u += a.ctas) {
+        // S lands in columns [0, TS): the previous unit's O_hi must be read out
+        if (i > 0 && !mbar_wait(o_hi_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t base = smem_u32(stages + st * C::kStageBytes);
+        for (int s = 0; s < kQKChunks; ++s, ++g) {
+          const int st = g % kStages;
+          if (!mbar_wait(&full[st], (g / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint32_t base = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tmem_base, sw128_desc(base + kk * 32, 16, 1024),
-                      sw128_desc(base + kHeads * 128 + kk * 32, 16, 1024), idesc_qk, (s | kk) != 0);
-        mma_commit(&empty[st]);
-      }
-      if (ok) {
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem_base, sw128_desc(base + kk * 32, 16, 1024),
+                        sw128_desc(base + kHeads * 128 + kk * 32, 16, 1024), idesc_qk, (s | kk) != 0);
+          mma_commit(&empty[st]);
+        }
+        if (!ok) break;
         mma_commit(s_full);
-        ok = mbar_wait(p_ready, 0, abort_flag, a.status);
+        if (!mbar_wait(p_ready, static_cast<uint32_t>(i & 1), abort_flag, a.status)) { ok = false; break; }
         tc_fence_after();
-      }
-      for (; s < C::kNumSt && ok; ++s) {
-        const int st = s % kStages;
-        if (!mbar_wait(&full[st], (s / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const int p = s - kQKChunks;
-        const int jh = p / (TS / 64), tc = p % (TS / 64);
-        const uint32_t d_tmem = tmem_base + (jh == 0 ? 256u : 0u);
-        const uint32_t base = smem_u32(stages + st * C::kStageBytes);
+        for (int s = kQKChunks; s < C::kNumSt; ++s, ++g) {
+          const int st = g % kStages;
+          if (!mbar_wait(&full[st], (g / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const int p = s - kQKChunks;
+          const int jh = p / (TS / 64), tc = p % (TS / 64);
+          const uint32_t d_tmem = tmem_base + (jh == 0 ? 256u : 0u);
+          const uint32_t base = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(d_tmem, sw128_desc(p_addr + tc * (kHeads * 128) + kk * 32, 16, 1024),
-                      sw128_desc(base + kk * 2048, 8192, 1024), idesc_pv, (tc | kk) != 0);
-        mma_commit(&empty[st]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(d_tmem, sw128_desc(p_addr + tc * (kHeads * 128) + kk * 32, 16, 1024),
+                        sw128_desc(base + kk * 2048, 8192, 1024), idesc_pv, (tc | kk) != 0);
+          mma_commit(&empty[st]);
+        }
+        if (!ok) break;
+        mma_commit(o_full);
       }
-      // o_full also serves as the "all MMAs retired" fence on the abort path
-      mma_commit(o_full);
-      if (!ok) mbar_drain(o_full, 0);
+      // every MMA issued has retired before TMEM is released
+      mma_commit(retire);
+      mbar_drain(retire, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax + output
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;           // head row within the block
-    const int head = hb * kHeads + r;
+    const int r = quad * 32 + lane;  // head row within the block
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const float c2 = a.sm_scale * kLog2e;
-    float mx = -INFINITY, l = 0.f;
-    bool ok = gather(0, kQKChunks);
-    ok = ok && mbar_wait(s_full, 0, abort_flag, a.status);
-    __syncwarp();  // tcgen05.ld is warp-collective
-    if (ok) {
+    uint8_t* tiles = ps + quad * (C::kOutSlots * 4096);
+    bool ok = true;
+    for (int i = 0, u = blockIdx.x; u < a.units && ok; ++i, u += a.ctas) {
+      const Unit w = unit_of(a, u);
+      const uint32_t* vm = vmask + (i & 1) * (TS / 32);
+      ok = mbar_wait(&idx_ready[i & 1], static_cast<uint32_t>((i >> 1) & 1), abort_flag, a.status) &&
+           mbar_wait(s_full, static_cast<uint32_t>(i & 1), abort_flag, a.status);
+      __syncwarp();  // tcgen05.ld is warp-collective
+      if (!ok) break;
       tc_fence_after();
       constexpr int kChunks = TS / 32;  // even: TS is a multiple of 64
       uint32_t rb0[32], rb1[32];
-      // pass 1: row max over valid tokens. Two register buffers: the load of
+      // pass 1: row max over valid rows. Two register buffers: the load of
       // chunk c+1 is in flight while chunk c is reduced; four partial maxima
       // keep the dependency chains short.
       float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      auto max_chunk = [&](const uint32_t (&rv)[32], uint32_t vm) {
+      auto max_chunk = [&](const uint32_t (&rv)[32], uint32_t vmw) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float x = ((vm >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
+          const float x = ((vmw >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
           mp[j & 3] = fmaxf(mp[j & 3], x);
         }
       };
@@ -324,24 +387,24 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
 #pragma unroll 1
       for (int c = 0; c < kChunks; c += 2) {
         tmem_ld32_issue(taddr + (c + 1) * 32, rb1);
-        max_chunk(rb0, vmask[c]);
+        max_chunk(rb0, vm[c]);
         tmem_ld_wait(rb1);
         if (c + 2 < kChunks) tmem_ld32_issue(taddr + (c + 2) * 32, rb0);
-        max_chunk(rb1, vmask[c + 1]);
+        max_chunk(rb1, vm[c + 1]);
         if (c + 2 < kChunks) tmem_ld_wait(rb0);
       }
       const float m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-      mx = m * c2;
-      const float mxe = m == -INFINITY ? 0.f : mx;  // every token invalid: all p = 0
+      const float mx = m * c2;
+      const float mxe = m == -INFINITY ? 0.f : mx;  // every row invalid: all p = 0
       // pass 2: P = 2^(z log2e - max) as bf16 into the A-operand layout; row
       // sum of the rounded values
       float lp[4] = {0.f, 0.f, 0.f, 0.f};
-      auto p_chunk = [&](const uint32_t (&rv)[32], uint32_t vm, int c0) {
+      auto p_chunk = [&](const uint32_t (&rv)[32], uint32_t vmw, int c0) {
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float x0 = ((vm >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
-          const float x1 = ((vm >> (j + 1)) & 1u) ? __uint_as_float(rv[j + 1]) : -INFINITY;
+          const float x0 = ((vmw >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
+          const float x1 = ((vmw >> (j + 1)) & 1u) ? __uint_as_float(rv[j + 1]) : -INFINITY;
           const __nv_bfloat162 pb =
               __floats2bfloat162_rn(ex2_approx(fmaf(x0, c2, -mxe)), ex2_approx(fmaf(x1, c2, -mxe)));
           lp[(j >> 1) & 3] += __low2float(pb) + __high2float(pb);
@@ -359,80 +422,93 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
 #pragma unroll 1
       for (int c = 0; c < kChunks; c += 2) {
         tmem_ld32_issue(taddr + (c + 1) * 32, rb1);
-        p_chunk(rb0, vmask[c], c * 32);
+        p_chunk(rb0, vm[c], c * 32);
         tmem_ld_wait(rb1);
         if (c + 2 < kChunks) tmem_ld32_issue(taddr + (c + 2) * 32, rb0);
-        p_chunk(rb1, vmask[c + 1], (c + 1) * 32);
+        p_chunk(rb1, vm[c + 1], (c + 1) * 32);
         if (c + 2 < kChunks) tmem_ld_wait(rb0);
       }
-      l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
+      const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(p_ready);
-      // the PV stages after the first kPvSolo are gathered by all seven warps
-      ok = gather(kQKChunks, C::kNumSt);
-      ok = ok && mbar_wait(o_full, 0, abort_flag, a.status);
+      mbar_arrive(&idx_free[i & 1]);
+      ok = mbar_wait(o_full, static_cast<uint32_t>(i & 1), abort_flag, a.status);
       __syncwarp();
-    }
-    if (ok) {
+      if (!ok) break;
       tc_fence_after();
-      // O / l (0 when no token was valid) as 32-row x 128-byte tiles in
-      // 128-byte-swizzled shared memory (the stage ring is idle once every
-      // MMA has retired), each written out by one TMA store; heads past H
-      // fall outside the map and are not written. O_lo sits in TMEM columns
-      // [256, 512), O_hi in [0, 256).
+      // O / l (0 when no row was valid) as 32-head x 128-byte tiles in
+      // 128-byte-swizzled shared memory (the P buffer: every PV MMA has
+      // retired), each written out by one TMA store; heads past H fall outside
+      // the map and are not written. O_hi sits in TMEM columns [0, 256) and is
+      // read first, so the next unit's QK can start; O_lo in [256, 512).
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      uint8_t* tiles = stages + quad * (kOutSlots * 4096);
-      const int head0 = hb * kHeads + quad * 32;
-      auto put_tile = [&](int t, const uint32_t (&w)[32], int x) {
-        const int slot = t % kOutSlots;
-        if (t >= kOutSlots) {
-          if (lane == 0) bulk_wait_read<kOutSlots - 1>();  // the slot's previous store has read it
+      const int head0 = w.hb * kHeads + quad * 32;
+      int nt = 0;  // tiles issued by this warp in this unit
+      auto put_tile = [&](const uint32_t (&wd)[32], int x) {
+        const int slot = nt % C::kOutSlots;
+        if (nt >= C::kOutSlots) {
+          if (lane == 0) bulk_wait_read<C::kOutSlots - 1>();  // the slot's previous store has read it
           __syncwarp();
         }
         uint8_t* tile = tiles + slot * 4096;
         const uint32_t tb = smem_u32(tile);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          st_shared_v4(tb + sw128_offset(lane, k), make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]));
+          st_shared_v4(tb + sw128_offset(lane, k),
+                       make_uint4(wd[4 * k], wd[4 * k + 1], wd[4 * k + 2], wd[4 * k + 3]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && head0 < a.H) {
-          tma_store_4d(&omap, tile, x, sp, head0, b);
+          tma_store_4d(&omap, tile, x, w.sp, head0, w.b);
           bulk_commit();
         }
+        ++nt;
       };
-      if (a.out_f32) {
+      // dims [256 t', ...): half 1 (O_hi, columns [0, 256)) first, then half 0
 #pragma unroll 1
-        for (int t = 0; t < 16; ++t) {  // 32 dims per tile
-          uint32_t rv[32];
-          tmem_ld32_issue(taddr + (t < 8 ? 256u + 32u * t : 32u * (t - 8)), rv);
-          tmem_ld_wait(rv);
+      for (int hh = 0; hh < 2; ++hh) {
+        const int half = 1 - hh;
+        const uint32_t col0 = half ? 0u : 256u;
+        if (a.out_f32) {
+#pragma unroll 1
+          for (int t = 0; t < 8; ++t) {  // 32 dims per tile
+            uint32_t rv[32];
+            tmem_ld32_issue(taddr + col0 + 32u * t, rv);
+            tmem_ld_wait(rv);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) rv[j] = __float_as_uint(__uint_as_float(rv[j]) * inv_l);
-          put_tile(t, rv, 32 * t);
+            for (int j = 0; j < 32; ++j) rv[j] = __float_as_uint(__uint_as_float(rv[j]) * inv_l);
+            put_tile(rv, half * 256 + 32 * t);
+          }
+        } else {
+#pragma unroll 1
+          for (int t = 0; t < 4; ++t) {  // 64 dims per tile
+            uint32_t rv[64];
+            tmem_ld64_issue(taddr + col0 + 64u * t, rv);
+            tmem_ld_wait64(rv);
+            uint32_t wd[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              wd[j] = pack_bf16x2(__uint_as_float(rv[2 * j]) * inv_l, __uint_as_float(rv[2 * j + 1]) * inv_l);
+            put_tile(wd, half * 256 + 64 * t);
+          }
         }
-      } else {
-#pragma unroll 1
-        for (int t = 0; t < 8; ++t) {  // 64 dims per tile
-          uint32_t rv[64];
-          tmem_ld64_issue(taddr + (t < 4 ? 256u + 64u * t : 64u * (t - 4)), rv);
-          tmem_ld_wait64(rv);
-          uint32_t w[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            w[j] = pack_bf16x2(__uint_as_float(rv[2 * j]) * inv_l, __uint_as_float(rv[2 * j + 1]) * inv_l);
-          put_tile(t, w, 64 * t);
+        if (hh == 0) {
+          tc_fence_before();
+          mbar_arrive(o_hi_free);
         }
       }
-      if (lane == 0) bulk_wait_read<0>();
+      if (lane == 0) bulk_wait_read<0>();  // the tiles (the next unit's P buffer) are read out
       __syncwarp();
+      const int head = w.hb * kHeads + r;
       if (head < a.H) {
-        const int64_t row = (static_cast<int64_t>(b) * a.H + head) * a.splits + sp;
+        const int64_t row = (static_cast<int64_t>(w.b) * a.H + head) * a.splits + w.sp;
         a.part_ml[row * 2 + 0] = mx;
         a.part_ml[row * 2 + 1] = l;
       }
     }
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -576,8 +652,7 @@ cudaError_t launch_ts(const CUtensorMap& qmap, const CUtensorMap& omap, const Ml
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.splits, a.B, (a.H + kHeads - 1) / kHeads);
-  return launch_kernel(kern, grid, dim3(kThreads), C::kSmemBytes, stream, pdl, qmap, omap, a);
+  return launch_kernel(kern, dim3(a.ctas), dim3(kThreads), C::kSmemBytes, stream, pdl, qmap, omap, a);
 }
 
 }  // namespace
