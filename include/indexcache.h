@@ -166,6 +166,14 @@ size_t ic_sparse_mla_workspace_size(int B, int H, int k);
  *   index_buf  [B, topk] int32 device buffer, owned by the caller.
  *   idx_trace  optional [L, B, topk] int32 device buffer: if not NULL, the
  *              index buffer each layer attended over is copied there.
+ *
+ * Streaming inputs (no counterpart in the pages): a layer's wait_event, if
+ * not NULL, is a cudaEvent_t (cast to void*) owned by the caller; the call
+ * makes `stream` wait on it (cudaStreamWaitEvent) before the layer's first
+ * kernel. A caller that uploads each layer's queries and gates on a copy
+ * stream and records one event per layer lets layer l run while later
+ * layers' inputs are still in flight. A failed wait returns IC_ERR_CUDA
+ * (earlier layers stay enqueued).
  * ------------------------------------------------------------------------- */
 typedef struct {
   int B;                       /* queries */
@@ -193,6 +201,7 @@ typedef struct {
   const void* gate;      /* [B, H, 512] bf16 or NULL */
   void* out;             /* [B, H, 512] out_dtype */
   float* lse;            /* [B, H] fp32 or NULL */
+  void* wait_event;      /* cudaEvent_t to wait on before the layer, or NULL */
 } ic_layer_t;
 
 ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule,

@@ -71,7 +71,7 @@ class ic_stack_shape_t(ctypes.Structure):
 class ic_layer_t(ctypes.Structure):
     _fields_ = [
         ("q_idx", _p), ("w", _p), ("k_idx", _p), ("k_scale", _p), ("q", _p), ("kv", _p), ("sink", _p),
-        ("gate", _p), ("out", _p), ("lse", _p),
+        ("gate", _p), ("out", _p), ("lse", _p), ("wait_event", _p),
     ]
 
 

@@ -406,6 +406,10 @@ ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule
   bool after_kernel = false;
   for (int l = 0; l < L; ++l) {
     const ic_layer_t& y = layers[l];
+    if (y.wait_event) {
+      if (cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(y.wait_event), 0) != cudaSuccess) return IC_ERR_CUDA;
+      after_kernel = false;
+    }
     if (schedule[l] == 'F') {
       g_launches = 0;
       ic_status_t r = indexer_impl(y.q_idx, y.w, y.k_idx, y.k_scale, s.k_dtype, s.B, s.H_I, s.d_I, s.N,

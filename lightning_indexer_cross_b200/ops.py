@@ -148,6 +148,19 @@ class LayerStack:
         self.trace = torch.empty((self.L, B, topk), dtype=torch.int32, device=dev) if trace else None
         self.ws = new_workspace(_abi.ic_layer_stack_workspace_size(sh), dev)
 
+    def set_wait_events(self, events: Optional[Sequence] = None) -> None:
+        """Per-layer ``torch.cuda.Event`` objects (or None entries) that each
+        step waits on before the layer's first kernel, e.g. events recorded
+        after that layer's inputs were copied on another stream. ``None``
+        clears them. Each event is recorded once here so that it has a
+        handle; the caller re-records it every step."""
+        for l in range(self.L):
+            e = None if events is None else events[l]
+            if e is not None and not e.cuda_event:
+                e.record()
+            self.table[l].wait_event = None if e is None else e.cuda_event
+        self._events = events  # keep the events alive while the table points at them
+
     def step(self, stream=None) -> int:
         """Enqueue one decode step; returns the number of kernels enqueued."""
         _abi.ic_layer_stack(self.table, self.L, self.schedule, self.shape, _ptr(self.index_buf), _ptr(self.trace),

@@ -127,3 +127,12 @@ def test_ops_refuse_cpu_tensors(abi):
     q = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.indexer_score(q, torch.zeros(1, 4), torch.zeros(1, 10, 64, dtype=torch.bfloat16))
+
+
+def test_layer_struct_matches_header(abi):
+    """ic_layer_t in the binding has the header's fields, in order."""
+    text = open(os.path.join(ROOT, "include", "indexcache.h")).read()
+    body = text[text.index("typedef struct {", text.index("ic_stack_shape_t;")):text.index("} ic_layer_t;")]
+    names = re.findall(r"\*?\s*(\w+);", re.sub(r"/\*.*?\*/", "", body, flags=re.S))
+    assert names == [f for f, _ in abi.ic_layer_t._fields_]
+    assert ctypes.sizeof(abi.ic_layer_t) == 8 * len(names)
