@@ -20,8 +20,10 @@
 //   warp 0      TMA producer: 128-key tiles of the key cache into a ring of
 //               shared-memory stages (128-byte swizzle, K-major).
 //   warp 1      TMEM owner and MMA issuer (one elected lane).
-//   warps 2..5  epilogue: TMEM -> registers -> score row; also stage the
+//   warps 2..    epilogue: TMEM -> registers -> score row; also stage the
 //               query group's Q (swizzled, zero-padded heads) and weights.
+//               bf16 keys: warps 2..9, two per TMEM lane quadrant, each
+//               reducing one half of the columns; e4m3 keys: warps 2..5.
 //   warps 6..9  (e4m3 keys only) convert e4m3 tiles to bf16 in shared memory.
 //               tcgen05 kind::f16 needs both operands bf16, and the e4m3 ->
 //               bf16 widening is exact; the per-token scale is applied to the
@@ -49,13 +51,14 @@ struct IdxCfg {
   static constexpr int kStages = FP8 ? 2 : (D_I == 128 ? 4 : 6);  // bf16 stages
   static constexpr int kRawStages = FP8 ? 4 : 0;
   static constexpr int kQBytes = kMaxCols * D_I * 2;
-  // 4 epilogue warps (one per TMEM lane quadrant); e4m3 keys add 4 converter
-  // warps. With 6 warps every thread may hold up to 255 registers, which the
-  // epilogue's 128-register TMEM payload needs.
-  static constexpr int kEpiWarps = 4;
-  static constexpr int kHalves = 1;
+  // bf16 keys: 8 epilogue warps, two per TMEM lane quadrant, each reducing
+  // one half of the columns (two warps per SM sub-partition hide each other's
+  // TMEM-load and FMA latencies). e4m3 keys: 4 epilogue warps (one per
+  // quadrant, whole rows) plus 4 converter warps.
+  static constexpr int kEpiWarps = FP8 ? 4 : 8;
+  static constexpr int kHalves = FP8 ? 1 : 2;
   static constexpr int kEpiThreads = kEpiWarps * 32;
-  static constexpr int kThreads = FP8 ? 320 : 192;
+  static constexpr int kThreads = (kEpiWarp0 + kEpiWarps + (FP8 ? 4 : 0)) * 32;
   // smem layout offsets (from a 1024-aligned base)
   static constexpr int kOffStages = 0;
   static constexpr int kOffRaw = kOffStages + kStages * kTileBytes;
@@ -270,15 +273,23 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
         // 32 columns.
         static_assert(kChunks == 4 || kChunks == 8, "half = 128 or 256 columns");
         constexpr int kLoads = kChunks / 2;  // 64-column loads of this half
+        // whole rows (one warp per quadrant): two loads in flight per wait;
+        // half rows (two warps per quadrant): one load at a time, the other
+        // warp of the sub-partition covers the latency
+        constexpr int kPerWait = C::kHalves == 1 ? 2 : 1;
 #pragma unroll
-        for (int pass = 0; pass < kLoads; pass += 2) {
+        for (int pass = 0; pass < kLoads; pass += kPerWait) {
           const int cA = (kC0 + 2 * pass) * 32, cB = cA + 64;
-          const bool haveA = cA < ncols, haveB = cB < ncols && pass + 1 < kLoads;
-          uint32_t ra[64], rb[64];
+          const bool haveA = cA < ncols, haveB = kPerWait == 2 && cB < ncols && pass + 1 < kLoads;
+          uint32_t ra[64], rb[kPerWait == 2 ? 64 : 1];
           if (haveA) tmem_ld64_issue(taddr + cA, ra);
-          if (haveB) tmem_ld64_issue(taddr + cB, rb);
+          if constexpr (kPerWait == 2) {
+            if (haveB) tmem_ld64_issue(taddr + cB, rb);
+          }
           if (haveA) tmem_ld_wait64(ra);
-          if (haveB) tmem_ld_wait64(rb);
+          if constexpr (kPerWait == 2) {
+            if (haveB) tmem_ld_wait64(rb);
+          }
           auto reduce64 = [&](const uint32_t (&rv)[64], int cbase) {
 #pragma unroll
             for (int j4 = 0; j4 < 16; ++j4) {
@@ -293,7 +304,9 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
             }
           };
           if (haveA) reduce64(ra, (kC0 + 2 * pass) * 32);
-          if (haveB) reduce64(rb, (kC0 + 2 * pass) * 32 + 64);
+          if constexpr (kPerWait == 2) {
+            if (haveB) reduce64(rb, (kC0 + 2 * pass) * 32 + 64);
+          }
         }
         tc_fence_before();
         mbar_arrive(&acc_empty[acc]);
