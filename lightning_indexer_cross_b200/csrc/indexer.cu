@@ -223,14 +223,31 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
         named_bar_sync(1, kNumEpiThreads);
         const int b0 = grp * a.G;
         constexpr int kChunksPerRow = D_I / 8;
-        for (int i = et; i < ncols * kChunksPerRow; i += kNumEpiThreads) {
-          const int r = i / kChunksPerRow;
-          const int c8 = i % kChunksPerRow;
-          const int g = r / HP, h = r % HP, b = b0 + g;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (h < a.H_I && b < a.B)
-            v = *reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * a.H_I + h) * D_I + c8 * 8);
-          st_shared_v4(smem_u32(qs + (c8 >> 3) * (kMaxCols * 128) + sw128_offset(r, c8 & 7)), v);
+        // 16-byte chunks in batches of 8 loads per thread, all issued before
+        // their stores, so one memory latency covers a batch
+        constexpr int kBatch = FP8 ? 2 : 8;
+        const int total = ncols * kChunksPerRow;
+        for (int i0 = et; i0 < total; i0 += kBatch * kNumEpiThreads) {
+          uint4 v[kBatch];
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int i = i0 + k * kNumEpiThreads;
+            v[k] = make_uint4(0, 0, 0, 0);
+            if (i < total) {
+              const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
+              const int g = r / HP, h = r % HP, b = b0 + g;
+              if (h < a.H_I && b < a.B)
+                v[k] = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * a.H_I + h) * D_I + c8 * 8));
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int i = i0 + k * kNumEpiThreads;
+            if (i < total) {
+              const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
+              st_shared_v4(smem_u32(qs + (c8 >> 3) * (kMaxCols * 128) + sw128_offset(r, c8 & 7)), v[k]);
+            }
+          }
         }
         for (int i = et; i < kMaxCols; i += kNumEpiThreads) {
           const int g = i / HP, h = i % HP, b = b0 + g;
