@@ -26,9 +26,12 @@
  *   - Workspaces: size them with the matching *_workspace_size call and
  *     zero a new one once before its first use (the status word must start
  *     at IC_OK). The status word keeps the first device error until
- *     ic_last_device_status reads and clears it; every other byte is
- *     scratch that each call initialises itself. Calls that share a
- *     workspace must not overlap in time on the device.
+ *     ic_last_device_status reads and clears it. The top-k passes keep a few
+ *     control words per row in the workspace that every completed call
+ *     leaves at zero; after a call that reported a device error, zero the
+ *     workspace again before reusing it. Every other byte is scratch that
+ *     each call initialises itself. Calls that share a workspace must not
+ *     overlap in time on the device.
  */
 #ifndef INDEXCACHE_H_
 #define INDEXCACHE_H_
@@ -106,7 +109,7 @@ size_t ic_topk_workspace_size(int B, int64_t N, int k);
  * The pages have no counterpart: this is an interface choice of the library.
  *
  * Same result and limits as ic_topk, but takes no workspace: its scratch is
- * a fixed array inside the library (4 MB on every GPU that loads it, held
+ * a fixed array inside the library (12 MB on every GPU that loads it, held
  * until exit). Meant for code that cannot call cudaMalloc, e.g.
  * enqueueing inside a CUDA-graph capture that forbids allocation, or engine
  * plugins that only receive their input and output buffers.

@@ -140,28 +140,28 @@ TopkLayout topk_layout(int B, int64_t N) {
   // the k-th key's 1/16-octave bin rarely holds more than a few percent of a
   // row; bigger bins fall back to passes over the row itself
   L.cand_cap = static_cast<int>(std::min<int64_t>(N, std::max<int64_t>(4096, N / 16)));
-  // histograms and control words first, so one memset clears both
-  L.hist_off = 0;
-  L.cnt_off = align256(L.hist_off + size_t(B) * 4096 * 4);
-  L.cand_off = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
-  L.total = align256(L.cand_off + size_t(B) * L.cand_cap * 4);
+  L.cnt_off = 0;  // control words: zero between calls
+  L.hist_off = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
+  L.cand_off = align256(L.hist_off + size_t(B) * L.cpr * 4096 * 4);
+  L.ckey_off = align256(L.cand_off + size_t(B) * L.cand_cap * 4);
+  L.total = align256(L.ckey_off + size_t(B) * L.cand_cap * 4);
   return L;
 }
 
 ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_valid, int k, int32_t* idx,
-                      uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream) {
+                      uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream, bool pdl) {
   if (!scores || !idx || !ws) return IC_ERR_INVALID_ARG;
   if (B < 1 || N < 1 || N >= (int64_t(1) << 31) || k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
   if (!aligned16(scores) || !aligned16(idx)) return IC_ERR_INVALID_ARG;
   TopkLayout L = topk_layout(B, N);
   if (ws_bytes < L.total) return IC_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(ws + L.hist_off, 0, L.cand_off - L.hist_off, stream) != cudaSuccess) return IC_ERR_CUDA;
   ic::TopkArgs a{};
   a.scores = scores;
   a.n_valid = n_valid;
   a.idx = idx;
   a.hist = reinterpret_cast<uint32_t*>(ws + L.hist_off);
   a.cand = reinterpret_cast<int32_t*>(ws + L.cand_off);
+  a.cand_key = reinterpret_cast<uint32_t*>(ws + L.ckey_off);
   a.counters = reinterpret_cast<uint32_t*>(ws + L.cnt_off);
   a.cand_cap = L.cand_cap;
   a.status = status;
@@ -171,9 +171,9 @@ ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_va
   a.cpr = L.cpr;
   a.slice = L.slice;
   int launches = 0;
-  cudaError_t e = ic::launch_topk(a, stream, &launches);
+  cudaError_t e = ic::launch_topk(a, stream, pdl, &launches);
   if (e != cudaSuccess) return IC_ERR_CUDA;
-  g_launches += launches + 1;  // + the memset
+  g_launches += launches;
   return IC_OK;
 }
 
@@ -348,7 +348,7 @@ ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_vali
   if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return topk_impl(scores, B, N, n_valid, k, idx, ws + kStatusBytes, ws_bytes - kStatusBytes,
-                   reinterpret_cast<int*>(ws), reinterpret_cast<cudaStream_t>(stream));
+                   reinterpret_cast<int*>(ws), reinterpret_cast<cudaStream_t>(stream), false);
 }
 
 size_t ic_sparse_mla_workspace_size(int B, int H, int k) {
@@ -418,7 +418,8 @@ ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule
       if (r != IC_OK) return r;
       total += g_launches;
       g_launches = 0;
-      r = topk_impl(scores, s.B, s.N, s.n_valid, s.topk, index_buf, ws + SL.topk_off, SL.tk.total, status, st);
+      r = topk_impl(scores, s.B, s.N, s.n_valid, s.topk, index_buf, ws + SL.topk_off, SL.tk.total, status, st,
+                    true);
       if (r != IC_OK) return r;
       total += g_launches;
       after_kernel = true;

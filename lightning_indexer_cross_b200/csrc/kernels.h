@@ -77,8 +77,9 @@ struct TopkArgs {
   const float* scores;      // [B, N]
   const int64_t* n_valid;   // [B] or null
   int32_t* idx;             // [B, k]
-  uint32_t* hist;           // [B][4096] histogram of the top 12 key bits
+  uint32_t* hist;           // [B][cpr][4096] per-CTA histograms of the top 12 key bits
   int32_t* cand;            // [B][cand_cap] candidate positions (the k-th key's bin)
+  uint32_t* cand_key;       // [B][cand_cap] their order-preserving keys
   uint32_t* counters;       // [B][kCtrlWords] per-row control state
   int* status;
   int B;
@@ -88,7 +89,7 @@ struct TopkArgs {
   int64_t slice;            // elements per CTA slice
   int cand_cap;             // candidate buffer entries per row
 };
-cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches);
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, bool pdl, int* launches);
 
 // Scratch layout of the top-k passes for B rows of N scores (byte offsets
 // from the start of the scratch region, which follows the status word).
@@ -96,12 +97,13 @@ struct TopkLayout {
   int cpr;
   int64_t slice;
   int cand_cap;
-  size_t hist_off, cand_off, cnt_off, total;
+  size_t hist_off, cand_off, ckey_off, cnt_off, total;
 };
 TopkLayout topk_layout(int B, int64_t N);
-// Validate, clear the scratch region and enqueue the top-k passes.
+// Validate and enqueue the top-k passes. The control words (cnt_off) must be
+// zero on entry; every call that completes leaves them zero again.
 ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_valid, int k, int32_t* idx,
-                      uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream);
+                      uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream, bool pdl);
 
 struct MlaArgs {
   const __nv_bfloat16* q;    // [B, H, 576]

@@ -4,17 +4,20 @@
 // Radix select on the order-preserving 32-bit key of each fp32 score
 // (negative floats: all bits flipped; others: sign bit set). Two launches,
 // neither of which ever waits on another CTA:
-//   histogram  a 12-bit histogram of key[31:20] over each row's valid
-//              positions (several CTAs per row, merged with atomics).
-//   filter     every CTA finds the bin d1 holding the k-th key from the
-//              row's histogram; keys in bins above d1 are final and are
-//              written straight to the output (compacted per CTA, one atomic
-//              reservation per CTA); keys in bin d1 are candidates, appended
-//              to a per-row buffer. The last CTA of the row (atomic ticket)
-//              resolves the exact k-th key T among the candidates (two more
-//              10-bit digits), writes the candidates above T, and then the
-//              r keys equal to T with the lowest indices -- ties resolve
-//              toward the lower index, so the selected set is deterministic.
+//   histogram  each CTA writes the 12-bit histogram of key[31:20] over its
+//              slice of the row to its own slot; the last CTA of the row
+//              (atomic ticket) sums the slots and picks the bin d1 holding
+//              the k-th key.
+//   filter     keys in bins above d1 are final and are written straight to
+//              the output (compacted per CTA with one warp scan per 128
+//              keys, one atomic reservation per CTA); keys in bin d1 are
+//              candidates, appended with their keys to a per-row buffer. The
+//              last CTA of the row resolves the exact k-th key T among the
+//              candidates (two more 10-bit digits), writes the candidates
+//              above T, and then the r keys equal to T with the lowest
+//              indices -- ties resolve toward the lower index, so the
+//              selected set is deterministic -- and finally zeroes the row's
+//              control words for the next call.
 // If bin d1 holds more candidates than the buffer, the last CTA runs the same
 // two digits over the row itself (correct, slower; only for rows whose scores
 // crowd into one 1/16-octave bin).
@@ -153,6 +156,25 @@ IC_DEV void hist_add(uint32_t* h, uint32_t bin, bool take) {
   if (take) atomicAdd(&h[bin], 1u);
 }
 
+// Append (i, key) to shared lists when `take` (warp-aggregated; all 32 lanes
+// call). Entries past `cap` are not stored but still counted.
+IC_DEV void list_push_key(int32_t* list, uint32_t* keys, uint32_t* count, uint32_t cap, int64_t i, uint32_t key,
+                          bool take) {
+  const uint32_t bal = __ballot_sync(0xffffffffu, take);
+  if (!bal) return;
+  const int lane = threadIdx.x & 31;
+  uint32_t base = 0;
+  if (lane == 0) base = atomicAdd(count, static_cast<uint32_t>(__popc(bal)));
+  base = __shfl_sync(0xffffffffu, base, 0);
+  if (take) {
+    const uint32_t pos = base + __popc(bal & ((1u << lane) - 1u));
+    if (pos < cap) {
+      list[pos] = static_cast<int32_t>(i);
+      keys[pos] = key;
+    }
+  }
+}
+
 // Append i to a shared list when `take` (warp-aggregated; all 32 lanes call).
 // Entries past `cap` are not stored but still counted.
 IC_DEV void list_push(int32_t* list, uint32_t* count, uint32_t cap, int64_t i, bool take) {
@@ -187,10 +209,13 @@ __global__ void __launch_bounds__(kThreads) topk_hist_kernel(const TopkArgs a) {
   if (lo < hi)
     for_slice(a, b, lo, hi, [&](int64_t, uint32_t key, bool valid) { hist_add(sh_hist, key >> 20, valid); });
   __syncthreads();
-  uint32_t* g = a.hist + static_cast<int64_t>(b) * kBins1;
-  for (int j = threadIdx.x; j < kBins1; j += kThreads)
-    if (sh_hist[j]) atomicAdd(g + j, sh_hist[j]);
-  // the last CTA of the row picks the bin of the k-th key once for everyone
+  // this CTA's histogram to its own slot (every bin; no atomics)
+  uint4* slots = reinterpret_cast<uint4*>(a.hist + static_cast<int64_t>(b) * a.cpr * kBins1);
+  constexpr int kVec = kBins1 / 4;  // uint4 per histogram
+  for (int j = threadIdx.x; j < kVec; j += kThreads)
+    slots[static_cast<int64_t>(c) * kVec + j] = reinterpret_cast<const uint4*>(sh_hist)[j];
+  // the last CTA of the row sums the slots and picks the bin of the k-th key
+  // once for everyone
   uint32_t* ctrl = row_ctrl(a, b);
   __threadfence();
   __syncthreads();
@@ -198,7 +223,30 @@ __global__ void __launch_bounds__(kThreads) topk_hist_kernel(const TopkArgs a) {
   __syncthreads();
   if (!sh_last) return;
   __threadfence();
-  for (int j = threadIdx.x; j < kBins1; j += kThreads) sh_hist[j] = __ldcg(g + j);
+  for (int j = threadIdx.x; j < kVec; j += kThreads) {
+    uint4 acc = make_uint4(0, 0, 0, 0);
+    int s0 = 0;
+    for (; s0 + 4 <= a.cpr; s0 += 4) {  // four slots' loads in flight
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldcg(&slots[static_cast<int64_t>(s0 + u) * kVec + j]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc.x += v[u].x;
+        acc.y += v[u].y;
+        acc.z += v[u].z;
+        acc.w += v[u].w;
+      }
+    }
+    for (; s0 < a.cpr; ++s0) {
+      const uint4 v = __ldcg(&slots[static_cast<int64_t>(s0) * kVec + j]);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    reinterpret_cast<uint4*>(sh_hist)[j] = acc;
+  }
   __syncthreads();
   select_digit(sh_hist, kBins1, static_cast<uint32_t>(a.k), &sh_d, &sh_kr, warp_tot);
   if (threadIdx.x == 0) {
@@ -213,6 +261,7 @@ struct FilterShared {
   uint32_t hist[kBins1];
   int32_t above[kLocalCap];
   int32_t cand[kLocalCap];
+  uint32_t cand_key[kLocalCap];
   uint32_t warp_tot[kWarps];
   uint32_t n_above, n_cand, base_above, base_cand;
   int d;
@@ -333,13 +382,85 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
   const int64_t lo = static_cast<int64_t>(c) * a.slice;
   const int64_t hi = lo + a.slice < nv ? lo + a.slice : nv;
   if (lo < hi) {
-    for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
-      const uint32_t bin = key >> 20;
-      // a few percent of the keys reach bin d1: one vote skips the rest
-      if (__ballot_sync(0xffffffffu, valid && bin >= d1) == 0u) return;
-      list_push(sh.above, &sh.n_above, kLocalCap, i, valid && bin > d1);
-      list_push(sh.cand, &sh.n_cand, kLocalCap, i, valid && bin == d1);
-    });
+    const bool vec = ((a.N & 3) == 0) && ((lo & 3) == 0);
+    if (vec) {
+      // four consecutive keys per lane: 4-bit masks of the keys above bin d1
+      // and in bin d1; one vote per 128 keys skips the (common) empty case,
+      // else one warp scan of the packed counts (above | cand << 16) gives
+      // every lane its positions in both lists
+      const float* row = a.scores + static_cast<int64_t>(b) * a.N;
+      const int warp = t >> 5, lane = t & 31;
+      constexpr int kWarpSpan = kUnroll * 128;
+      for (int64_t base = lo + static_cast<int64_t>(warp) * kWarpSpan; base < hi; base += kThreads * 4 * kUnroll) {
+        float4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int64_t i = base + u * 128 + lane * 4;
+          if (i + 3 < hi) {
+            v[u] = __ldcg(reinterpret_cast<const float4*>(row + i));
+          } else {
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < hi) v[u].x = __ldcg(row + i);
+            if (i + 1 < hi) v[u].y = __ldcg(row + i + 1);
+            if (i + 2 < hi) v[u].z = __ldcg(row + i + 2);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int64_t i0 = base + u * 128 + lane * 4;
+          const float f4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          uint32_t kk[4], ma = 0, mc = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kk[e] = score_key(f4[e]);
+            const uint32_t bin = kk[e] >> 20;
+            const bool valid = i0 + e < hi;
+            ma |= (valid && bin > d1) ? (1u << e) : 0u;
+            mc |= (valid && bin == d1) ? (1u << e) : 0u;
+          }
+          if (__ballot_sync(0xffffffffu, (ma | mc) != 0u) == 0u) continue;
+          const uint32_t cnt = static_cast<uint32_t>(__popc(ma)) | (static_cast<uint32_t>(__popc(mc)) << 16);
+          uint32_t incl = cnt;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t n = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += n;
+          }
+          const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+          uint32_t ba = 0, bc = 0;
+          if (lane == 31) {
+            if (tot & 0xffffu) ba = atomicAdd(&sh.n_above, tot & 0xffffu);
+            if (tot >> 16) bc = atomicAdd(&sh.n_cand, tot >> 16);
+          }
+          ba = __shfl_sync(0xffffffffu, ba, 31);
+          bc = __shfl_sync(0xffffffffu, bc, 31);
+          const uint32_t ex = incl - cnt;
+          uint32_t pa = ba + (ex & 0xffffu), pc = bc + (ex >> 16);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if ((ma >> e) & 1u) {
+              if (pa < static_cast<uint32_t>(kLocalCap)) sh.above[pa] = static_cast<int32_t>(i0 + e);
+              ++pa;
+            }
+            if ((mc >> e) & 1u) {
+              if (pc < static_cast<uint32_t>(kLocalCap)) {
+                sh.cand[pc] = static_cast<int32_t>(i0 + e);
+                sh.cand_key[pc] = kk[e];
+              }
+              ++pc;
+            }
+          }
+        }
+      }
+    } else {
+      for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
+        const uint32_t bin = key >> 20;
+        // a few percent of the keys reach bin d1: one vote skips the rest
+        if (__ballot_sync(0xffffffffu, valid && bin >= d1) == 0u) return;
+        list_push(sh.above, &sh.n_above, kLocalCap, i, valid && bin > d1);
+        list_push_key(sh.cand, sh.cand_key, &sh.n_cand, kLocalCap, i, key, valid && bin == d1);
+      });
+    }
   }
   __syncthreads();
   // flush: one reservation per list per CTA; if a shared list overflowed,
@@ -351,6 +472,7 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
   }
   __syncthreads();
   int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
+  uint32_t* ckbuf = a.cand_key + static_cast<int64_t>(b) * a.cand_cap;
   if (na <= static_cast<uint32_t>(kLocalCap) && nc <= static_cast<uint32_t>(kLocalCap)) {
     for (uint32_t j = t; j < na; j += kThreads) {
       const uint32_t gp = sh.base_above + j;
@@ -359,7 +481,10 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
     }
     for (uint32_t j = t; j < nc; j += kThreads) {
       const uint32_t gp = sh.base_cand + j;
-      if (gp < static_cast<uint32_t>(a.cand_cap)) cbuf[gp] = sh.cand[j];
+      if (gp < static_cast<uint32_t>(a.cand_cap)) {
+        cbuf[gp] = sh.cand[j];
+        ckbuf[gp] = sh.cand_key[j];
+      }
     }
   } else {
     __syncthreads();
@@ -388,7 +513,10 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
       }
       if (tc) {
         const uint32_t gp = sh.base_cand + oc + __popc(bc & lt);
-        if (gp < static_cast<uint32_t>(a.cand_cap)) cbuf[gp] = static_cast<int32_t>(i);
+        if (gp < static_cast<uint32_t>(a.cand_cap)) {
+          cbuf[gp] = static_cast<int32_t>(i);
+          ckbuf[gp] = key;
+        }
       }
     });
   }
@@ -399,11 +527,10 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
   __syncthreads();
   if (!sh.last) return;
   __threadfence();
-  const float* row = a.scores + static_cast<int64_t>(b) * a.N;
   if (n_cand_row <= static_cast<uint32_t>(kRegCand * kThreads) &&
       n_cand_row <= static_cast<uint32_t>(a.cand_cap)) {
-    // up to kRegCand candidates per thread, fetched once into registers
-    // (keys re-read from the score row); every digit pass then runs on them
+    // up to kRegCand candidates per thread (positions and keys), fetched once
+    // into registers; every digit pass then runs on them
     const uint32_t n = n_cand_row;
     int32_t ci[kRegCand];
     uint32_t ck[kRegCand];
@@ -411,11 +538,7 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
     for (int u = 0; u < kRegCand; ++u) {
       const uint32_t x = static_cast<uint32_t>(u) * kThreads + t;
       ci[u] = x < n ? __ldcg(cbuf + x) : 0;
-    }
-#pragma unroll
-    for (int u = 0; u < kRegCand; ++u) {
-      const uint32_t x = static_cast<uint32_t>(u) * kThreads + t;
-      ck[u] = x < n ? score_key(__ldcg(row + ci[u])) : 0u;
+      ck[u] = x < n ? __ldcg(ckbuf + x) : 0u;
     }
     resolve_bin(a, b, nv, d1, kr1, n_above, sh, [&](auto&& f) {
 #pragma unroll
@@ -435,11 +558,7 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
         for (int u = 0; u < 8; ++u) {
           const uint32_t x = base + static_cast<uint32_t>(u) * kThreads + t;
           bi[u] = x < n ? __ldcg(cbuf + x) : 0;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t x = base + static_cast<uint32_t>(u) * kThreads + t;
-          bk[u] = x < n ? score_key(__ldcg(row + bi[u])) : 0u;
+          bk[u] = x < n ? __ldcg(ckbuf + x) : 0u;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -451,18 +570,21 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
   } else {
     resolve_bin(a, b, nv, d1, kr1, n_above, sh, [&](auto&& f) { for_slice(a, b, 0, nv, f); });
   }
+  // every CTA of the row is done with the control words: leave them zero
+  __syncthreads();
+  if (t < kCtrlWords) ctrl[t] = 0u;
 }
 
 }  // namespace
 
-cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, int* launches) {
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, bool pdl, int* launches) {
   static bool done[64] = {false};  // one flag set per device
   cudaError_t e = set_smem_once(topk_filter_kernel, static_cast<int>(sizeof(FilterShared)), done);
   if (e != cudaSuccess) return e;
   dim3 grid(a.cpr, a.B);
-  // the histogram pass follows the caller's memset of its counters (no
-  // programmatic overlap); the filter pass overlaps the histogram pass's tail
-  e = launch_kernel(topk_hist_kernel, grid, dim3(kThreads), 0, stream, false, a);
+  // the filter pass overlaps the histogram pass's tail; the histogram pass
+  // overlaps the previous kernel when the caller says one precedes it
+  e = launch_kernel(topk_hist_kernel, grid, dim3(kThreads), 0, stream, pdl, a);
   if (e != cudaSuccess) return e;
   e = launch_kernel(topk_filter_kernel, grid, dim3(kThreads), sizeof(FilterShared), stream, true, a);
   if (e != cudaSuccess) return e;

@@ -13,7 +13,7 @@
 // For them this entry point allocates nothing: it needs only the scores and
 // the output index buffer. Its scratch is g_topk_scratch below, a
 // __device__ array that every GPU which loads this library holds until the
-// process exits (kScratchBytes, 4 MB).
+// process exits (kScratchBytes, 12 MB).
 //
 // Limits. At most IC_TOPK_NOALLOC_MAX_ROWS rows per call (64), and the
 // call's histograms and candidate buffers must fit the array (64 rows of up
@@ -39,7 +39,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = 4 * 1024 * 1024;
+constexpr size_t kScratchBytes = 12 * 1024 * 1024;
 constexpr size_t kStatusBytes = 256;
 
 static __device__ __align__(256) unsigned char g_topk_scratch[kScratchBytes];
@@ -77,8 +77,11 @@ extern "C" ic_status_t ic_topk_noalloc(const float* scores, int B, int64_t N, co
   if (scratch_address(&base) != cudaSuccess) return IC_ERR_CUDA;
   uint8_t* scratch = static_cast<uint8_t*>(base);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the previous call left its contents here: clear the status word too
+  // the status word and the control words start at zero on every call
+  // (a previous call that hit a device error may have left them set)
   if (cudaMemsetAsync(scratch, 0, kStatusBytes, s) != cudaSuccess) return IC_ERR_CUDA;
+  if (cudaMemsetAsync(scratch + kStatusBytes + L.cnt_off, 0, size_t(B) * ic::kCtrlWords * 4, s) != cudaSuccess)
+    return IC_ERR_CUDA;
   return ic::topk_impl(scores, B, N, n_valid, k, idx, scratch + kStatusBytes, kScratchBytes - kStatusBytes,
-                       reinterpret_cast<int*>(scratch), s);
+                       reinterpret_cast<int*>(scratch), s, false);
 }
