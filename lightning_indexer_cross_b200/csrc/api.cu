@@ -137,12 +137,26 @@ TopkLayout topk_layout(int B, int64_t N) {
   cpr = ceil_div<int64_t>(N, slice);
   L.cpr = static_cast<int>(cpr);
   L.slice = slice;
+  // one clustered launch per row (a cluster of c <= 4 CTAs, one per SM, each
+  // holding up to 32768 scores) when the rows keep at least half of the SMs
+  // busy; c grows while the grid still fits one wave
+  L.fused = 0;
+  if ((N & 3) == 0 && N <= 4 * 32768) {
+    int c = 1;
+    while (c < 4 && ceil_div<int64_t>(N, c) > 32768) c *= 2;
+    while (c < 4 && int64_t(B) * c * 2 <= num_sms() && ceil_div<int64_t>(N, c * 2) >= 4096) c *= 2;
+    if (int64_t(B) * c * 2 >= num_sms()) {
+      L.fused = 1;
+      L.cpr = c;
+      L.slice = ceil_div<int64_t>(ceil_div<int64_t>(N, c), 4) * 4;
+    }
+  }
   // the k-th key's 1/16-octave bin rarely holds more than a few percent of a
   // row; bigger bins fall back to passes over the row itself
   L.cand_cap = static_cast<int>(std::min<int64_t>(N, std::max<int64_t>(4096, N / 16)));
   L.cnt_off = 0;  // control words: zero between calls
   L.hist_off = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
-  L.cand_off = align256(L.hist_off + size_t(B) * L.cpr * 4096 * 4);
+  L.cand_off = align256(L.hist_off + size_t(B) * std::max<int64_t>(L.cpr, cpr) * 4096 * 4);
   L.ckey_off = align256(L.cand_off + size_t(B) * L.cand_cap * 4);
   L.total = align256(L.ckey_off + size_t(B) * L.cand_cap * 4);
   return L;
@@ -170,6 +184,7 @@ ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_va
   a.k = k;
   a.cpr = L.cpr;
   a.slice = L.slice;
+  a.fused = L.fused;
   int launches = 0;
   cudaError_t e = ic::launch_topk(a, stream, pdl, &launches);
   if (e != cudaSuccess) return IC_ERR_CUDA;

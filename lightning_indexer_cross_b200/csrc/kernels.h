@@ -49,6 +49,27 @@ inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, 
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// The same with thread-block clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                         cudaStream_t stream, bool pdl, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 struct IndexerArgs {
   const __nv_bfloat16* q;      // [B, H_I, d_I]
   const float* w;              // [B, H_I]
@@ -88,14 +109,16 @@ struct TopkArgs {
   int cpr;                  // CTAs per row
   int64_t slice;            // elements per CTA slice
   int cand_cap;             // candidate buffer entries per row
+  int fused;                // one clustered launch per row (cpr CTAs = one cluster) instead of two
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, bool pdl, int* launches);
 
 // Scratch layout of the top-k passes for B rows of N scores (byte offsets
 // from the start of the scratch region, which follows the status word).
 struct TopkLayout {
-  int cpr;
-  int64_t slice;
+  int cpr;         // CTAs per row
+  int64_t slice;   // scores per CTA
+  int fused;       // one clustered launch (cpr <= 4, slices <= 32768 scores)
   int cand_cap;
   size_t hist_off, cand_off, ckey_off, cnt_off, total;
 };

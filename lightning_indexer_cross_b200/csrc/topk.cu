@@ -353,115 +353,83 @@ IC_DEV void resolve_bin(const TopkArgs& a, int b, int64_t nv, uint32_t d1, uint3
   }
 }
 
-__global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  FilterShared& sh = *reinterpret_cast<FilterShared*>(smem_raw);
-  const int b = blockIdx.y, c = blockIdx.x;
-  const int t = threadIdx.x;
-  pdl_trigger();
-  pdl_wait();
-  int32_t* out = a.idx + static_cast<int64_t>(b) * a.k;
-  const int64_t nv = row_valid(a, b);
-  if (nv <= a.k) {
-    if (c == 0)
-      for (int i = t; i < a.k; i += kThreads) out[i] = i < nv ? i : -1;
-    return;
-  }
-  uint32_t* ctrl = row_ctrl(a, b);
-  // the bin of the k-th key, chosen by the histogram pass
-  const uint32_t d1 = __ldcg(&ctrl[kBin]);
-  const uint32_t kr1 = __ldcg(&ctrl[kBinRank]);        // rank of the k-th key inside bin d1
-  const uint32_t n_cand_row = __ldcg(&ctrl[kBinCount]); // keys in bin d1 (whole row)
-  const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
-  if (t == 0) {
-    sh.n_above = 0;
-    sh.n_cand = 0;
-  }
-  __syncthreads();
-
-  const int64_t lo = static_cast<int64_t>(c) * a.slice;
-  const int64_t hi = lo + a.slice < nv ? lo + a.slice : nv;
-  if (lo < hi) {
-    const bool vec = ((a.N & 3) == 0) && ((lo & 3) == 0);
-    if (vec) {
-      // four consecutive keys per lane: 4-bit masks of the keys above bin d1
-      // and in bin d1; one vote per 128 keys skips the (common) empty case,
-      // else one warp scan of the packed counts (above | cand << 16) gives
-      // every lane its positions in both lists
-      const float* row = a.scores + static_cast<int64_t>(b) * a.N;
-      const int warp = t >> 5, lane = t & 31;
-      constexpr int kWarpSpan = kUnroll * 128;
-      for (int64_t base = lo + static_cast<int64_t>(warp) * kWarpSpan; base < hi; base += kThreads * 4 * kUnroll) {
-        float4 v[kUnroll];
+// Classify keys [lo, hi) of row b against bin d1, four consecutive keys per
+// lane (lo a multiple of 4): 4-bit masks of the keys above bin d1 and in bin
+// d1; one vote per 128 keys skips the (common) empty case, else one warp scan
+// of the packed counts (above | cand << 16) gives every lane its positions in
+// both shared lists. keys4(i) returns the keys of positions i .. i+3 (any
+// value past hi).
+template <typename Keys4>
+IC_DEV void filter_scan4(FilterShared& sh, int64_t lo, int64_t hi, uint32_t d1, Keys4&& keys4) {
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  constexpr int kWarpSpan = kUnroll * 128;
+  for (int64_t base = lo + static_cast<int64_t>(warp) * kWarpSpan; base < hi; base += kThreads * 4 * kUnroll) {
+    uint4 kv[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int64_t i = base + u * 128 + lane * 4;
-          if (i + 3 < hi) {
-            v[u] = __ldcg(reinterpret_cast<const float4*>(row + i));
-          } else {
-            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < hi) v[u].x = __ldcg(row + i);
-            if (i + 1 < hi) v[u].y = __ldcg(row + i + 1);
-            if (i + 2 < hi) v[u].z = __ldcg(row + i + 2);
-          }
+    for (int u = 0; u < kUnroll; ++u) kv[u] = keys4(base + u * 128 + lane * 4);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i0 = base + u * 128 + lane * 4;
+      const int64_t rem = hi - i0;  // valid keys from i0 on
+      const uint32_t kk[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+      uint32_t ma = 0, mc = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t bin = kk[e] >> 20;
+        const bool valid = e < rem;
+        ma |= (valid && bin > d1) ? (1u << e) : 0u;
+        mc |= (valid && bin == d1) ? (1u << e) : 0u;
+      }
+      if (__ballot_sync(0xffffffffu, (ma | mc) != 0u) == 0u) continue;
+      const uint32_t cnt = static_cast<uint32_t>(__popc(ma)) | (static_cast<uint32_t>(__popc(mc)) << 16);
+      uint32_t incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+      }
+      const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+      uint32_t ba = 0, bc = 0;
+      if (lane == 31) {
+        if (tot & 0xffffu) ba = atomicAdd(&sh.n_above, tot & 0xffffu);
+        if (tot >> 16) bc = atomicAdd(&sh.n_cand, tot >> 16);
+      }
+      ba = __shfl_sync(0xffffffffu, ba, 31);
+      bc = __shfl_sync(0xffffffffu, bc, 31);
+      const uint32_t ex = incl - cnt;
+      uint32_t pa = ba + (ex & 0xffffu), pc = bc + (ex >> 16);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if ((ma >> e) & 1u) {
+          if (pa < static_cast<uint32_t>(kLocalCap)) sh.above[pa] = static_cast<int32_t>(i0 + e);
+          ++pa;
         }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-          const int64_t i0 = base + u * 128 + lane * 4;
-          const float f4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-          uint32_t kk[4], ma = 0, mc = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            kk[e] = score_key(f4[e]);
-            const uint32_t bin = kk[e] >> 20;
-            const bool valid = i0 + e < hi;
-            ma |= (valid && bin > d1) ? (1u << e) : 0u;
-            mc |= (valid && bin == d1) ? (1u << e) : 0u;
+        if ((mc >> e) & 1u) {
+          if (pc < static_cast<uint32_t>(kLocalCap)) {
+            sh.cand[pc] = static_cast<int32_t>(i0 + e);
+            sh.cand_key[pc] = kk[e];
           }
-          if (__ballot_sync(0xffffffffu, (ma | mc) != 0u) == 0u) continue;
-          const uint32_t cnt = static_cast<uint32_t>(__popc(ma)) | (static_cast<uint32_t>(__popc(mc)) << 16);
-          uint32_t incl = cnt;
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) {
-            const uint32_t n = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += n;
-          }
-          const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
-          uint32_t ba = 0, bc = 0;
-          if (lane == 31) {
-            if (tot & 0xffffu) ba = atomicAdd(&sh.n_above, tot & 0xffffu);
-            if (tot >> 16) bc = atomicAdd(&sh.n_cand, tot >> 16);
-          }
-          ba = __shfl_sync(0xffffffffu, ba, 31);
-          bc = __shfl_sync(0xffffffffu, bc, 31);
-          const uint32_t ex = incl - cnt;
-          uint32_t pa = ba + (ex & 0xffffu), pc = bc + (ex >> 16);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if ((ma >> e) & 1u) {
-              if (pa < static_cast<uint32_t>(kLocalCap)) sh.above[pa] = static_cast<int32_t>(i0 + e);
-              ++pa;
-            }
-            if ((mc >> e) & 1u) {
-              if (pc < static_cast<uint32_t>(kLocalCap)) {
-                sh.cand[pc] = static_cast<int32_t>(i0 + e);
-                sh.cand_key[pc] = kk[e];
-              }
-              ++pc;
-            }
-          }
+          ++pc;
         }
       }
-    } else {
-      for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
-        const uint32_t bin = key >> 20;
-        // a few percent of the keys reach bin d1: one vote skips the rest
-        if (__ballot_sync(0xffffffffu, valid && bin >= d1) == 0u) return;
-        list_push(sh.above, &sh.n_above, kLocalCap, i, valid && bin > d1);
-        list_push_key(sh.cand, sh.cand_key, &sh.n_cand, kLocalCap, i, key, valid && bin == d1);
-      });
     }
   }
+}
+
+IC_DEV void filter_resolve(const TopkArgs& a, int b, int64_t nv, uint32_t d1, uint32_t kr1, uint32_t n_cand_row,
+                           FilterShared& sh);
+IC_DEV void resolve_candidates(const TopkArgs& a, int b, int64_t nv, uint32_t d1, uint32_t kr1,
+                               uint32_t n_cand_row, FilterShared& sh);
+
+// After the scan of [lo, hi): write this CTA's final keys and candidates out
+// (one reservation per list), take the row's filter ticket, and in the last
+// CTA resolve bin d1 and zero the row's control words.
+IC_DEV void filter_finish(const TopkArgs& a, int b, int64_t nv, int64_t lo, int64_t hi, uint32_t d1, uint32_t kr1,
+                          uint32_t n_cand_row, FilterShared& sh) {
+  const int t = threadIdx.x;
+  int32_t* out = a.idx + static_cast<int64_t>(b) * a.k;
+  uint32_t* ctrl = row_ctrl(a, b);
+  const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
   __syncthreads();
   // flush: one reservation per list per CTA; if a shared list overflowed,
   // the slice is scanned again and written through the reserved ranges
@@ -493,33 +461,46 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
       sh.n_cand = 0;
     }
     __syncthreads();
-    for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
-      const uint32_t bin = key >> 20;
-      const bool ta = valid && bin > d1, tc = valid && bin == d1;
-      const int lane = threadIdx.x & 31;
-      const uint32_t ba = __ballot_sync(0xffffffffu, ta), bc = __ballot_sync(0xffffffffu, tc);
-      uint32_t oa = 0, oc = 0;
-      if (lane == 0) {
-        if (ba) oa = atomicAdd(&sh.n_above, static_cast<uint32_t>(__popc(ba)));
-        if (bc) oc = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bc)));
-      }
-      oa = __shfl_sync(0xffffffffu, oa, 0);
-      oc = __shfl_sync(0xffffffffu, oc, 0);
-      const uint32_t lt = (1u << lane) - 1u;
-      if (ta) {
-        const uint32_t gp = sh.base_above + oa + __popc(ba & lt);
-        if (gp < n_above) out[gp] = static_cast<int32_t>(i);
-        else record_status(a.status, IC_ERR_BAD_INDEX);
-      }
-      if (tc) {
-        const uint32_t gp = sh.base_cand + oc + __popc(bc & lt);
-        if (gp < static_cast<uint32_t>(a.cand_cap)) {
-          cbuf[gp] = static_cast<int32_t>(i);
-          ckbuf[gp] = key;
+    if (lo < hi)
+      for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
+        const uint32_t bin = key >> 20;
+        const bool ta = valid && bin > d1, tc = valid && bin == d1;
+        const int lane = threadIdx.x & 31;
+        const uint32_t ba = __ballot_sync(0xffffffffu, ta), bc = __ballot_sync(0xffffffffu, tc);
+        uint32_t oa = 0, oc = 0;
+        if (lane == 0) {
+          if (ba) oa = atomicAdd(&sh.n_above, static_cast<uint32_t>(__popc(ba)));
+          if (bc) oc = atomicAdd(&sh.n_cand, static_cast<uint32_t>(__popc(bc)));
         }
-      }
-    });
+        oa = __shfl_sync(0xffffffffu, oa, 0);
+        oc = __shfl_sync(0xffffffffu, oc, 0);
+        const uint32_t lt = (1u << lane) - 1u;
+        if (ta) {
+          const uint32_t gp = sh.base_above + oa + __popc(ba & lt);
+          if (gp < n_above) out[gp] = static_cast<int32_t>(i);
+          else record_status(a.status, IC_ERR_BAD_INDEX);
+        }
+        if (tc) {
+          const uint32_t gp = sh.base_cand + oc + __popc(bc & lt);
+          if (gp < static_cast<uint32_t>(a.cand_cap)) {
+            cbuf[gp] = static_cast<int32_t>(i);
+            ckbuf[gp] = key;
+          }
+        }
+      });
   }
+  filter_resolve(a, b, nv, d1, kr1, n_cand_row, sh);
+}
+
+// Take the row's filter ticket (this CTA's keys are written out); the last
+// CTA of the row resolves bin d1 and zeroes the row's control words.
+IC_DEV void filter_resolve(const TopkArgs& a, int b, int64_t nv, uint32_t d1, uint32_t kr1, uint32_t n_cand_row,
+                           FilterShared& sh) {
+  const int t = threadIdx.x;
+  uint32_t* ctrl = row_ctrl(a, b);
+  const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
+  int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
+  uint32_t* ckbuf = a.cand_key + static_cast<int64_t>(b) * a.cand_cap;
   // the last CTA of the row resolves bin d1
   __threadfence();
   __syncthreads();
@@ -527,6 +508,20 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
   __syncthreads();
   if (!sh.last) return;
   __threadfence();
+  resolve_candidates(a, b, nv, d1, kr1, n_cand_row, sh);
+  // every CTA of the row is done with the control words: leave them zero
+  __syncthreads();
+  if (t < kCtrlWords) ctrl[t] = 0u;
+}
+
+// The exact k-th key among the row's candidates of bin d1 (positions and keys
+// in the row's candidate buffers), and the output entries it decides.
+IC_DEV void resolve_candidates(const TopkArgs& a, int b, int64_t nv, uint32_t d1, uint32_t kr1,
+                               uint32_t n_cand_row, FilterShared& sh) {
+  const int t = threadIdx.x;
+  const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
+  int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
+  uint32_t* ckbuf = a.cand_key + static_cast<int64_t>(b) * a.cand_cap;
   if (n_cand_row <= static_cast<uint32_t>(kRegCand * kThreads) &&
       n_cand_row <= static_cast<uint32_t>(a.cand_cap)) {
     // up to kRegCand candidates per thread (positions and keys), fetched once
@@ -570,18 +565,305 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
   } else {
     resolve_bin(a, b, nv, d1, kr1, n_above, sh, [&](auto&& f) { for_slice(a, b, 0, nv, f); });
   }
-  // every CTA of the row is done with the control words: leave them zero
+}
+
+// Rows with n_valid <= k: every valid index, padded with -1 (CTA 0 of the row).
+IC_DEV bool small_row(const TopkArgs& a, int b, int c, int64_t nv) {
+  if (nv > a.k) return false;
+  if (c == 0) {
+    int32_t* out = a.idx + static_cast<int64_t>(b) * a.k;
+    for (int i = threadIdx.x; i < a.k; i += kThreads) out[i] = i < nv ? i : -1;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  FilterShared& sh = *reinterpret_cast<FilterShared*>(smem_raw);
+  const int b = blockIdx.y, c = blockIdx.x;
+  const int t = threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
+  const int64_t nv = row_valid(a, b);
+  if (small_row(a, b, c, nv)) return;
+  uint32_t* ctrl = row_ctrl(a, b);
+  // the bin of the k-th key, chosen by the histogram pass
+  const uint32_t d1 = __ldcg(&ctrl[kBin]);
+  const uint32_t kr1 = __ldcg(&ctrl[kBinRank]);        // rank of the k-th key inside bin d1
+  const uint32_t n_cand_row = __ldcg(&ctrl[kBinCount]); // keys in bin d1 (whole row)
+  if (t == 0) {
+    sh.n_above = 0;
+    sh.n_cand = 0;
+  }
   __syncthreads();
-  if (t < kCtrlWords) ctrl[t] = 0u;
+  const int64_t lo = static_cast<int64_t>(c) * a.slice;
+  const int64_t hi = lo + a.slice < nv ? lo + a.slice : nv;
+  if (lo < hi) {
+    if (((a.N & 3) == 0) && ((lo & 3) == 0)) {
+      const float* row = a.scores + static_cast<int64_t>(b) * a.N;
+      filter_scan4(sh, lo, hi, d1, [&](int64_t i) {
+        float4 v;
+        if (i + 3 < hi) {
+          v = __ldcg(reinterpret_cast<const float4*>(row + i));
+        } else {
+          v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < hi) v.x = __ldcg(row + i);
+          if (i + 1 < hi) v.y = __ldcg(row + i + 1);
+          if (i + 2 < hi) v.z = __ldcg(row + i + 2);
+        }
+        return make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+      });
+    } else {
+      for_slice(a, b, lo, hi, [&](int64_t i, uint32_t key, bool valid) {
+        const uint32_t bin = key >> 20;
+        // a few percent of the keys reach bin d1: one vote skips the rest
+        if (__ballot_sync(0xffffffffu, valid && bin >= d1) == 0u) return;
+        list_push(sh.above, &sh.n_above, kLocalCap, i, valid && bin > d1);
+        list_push_key(sh.cand, sh.cand_key, &sh.n_cand, kLocalCap, i, key, valid && bin == d1);
+      });
+    }
+  }
+  filter_finish(a, b, nv, lo, hi, d1, kr1, n_cand_row, sh);
+}
+
+// ------------------------------------------------------------------ one launch
+// Both passes in one kernel, one thread-block cluster per row (C <= 4 CTAs,
+// one per SM, each a slice of at most kFusedSlice keys kept in shared
+// memory; measured on B200: the CTAs of larger clusters are spread one per SM
+// and the grid then runs in several waves). The CTAs of
+// a row exchange histograms, counts and the chosen bin through distributed
+// shared memory between cluster barriers, so nothing is kept in global memory
+// between calls and no CTA waits on a flag:
+//   1 keys of the slice into shared memory and their 12-bit histogram;
+//   2 CTA r sums bins [r 4096/C, (r+1) 4096/C) over the cluster; every CTA
+//     finds the portion and then the bin d1 holding the k-th key;
+//   3 each CTA counts its keys above d1 and in d1 (one warp reduction per
+//     128 keys), takes its offsets from the lower-ranked CTAs' counts and
+//     writes final keys and candidates straight to their positions;
+//   4 CTA 0 resolves the k-th key among the candidates.
+constexpr int kFusedSlice = 32768;  // keys per CTA slice kept in shared memory
+
+struct FusedShared {
+  FilterShared f;
+  uint32_t part[kBins1];  // this CTA's portion of the row histogram
+  uint32_t portion_total;
+  uint32_t na, nc;        // this CTA's keys above bin d1 / in bin d1
+  uint32_t pq, krp;       // portion holding the k-th key, rank inside it
+  uint32_t wsum[kWarps];
+  __align__(16) uint32_t keys[kFusedSlice + 4];
+};
+
+__global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(const TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  FusedShared& fs = *reinterpret_cast<FusedShared*>(smem_raw);
+  FilterShared& sh = fs.f;
+  const int b = blockIdx.y;
+  const int C = a.cpr;                           // cluster = the row's CTAs
+  const uint32_t r = cluster_ctarank();
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  pdl_trigger();
+  pdl_wait();
+  const int64_t nv = row_valid(a, b);
+  // the whole cluster takes this branch together, before any cluster barrier
+  if (small_row(a, b, static_cast<int>(r), nv)) return;
+  const int64_t lo = static_cast<int64_t>(r) * a.slice;
+  const int64_t hi = lo + a.slice < nv ? lo + a.slice : nv;
+  const int n = lo < hi ? static_cast<int>(hi - lo) : 0;  // <= kFusedSlice
+  for (int j = t; j < kBins1; j += kThreads) sh.hist[j] = 0;
+  __syncthreads();
+  // 1: keys and histogram
+  {
+    const float* row = a.scores + static_cast<int64_t>(b) * a.N + lo;
+    constexpr int kU = 4;
+    for (int j0 = t * 4; j0 < n; j0 += kThreads * 4 * kU) {
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int j = j0 + u * kThreads * 4;
+        if (j + 3 < n) {
+          v[u] = __ldcg(reinterpret_cast<const float4*>(row + j));
+        } else {
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (j < n) v[u].x = __ldcg(row + j);
+          if (j + 1 < n) v[u].y = __ldcg(row + j + 1);
+          if (j + 2 < n) v[u].z = __ldcg(row + j + 2);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int j = j0 + u * kThreads * 4;
+        if (j < n) {
+          const uint4 kv = make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z), score_key(v[u].w));
+          *reinterpret_cast<uint4*>(&fs.keys[j]) = kv;
+          hist_add(sh.hist, kv.x >> 20, true);
+          hist_add(sh.hist, kv.y >> 20, j + 1 < n);
+          hist_add(sh.hist, kv.z >> 20, j + 2 < n);
+          hist_add(sh.hist, kv.w >> 20, j + 3 < n);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  cluster_sync();
+  // 2: this CTA's portion of the row histogram, and its total
+  const int P = kBins1 / C;
+  uint32_t mine = 0;
+  for (int j = t; j < P; j += kThreads) {
+    uint32_t sum = 0;
+    for (int q = 0; q < C; ++q) sum += ld_dsmem_u32(dsmem_addr(&sh.hist[r * P + j], static_cast<uint32_t>(q)));
+    fs.part[j] = sum;
+    mine += sum;
+  }
+  mine = __reduce_add_sync(0xffffffffu, mine);
+  if (lane == 0) fs.wsum[warp] = mine;
+  __syncthreads();
+  if (t == 0) {
+    uint32_t tot = 0;
+    for (int w = 0; w < kWarps; ++w) tot += fs.wsum[w];
+    fs.portion_total = tot;
+  }
+  __syncthreads();
+  cluster_sync();
+  if (t == 0) {
+    // portions in descending bin order: the one holding the k-th largest key
+    uint32_t above = 0, pq = 0, krp = 1;
+    for (int q = C - 1; q >= 0; --q) {
+      const uint32_t tq = ld_dsmem_u32(dsmem_addr(&fs.portion_total, static_cast<uint32_t>(q)));
+      if (above + tq >= static_cast<uint32_t>(a.k)) {
+        pq = static_cast<uint32_t>(q);
+        krp = static_cast<uint32_t>(a.k) - above;
+        break;
+      }
+      above += tq;
+    }
+    fs.pq = pq;
+    fs.krp = krp;
+  }
+  __syncthreads();
+  const uint32_t pq = fs.pq;
+  for (int j = t; j < P; j += kThreads) sh.hist[j] = ld_dsmem_u32(dsmem_addr(&fs.part[j], pq));
+  __syncthreads();
+  select_digit(sh.hist, P, fs.krp, &sh.d, &sh.kr, sh.warp_tot);
+  const uint32_t d1 = pq * static_cast<uint32_t>(P) + static_cast<uint32_t>(sh.d);
+  const uint32_t kr1 = sh.kr;                                     // rank of the k-th key inside bin d1
+  const uint32_t n_cand_row = sh.hist[sh.d];                      // keys in bin d1 (whole row)
+  const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
+  // 3: each lane counts its keys above bin d1 and in bin d1 (packed
+  // above | cand << 16; a lane sees at most kFusedSlice / kThreads keys), one
+  // warp scan and one prefix over the warps and the cluster's lower-ranked
+  // CTAs give every lane its first position in both lists; the second sweep
+  // visits the lane's keys in the same order and writes each one there.
+  constexpr int kWarpKeys = 128 * kUnroll;
+  auto classify = [&](int j0, uint32_t& ma, uint32_t& mc, uint4& kv) {  // keys j0 .. j0+3 of the slice
+    kv = *reinterpret_cast<const uint4*>(&fs.keys[j0]);
+    const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+    ma = mc = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t bin = kk[e] >> 20;
+      const bool valid = j0 + e < n;
+      ma |= (valid && bin > d1) ? (1u << e) : 0u;
+      mc |= (valid && bin == d1) ? (1u << e) : 0u;
+    }
+  };
+  uint32_t lcnt = 0;
+  for (int base = warp * kWarpKeys; base < n; base += kThreads * 4 * kUnroll)
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      uint32_t ma, mc;
+      uint4 kv;
+      classify(base + u * 128 + lane * 4, ma, mc, kv);
+      lcnt += static_cast<uint32_t>(__popc(ma)) | (static_cast<uint32_t>(__popc(mc)) << 16);
+    }
+  uint32_t incl = lcnt;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t m = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += m;
+  }
+  if (lane == 31) fs.wsum[warp] = incl;  // the warp's total
+  __syncthreads();
+  if (t == 0) {
+    uint32_t run = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const uint32_t v = fs.wsum[w];
+      fs.wsum[w] = run;  // exclusive prefix over this CTA's warps
+      run += v;
+    }
+    fs.na = run & 0xffffu;
+    fs.nc = run >> 16;
+  }
+  __syncthreads();
+  cluster_sync();
+  if (t == 0) {
+    uint32_t ba = 0, bc = 0;
+    for (uint32_t q = 0; q < r; ++q) {
+      ba += ld_dsmem_u32(dsmem_addr(&fs.na, q));
+      bc += ld_dsmem_u32(dsmem_addr(&fs.nc, q));
+    }
+    sh.base_above = ba;
+    sh.base_cand = bc;
+  }
+  __syncthreads();
+  {
+    int32_t* out = a.idx + static_cast<int64_t>(b) * a.k;
+    int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
+    uint32_t* ckbuf = a.cand_key + static_cast<int64_t>(b) * a.cand_cap;
+    const uint32_t first = fs.wsum[warp] + incl - lcnt;  // this lane's first positions (packed)
+    uint32_t pa = sh.base_above + (first & 0xffffu), pc = sh.base_cand + (first >> 16);
+    for (int base = warp * kWarpKeys; base < n; base += kThreads * 4 * kUnroll)
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int j0 = base + u * 128 + lane * 4;
+        uint32_t ma, mc;
+        uint4 kv;
+        classify(j0, ma, mc, kv);
+        if ((ma | mc) == 0u) continue;
+        const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int32_t pos = static_cast<int32_t>(lo + j0 + e);
+          if ((ma >> e) & 1u) {
+            if (pa < n_above) out[pa] = pos;
+            else record_status(a.status, IC_ERR_BAD_INDEX);  // cannot happen with consistent counts
+            ++pa;
+          }
+          if ((mc >> e) & 1u) {
+            if (pc < static_cast<uint32_t>(a.cand_cap)) {
+              cbuf[pc] = pos;
+              ckbuf[pc] = kk[e];
+            }
+            ++pc;
+          }
+        }
+      }
+  }
+  // 4: every CTA's writes are visible to CTA 0, and no CTA reads another's
+  // shared memory after this barrier
+  __syncthreads();
+  cluster_sync();
+  if (r != 0) return;
+  resolve_candidates(a, b, nv, d1, kr1, n_cand_row, sh);
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, bool pdl, int* launches) {
-  static bool done[64] = {false};  // one flag set per device
-  cudaError_t e = set_smem_once(topk_filter_kernel, static_cast<int>(sizeof(FilterShared)), done);
-  if (e != cudaSuccess) return e;
   dim3 grid(a.cpr, a.B);
+  cudaError_t e;
+  if (a.fused) {
+    static bool done_c[64] = {false};
+    e = set_smem_once(topk_cluster_kernel, static_cast<int>(sizeof(FusedShared)), done_c);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel_cluster(topk_cluster_kernel, grid, dim3(kThreads), sizeof(FusedShared), stream, pdl,
+                              static_cast<unsigned>(a.cpr), a);
+    if (e != cudaSuccess) return e;
+    *launches += 1;
+    return cudaGetLastError();
+  }
+  static bool done[64] = {false};  // one flag set per device
+  e = set_smem_once(topk_filter_kernel, static_cast<int>(sizeof(FilterShared)), done);
+  if (e != cudaSuccess) return e;
   // the filter pass overlaps the histogram pass's tail; the histogram pass
   // overlaps the previous kernel when the caller says one precedes it
   e = launch_kernel(topk_hist_kernel, grid, dim3(kThreads), 0, stream, pdl, a);

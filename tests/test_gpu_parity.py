@@ -64,6 +64,11 @@ TOPK_CASES = [
     (2, 2048, 2048, False, 0.0, False),
     (1, 70001, 1, False, 0.0, False),
     (3, 9000, 500, True, 0.5, True),
+    # enough rows for the one-launch form (one thread-block cluster per row)
+    (150, 4096, 256, False, 0.0, False),      # clusters of one CTA
+    (40, 20000, 2048, False, 0.0, True),      # two-CTA clusters, causal rows
+    (24, 131072, 2048, True, 0.3, False),     # four-CTA clusters, heavy ties, -inf
+    (20, 131072, 1, False, 0.0, False),
 ]
 
 
