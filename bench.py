@@ -154,7 +154,9 @@ def cpu_tokens_per_s(tf, ta):
 
 
 # ----------------------------------------------------------------------------- dist
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """One process per GPU (torchrun): NCCL between the ranks' GPUs; the CPU
+    tests pass backend="gloo"."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -162,9 +164,13 @@ def dist_setup(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
@@ -175,13 +181,25 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The maximum of a per-rank device time over all ranks."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(rank):
+    """Each rank runs an independent replica of the decode batch."""
+    return 2 + rank
+
+
+def replica_value(world, queries, steps, ms_max):
+    """Whole-job decode tokens/s: every rank's queries over the slowest rank's time."""
+    return world * queries * steps / (ms_max / 1000.0)
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -236,7 +254,7 @@ def run_native(args):
     torch.cuda.set_device(dev)
     hbm_gbs, tf_burst, tf_sust, peak_kind = peaks()
 
-    wl = W.stack(dev, seed=2 + rank, L=L, n_full=N_FULL, B=B, N=N, H_I=H_I, d_I=D_I, topk=TOPK, H=H)
+    wl = W.stack(dev, seed=replica_seed(rank), L=L, n_full=N_FULL, B=B, N=N, H_I=H_I, d_I=D_I, topk=TOPK, H=H)
     st = ops.stack_from_workload(wl, trace=False)
     torch.cuda.synchronize()
 
@@ -291,7 +309,7 @@ def run_native(args):
     ms_max = max_over_ranks(ms, world)
     if st.device_status() != 0:
         raise RuntimeError("device status not OK after the timed steps")
-    value = world * B * args.steps / (ms_max / 1000.0)
+    value = replica_value(world, B, args.steps, ms_max)
 
     # ------------------------------------------------------------------ per-kernel timing
     kern = time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst)
@@ -346,12 +364,11 @@ def run_native(args):
 
 
 def load_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if one exists for
-    the current kernel build; else None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch from the committed ncu summary under profiles/,
+    if one was taken on the current kernel sources; else None."""
+    from lightning_indexer_cross_b200.ncu_summary import read_traffic
     try:
-        d = json.load(open(p))
-        return d.get(kernel)
+        return read_traffic(kernel, os.path.join(ROOT, "profiles"))
     except Exception:
         return None
 
