@@ -520,70 +520,42 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   }
 }
 
-// One warp per (query, head): merge the splits' normalised partials
-// (m, l, O / l), add e^{sink} once to the denominator, normalise, gate, write
-// out and lse. Lane `lane` owns 16 of the 512 output dims: with bf16 partials
-// dims [8 lane, 8 lane + 8) and [256 + 8 lane, 256 + 8 lane + 8) (two 16-byte
-// loads per split), with fp32 partials dims 128 i + 4 lane + [0, 4) for
-// i < 4. Every split of a chunk of CH splits is requested before any is
-// reduced, so one memory latency covers a whole chunk; chunks are merged with
-// a running maximum.
+// One warp, one half of one (query, head) row gw = b H + h: merge the
+// splits' normalised partials (m, l, O / l) over dims [256 half, 256 half +
+// 256), add e^{sink} once to the denominator, normalise, gate, write out (and
+// lse, from half 0). Lane `lane` owns the 8 consecutive dims 256 half +
+// 8 lane + [0, 8): one 16-byte load per split for bf16 partials, two for
+// fp32. Every split of a chunk of CH splits is requested before any is
+// reduced, so one memory latency covers a chunk; chunks are merged with a
+// running maximum.
 template <bool F32>
-IC_DEV int comb_dim(int lane, int e) {
-  if constexpr (F32) return (e >> 2) * 128 + lane * 4 + (e & 3);
-  else return (e >> 3) * 256 + lane * 8 + (e & 7);
-}
-
-template <bool F32>
-__global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
+IC_DEV void combine_half(const MlaArgs& a, int64_t gw, int half, int lane) {
   constexpr int CH = F32 ? 4 : 8;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * 4 + warp;
-  pdl_trigger();
-  pdl_wait();
-  if (gw >= static_cast<int64_t>(a.B) * a.H) return;
+  constexpr int NV = F32 ? 2 : 1;  // 16-byte words per split and lane
   const int h = static_cast<int>(gw % a.H);
   const int S = a.splits;
+  const int d0 = half * 256 + lane * 8;
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + gw * S;
-  // gate logits (independent of the partials)
-  float g[16];
-  if (a.gate) {
-    const __nv_bfloat16* gp = a.gate + gw * kDv;
-#pragma unroll
-    for (int r = 0; r < (F32 ? 4 : 2); ++r) {
-      const int d0 = comb_dim<F32>(lane, r * (F32 ? 4 : 8));
-      if constexpr (F32) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(gp + d0));
-        const uint32_t w[2] = {v.x, v.y};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) g[4 * r + e] = bf16_lane(w[e >> 1], e & 1);
-      } else {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(gp + d0));
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) g[8 * r + e] = bf16_lane(w[e >> 1], e & 1);
-      }
-    }
-  }
+  uint4 graw = make_uint4(0, 0, 0, 0);  // 8 bf16 gate logits, unpacked at the end
+  if (a.gate) graw = __ldg(reinterpret_cast<const uint4*>(a.gate + gw * kDv + d0));
   const float sink2 = a.sink[h] * kLog2e;
   float M = sink2, den = 1.f;  // the sink's term e^{sink - M}, M = sink so far
-  float acc[16];
+  float acc[8];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   for (int s0 = 0; s0 < S; s0 += CH) {
     float2 mlv[CH];
-    uint4 raw[CH][F32 ? 4 : 2];
+    uint4 raw[CH][NV];
 #pragma unroll
     for (int u = 0; u < CH; ++u) {
       if (s0 + u < S) {
         mlv[u] = __ldcg(&ml[s0 + u]);
-        const int64_t rowoff = (gw * S + s0 + u) * kDv;
-#pragma unroll
-        for (int r = 0; r < (F32 ? 4 : 2); ++r) {
-          const int d0 = comb_dim<F32>(lane, r * (F32 ? 4 : 8));
-          raw[u][r] = F32 ? __ldcg(reinterpret_cast<const uint4*>(static_cast<const float*>(a.part_o) + rowoff + d0))
-                          : __ldcg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.part_o) +
-                                                                  rowoff + d0));
+        const int64_t off = (gw * S + s0 + u) * kDv + d0;
+        if constexpr (F32) {
+          raw[u][0] = __ldcg(reinterpret_cast<const uint4*>(static_cast<const float*>(a.part_o) + off));
+          raw[u][NV - 1] = __ldcg(reinterpret_cast<const uint4*>(static_cast<const float*>(a.part_o) + off + 4));
+        } else {
+          raw[u][0] = __ldcg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.part_o) + off));
         }
       } else {
         mlv[u] = make_float2(-INFINITY, 0.f);
@@ -595,53 +567,58 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
     const float sc = exp2f(M - Mc);
     den *= sc;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) acc[e] *= sc;
+    for (int e = 0; e < 8; ++e) acc[e] *= sc;
     M = Mc;
 #pragma unroll
     for (int u = 0; u < CH; ++u) {
-      if (mlv[u].x == -INFINITY) continue;  // no valid token in that split
+      if (mlv[u].x == -INFINITY) continue;  // no valid row in that split
       const float wgt = exp2f(mlv[u].x - Mc) * mlv[u].y;
       den += wgt;
+      if constexpr (F32) {
+        const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                               raw[u][NV - 1].x, raw[u][NV - 1].y, raw[u][NV - 1].z, raw[u][NV - 1].w};
 #pragma unroll
-      for (int r = 0; r < (F32 ? 4 : 2); ++r) {
-        const uint32_t w[4] = {raw[u][r].x, raw[u][r].y, raw[u][r].z, raw[u][r].w};
-        if constexpr (F32) {
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, __uint_as_float(w[e]), acc[e]);
+      } else {
+        const uint32_t w[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[4 * r + e] = fmaf(wgt, __uint_as_float(w[e]), acc[4 * r + e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[8 * r + e] = fmaf(wgt, bf16_lane(w[e >> 1], e & 1), acc[8 * r + e]);
-        }
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, bf16_lane(w[e >> 1], e & 1), acc[e]);
       }
     }
   }
   const float inv = 1.f / den;
-  float o[16];
+  const uint32_t gwd[4] = {graw.x, graw.y, graw.z, graw.w};
+  float o[8];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
+  for (int e = 0; e < 8; ++e) {
     o[e] = acc[e] * inv;
-    if (a.gate) o[e] *= 1.f / (1.f + __expf(-g[e]));
+    if (a.gate) o[e] *= 1.f / (1.f + __expf(-bf16_lane(gwd[e >> 1], e & 1)));
   }
-#pragma unroll
-  for (int r = 0; r < (F32 ? 4 : 2); ++r) {
-    const int d0 = comb_dim<F32>(lane, r * (F32 ? 4 : 8));
-    if (a.out_f32) {
-      float* dst = static_cast<float*>(a.out) + gw * kDv + d0;
-      if constexpr (F32) {
-        *reinterpret_cast<float4*>(dst) = make_float4(o[4 * r], o[4 * r + 1], o[4 * r + 2], o[4 * r + 3]);
-      }
-    } else {
-      if constexpr (!F32) {
-        uint4 pk;
-        pk.x = pack_bf16x2(o[8 * r], o[8 * r + 1]);
-        pk.y = pack_bf16x2(o[8 * r + 2], o[8 * r + 3]);
-        pk.z = pack_bf16x2(o[8 * r + 4], o[8 * r + 5]);
-        pk.w = pack_bf16x2(o[8 * r + 6], o[8 * r + 7]);
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + d0) = pk;
-      }
-    }
+  if (a.out_f32) {
+    float* dst = static_cast<float*>(a.out) + gw * kDv + d0;
+    *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<float4*>(dst + 4) = make_float4(o[4], o[5], o[6], o[7]);
+  } else {
+    uint4 pk;
+    pk.x = pack_bf16x2(o[0], o[1]);
+    pk.y = pack_bf16x2(o[2], o[3]);
+    pk.z = pack_bf16x2(o[4], o[5]);
+    pk.w = pack_bf16x2(o[6], o[7]);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + d0) = pk;
   }
-  if (a.lse && lane == 0) a.lse[gw] = (M + log2f(den)) / kLog2e;
+  if (a.lse && half == 0 && lane == 0) a.lse[gw] = (M + log2f(den)) / kLog2e;
+}
+
+// The split combine: one warp per half of a (query, head) row, after the
+// main kernel has completed.
+__global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t item = static_cast<int64_t>(blockIdx.x) * 4 + warp;  // half-rows
+  pdl_trigger();
+  pdl_wait();
+  if (item >= 2 * static_cast<int64_t>(a.B) * a.H) return;
+  if (a.out_f32) combine_half<true>(a, item >> 1, static_cast<int>(item & 1), lane);
+  else combine_half<false>(a, item >> 1, static_cast<int>(item & 1), lane);
 }
 
 template <int TS>
@@ -675,10 +652,9 @@ cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, 
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  const int64_t warps = static_cast<int64_t>(a.B) * a.H;
+  const int64_t warps = 2 * static_cast<int64_t>(a.B) * a.H;  // one per half row
   const dim3 grid(static_cast<unsigned>((warps + 3) / 4));
-  e = a.out_f32 ? launch_kernel(mla_combine_kernel<true>, grid, dim3(128), 0, stream, true, a)
-                : launch_kernel(mla_combine_kernel<false>, grid, dim3(128), 0, stream, true, a);
+  e = launch_kernel(mla_combine_kernel, grid, dim3(128), 0, stream, true, a);
   if (e != cudaSuccess) return e;
   *launches += 2;
   return cudaGetLastError();
