@@ -371,11 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       tc_fence_after();
       constexpr int kChunks = TS / 32;  // even: TS is a multiple of 64
       uint32_t rb0[32], rb1[32];
-      // pass 1: row max over valid rows. Two register buffers: the load of
-      // chunk c+1 is in flight while chunk c is reduced; four partial maxima
-      // keep the dependency chains short.
-      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      auto max_chunk = [&](const uint32_t (&rv)[32], uint32_t vmw) {
+      // The exponent reference is the max over the first 32-column chunk's
+      // valid entries (one TMEM load), not the row max: P = 2^(z log2e - ref)
+      // then exceeds 1 by at most 2^(row max - ref), and the row max is
+      // tracked on the way. Only if they differ by more than kSafe (log2
+      // units; P stays finite in bf16 and fp32 far beyond, and no valid entry
+      // underflows) is the pass redone with the row max. The partial's (m, l)
+      // use the same reference.
+      constexpr float kSafe = 64.f;
+      float mp[4];
+      auto chunk_max = [&](const uint32_t (&rv)[32], uint32_t vmw) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const float x = ((vmw >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
@@ -384,27 +389,20 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       };
       tmem_ld32_issue(taddr, rb0);
       tmem_ld_wait(rb0);
-#pragma unroll 1
-      for (int c = 0; c < kChunks; c += 2) {
-        tmem_ld32_issue(taddr + (c + 1) * 32, rb1);
-        max_chunk(rb0, vm[c]);
-        tmem_ld_wait(rb1);
-        if (c + 2 < kChunks) tmem_ld32_issue(taddr + (c + 2) * 32, rb0);
-        max_chunk(rb1, vm[c + 1]);
-        if (c + 2 < kChunks) tmem_ld_wait(rb0);
-      }
-      const float m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
-      const float mx = m * c2;
-      const float mxe = m == -INFINITY ? 0.f : mx;  // every row invalid: all p = 0
-      // pass 2: P = 2^(z log2e - max) as bf16 into the A-operand layout; row
-      // sum of the rounded values
-      float lp[4] = {0.f, 0.f, 0.f, 0.f};
+      mp[0] = mp[1] = mp[2] = mp[3] = -INFINITY;
+      chunk_max(rb0, vm[0]);
+      const float m0 = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+      float mxe = m0 == -INFINITY ? 0.f : m0 * c2;
+      float lp[4];
+      // P = 2^(z log2e - mxe) as bf16 into the A-operand layout; row sum of
+      // the rounded values; running row max
       auto p_chunk = [&](const uint32_t (&rv)[32], uint32_t vmw, int c0) {
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float x0 = ((vmw >> j) & 1u) ? __uint_as_float(rv[j]) : -INFINITY;
           const float x1 = ((vmw >> (j + 1)) & 1u) ? __uint_as_float(rv[j + 1]) : -INFINITY;
+          mp[(j >> 1) & 3] = fmaxf(mp[(j >> 1) & 3], fmaxf(x0, x1));
           const __nv_bfloat162 pb =
               __floats2bfloat162_rn(ex2_approx(fmaf(x0, c2, -mxe)), ex2_approx(fmaf(x1, c2, -mxe)));
           lp[(j >> 1) & 3] += __low2float(pb) + __high2float(pb);
@@ -417,17 +415,31 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           st_shared_v4(blk + sw128_offset(r, ch0 + q4),
                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]));
       };
-      tmem_ld32_issue(taddr, rb0);
-      tmem_ld_wait(rb0);
+      float m = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < kChunks; c += 2) {
-        tmem_ld32_issue(taddr + (c + 1) * 32, rb1);
-        p_chunk(rb0, vm[c], c * 32);
-        tmem_ld_wait(rb1);
-        if (c + 2 < kChunks) tmem_ld32_issue(taddr + (c + 2) * 32, rb0);
-        p_chunk(rb1, vm[c + 1], (c + 1) * 32);
-        if (c + 2 < kChunks) tmem_ld_wait(rb0);
+      for (int pass = 0; pass < 2; ++pass) {  // the second pass only if some row needs it (warp-uniform)
+        lp[0] = lp[1] = lp[2] = lp[3] = 0.f;
+        mp[0] = mp[1] = mp[2] = mp[3] = -INFINITY;
+        if (pass > 0) {
+          tmem_ld32_issue(taddr, rb0);
+          tmem_ld_wait(rb0);
+        }
+#pragma unroll 1
+        for (int c = 0; c < kChunks; c += 2) {
+          tmem_ld32_issue(taddr + (c + 1) * 32, rb1);
+          p_chunk(rb0, vm[c], c * 32);
+          tmem_ld_wait(rb1);
+          if (c + 2 < kChunks) tmem_ld32_issue(taddr + (c + 2) * 32, rb0);
+          p_chunk(rb1, vm[c + 1], (c + 1) * 32);
+          if (c + 2 < kChunks) tmem_ld_wait(rb0);
+        }
+        m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+        // (two-sided: with no valid entry in the first chunk the reference is 0)
+        const bool redo = m != -INFINITY && fabsf(m * c2 - mxe) > kSafe;
+        if (!__any_sync(0xffffffffu, redo)) break;
+        if (redo) mxe = m * c2;
       }
+      const float mx = m == -INFINITY ? -INFINITY : mxe;  // every row invalid: all p = 0
       const float l = (lp[0] + lp[1]) + (lp[2] + lp[3]);
       tc_fence_before();
       fence_proxy_async_smem();

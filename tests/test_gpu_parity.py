@@ -138,6 +138,42 @@ def test_sparse_mla_all_padding_gives_zero_and_sink_lse(cuda_dev):
     torch.testing.assert_close(lse, sink.unsqueeze(0).expand(2, -1).contiguous(), rtol=1e-5, atol=1e-5)
 
 
+def test_sparse_mla_very_negative_logits_after_an_empty_first_chunk(cuda_dev):
+    """Every selected row equal to v, q = -c v with logits of about -200 and a
+    sink of -1000: the softmax is uniform over the valid rows, so the output is
+    v. The first 64 selected slots are -1, so the exponent reference cannot
+    come from them; exponents taken against 0 would underflow to an empty row."""
+    B, N, H, k = 2, 3000, 128, 512
+    g = torch.Generator(device=cuda_dev).manual_seed(31)
+    v = torch.randn(576, generator=g, device=cuda_dev)
+    v = (v / v.norm()).to(torch.bfloat16).float()
+    kv = v.to(torch.bfloat16).expand(1, N, 576).contiguous()
+    sm_scale = 1.0 / 24.0
+    q = (-(200.0 / (sm_scale * float(v.double().pow(2).sum()))) * v).to(torch.bfloat16)
+    q = q.expand(B, H, 576).contiguous()
+    idx = torch.stack([torch.randperm(N, generator=g, device=cuda_dev)[:k] for _ in range(B)]).to(torch.int32)
+    idx[:, :64] = -1
+    sink = torch.full((H,), -1000.0, device=cuda_dev)
+    out, _ = _ops().sparse_mla_decode(q, kv, idx, sink, None, sm_scale=sm_scale, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref, _ = oracle.sparse_mla(q, kv, idx, sink, None, sm_scale)
+    assert float(np.abs(ref).max()) > 0.01  # the reference output is v, not an empty row
+    err = attn_row_error(out, ref)
+    assert err <= ATTN_TOL[torch.float32], f"attention row error {err:.3e}"
+
+
+def test_sparse_mla_wide_logit_spread(cuda_dev):
+    """A large softmax scale spreads the logits far beyond the first chunk's
+    maximum (the exponents are then rebased on the row max)."""
+    q, kv, idx, sink, g = W.attention_case(2, 5000, 128, 1024, shared=True, gate=True, seed=32, device=cuda_dev)
+    out, lse = _ops().sparse_mla_decode(q, kv, idx, sink, g, sm_scale=3.0, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.sparse_mla(q, kv, idx, sink, g, 3.0)
+    err = attn_row_error(out, ref)
+    assert err <= ATTN_TOL[torch.float32], f"attention row error {err:.3e}"
+    np.testing.assert_allclose(lse.double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-2)
+
+
 def test_sparse_mla_bad_index_is_reported_and_skipped(cuda_dev):
     from lightning_indexer_cross_b200 import _abi
     ops = _ops()
