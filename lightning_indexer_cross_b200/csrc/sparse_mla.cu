@@ -27,8 +27,8 @@
 // combine kernel merges the splits, adds e^{sink} once to the denominator,
 // applies the gate and writes out / lse.
 //
-// Warp roles (12 warps): 0-6 gather every stage of every unit (one ring of
-// three stages), 7 issues the MMAs, 8-11 run the softmax and the output.
+// Warp roles (16 warps): 0-10 gather every stage of every unit (one ring of
+// three stages), 11 issues the MMAs, 12-15 run the softmax and the output.
 // Gathers are cp.async (16 B, zero fill for -1 rows) into 128-byte-swizzled
 // stages; the gathering threads fence the async proxy before signalling the
 // MMA. Each unit's row indices are loaded one unit ahead.
@@ -43,16 +43,22 @@ constexpr int kD = 576;
 constexpr int kDv = 512;
 constexpr int kHeads = 128;      // heads per CTA (MMA M)
 constexpr int kQKChunks = kD / 64;
-// 12 warps (three per SM sub-partition, so at most 168 registers per thread):
-// seven gather warps, the MMA issuer, four softmax/output warps (one per TMEM
-// lane quadrant, quadrant = warp % 4)
-constexpr int kGatherWarps = 7;
+// 16 warps in four warpgroups: warps 0-10 gather, warp 11 issues the MMAs,
+// warps 12-15 run the softmax and the output (one per TMEM lane quadrant,
+// quadrant = warp % 4). Launched at 128 registers per thread; warpgroups 0-2
+// drop to kLowRegs and warpgroup 3 rises to kHighRegs. (Measured on B200: a
+// CTA's random 16-byte gathers scale with the threads issuing them, about
+// 51 GB/s from 224 threads and 66 GB/s from 512.)
+constexpr int kGatherWarps = 11;
 constexpr int kGather = kGatherWarps * 32;
-constexpr int kMmaWarp = 7;
-constexpr int kEpiWarp0 = 8;
-constexpr int kThreads = 384;
+constexpr int kMmaWarp = 11;
+constexpr int kEpiWarp0 = 12;
+constexpr int kThreads = 512;
+constexpr int kLaunchRegs = 65536 / kThreads;
+constexpr int kLowRegs = 96;
+constexpr int kHighRegs = 216;
+static_assert(3 * 128 * kLowRegs + 128 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the CTA's");
 constexpr int kStages = 3;
-constexpr int kLookahead = kStages - 1;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int TS>
@@ -180,6 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  if (warp < kEpiWarp0) setmaxnreg_dec<kLowRegs>();
+  else setmaxnreg_inc<kHighRegs>();
 
   if (warp < kGatherWarps) {
     // ------------------------------------------------------------ gather warps
@@ -195,12 +203,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     constexpr int kQRowStep = kGather / 8;
     constexpr int kNQ = (TS + kQRowStep - 1) / kQRowStep;
     const int gcc = gt & 7, gq0 = gt >> 3;
-    // global stage r's copies are in place: every gather thread arrives once;
-    // for QK stages thread 0's arrival also books the TMA bytes of the Q slice
-    auto arrive_stage = [&](int r) {
-      if (gt == 0 && r % C::kNumSt < kQKChunks) mbar_arrive_expect_tx(&full[r % kStages], kHeads * 128);
-      else mbar_arrive(&full[r % kStages]);
-    };
     // Thread gt holds rows gt and gt + kGather of a unit's selection in
     // registers; the next unit's are loaded one unit ahead.
     auto load_rows = [&](int u, int (&v)[2]) {
@@ -265,8 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         const uint32_t base_u = smem_u32(base);
         if (s < kQKChunks) {
           // rows past the last query read zeros; rows of a neighbouring query
-          // are never written out
-          if (gt == 0) tma_load_2d(base, &qmap, &full[st], s * 64, w.b * a.H + w.hb * kHeads);
+          // are never written out. The Q bytes are booked before thread 0's
+          // own arrival can complete the phase.
+          if (gt == 0) {
+            mbar_expect_tx(&full[st], kHeads * 128);
+            tma_load_2d(base, &qmap, &full[st], s * 64, w.b * a.H + w.hb * kHeads);
+          }
           const uint32_t kv_u = base_u + kHeads * 128;
 #pragma unroll
           for (int n = 0; n < kNQ; ++n) {
@@ -280,22 +286,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         } else {
           gather_pv_stage<TS, kGather>(base_u, ids, kvb, a.kv, gt, s - kQKChunks);
         }
-        cp_async_commit();
-        if (g >= kLookahead) {
-          cp_async_wait<kLookahead>();
-          fence_proxy_async_smem();
-          arrive_stage(g - kLookahead);
-        }
+        // this thread's arrival on the stage happens when its copies have
+        // landed; the MMA thread fences the async proxy after its wait
+        cp_async_arrive_noinc(&full[st]);
       }
       cur[0] = nxt[0];
       cur[1] = nxt[1];
     }
     // land everything still in flight (also on the abort path)
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (ok) {
-      for (int r = (g > kLookahead ? g - kLookahead : 0); r < g; ++r) arrive_stage(r);
-    } else if (gt == 0) {
+    cp_async_wait_all();
+    if (!ok && gt == 0) {
       // wind down: Q loads of QK stages still pending must land (bounded waits)
       for (int r = (g > kStages ? g - kStages : 0); r < g; ++r)
         if (r % C::kNumSt < kQKChunks) mbar_drain(&full[r % kStages], static_cast<uint32_t>((r / kStages) & 1));
@@ -641,6 +641,17 @@ cudaError_t launch_ts(const CUtensorMap& qmap, const CUtensorMap& omap, const Ml
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
+  // The register split draws on the registers the CTA is launched with: a
+  // build that launches with fewer than kLaunchRegs per thread would leave
+  // the increase waiting, so it is refused.
+  static int regs = 0;
+  if (regs == 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    regs = fa.numRegs;
+  }
+  if (regs < kLaunchRegs) return cudaErrorInvalidConfiguration;
   return launch_kernel(kern, dim3(a.ctas), dim3(kThreads), C::kSmemBytes, stream, pdl, qmap, omap, a);
 }
 
