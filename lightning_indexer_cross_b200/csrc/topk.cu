@@ -498,9 +498,6 @@ IC_DEV void filter_resolve(const TopkArgs& a, int b, int64_t nv, uint32_t d1, ui
                            FilterShared& sh) {
   const int t = threadIdx.x;
   uint32_t* ctrl = row_ctrl(a, b);
-  const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
-  int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
-  uint32_t* ckbuf = a.cand_key + static_cast<int64_t>(b) * a.cand_cap;
   // the last CTA of the row resolves bin d1
   __threadfence();
   __syncthreads();
@@ -538,6 +535,7 @@ IC_DEV void resolve_candidates(const TopkArgs& a, int b, int64_t nv, uint32_t d1
     resolve_bin(a, b, nv, d1, kr1, n_above, sh, [&](auto&& f) {
 #pragma unroll
       for (int u = 0; u < kRegCand; ++u) {
+        if (static_cast<uint32_t>(u) * kThreads >= n) break;  // the same for every thread
         const uint32_t x = static_cast<uint32_t>(u) * kThreads + t;
         f(static_cast<int64_t>(ci[u]), ck[u], x < n);
       }
@@ -637,15 +635,17 @@ __global__ void __launch_bounds__(kThreads) topk_filter_kernel(const TopkArgs a)
 //   1 keys of the slice into shared memory and their 12-bit histogram;
 //   2 CTA r sums bins [r 4096/C, (r+1) 4096/C) over the cluster; every CTA
 //     finds the portion and then the bin d1 holding the k-th key;
-//   3 each CTA counts its keys above d1 and in d1 (one warp reduction per
-//     128 keys), takes its offsets from the lower-ranked CTAs' counts and
-//     writes final keys and candidates straight to their positions;
+//   3 each CTA counts its keys above d1 and in d1, takes its offsets from the
+//     lower-ranked CTAs' counts and writes final keys and candidates straight
+//     to their positions;
 //   4 CTA 0 resolves the k-th key among the candidates.
 constexpr int kFusedSlice = 32768;  // keys per CTA slice kept in shared memory
+constexpr int kSliceVecs = kFusedSlice / (kThreads * 4);  // float4 loads per thread
+static_assert(kFusedSlice % (kThreads * 4 * kUnroll) == 0, "whole groups per lane");
 
 struct FusedShared {
   FilterShared f;
-  uint32_t part[kBins1];  // this CTA's portion of the row histogram
+  __align__(16) uint32_t part[kBins1];  // this CTA's portion of the row histogram
   uint32_t portion_total;
   uint32_t na, nc;        // this CTA's keys above bin d1 / in bin d1
   uint32_t pq, krp;       // portion holding the k-th key, rank inside it
@@ -671,110 +671,132 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(const TopkArg
   const int n = lo < hi ? static_cast<int>(hi - lo) : 0;  // <= kFusedSlice
   for (int j = t; j < kBins1; j += kThreads) sh.hist[j] = 0;
   __syncthreads();
-  // 1: keys and histogram
+  // 1: keys and histogram; every load of the slice is in flight at once
   {
     const float* row = a.scores + static_cast<int64_t>(b) * a.N + lo;
-    constexpr int kU = 4;
-    for (int j0 = t * 4; j0 < n; j0 += kThreads * 4 * kU) {
-      float4 v[kU];
+    float4 v[kSliceVecs];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int j = j0 + u * kThreads * 4;
-        if (j + 3 < n) {
-          v[u] = __ldcg(reinterpret_cast<const float4*>(row + j));
-        } else {
-          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (j < n) v[u].x = __ldcg(row + j);
-          if (j + 1 < n) v[u].y = __ldcg(row + j + 1);
-          if (j + 2 < n) v[u].z = __ldcg(row + j + 2);
-        }
+    for (int u = 0; u < kSliceVecs; ++u) {
+      const int j = (u * kThreads + t) * 4;
+      if (j + 3 < n) {
+        v[u] = __ldcg(reinterpret_cast<const float4*>(row + j));
+      } else {
+        v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j < n) v[u].x = __ldcg(row + j);
+        if (j + 1 < n) v[u].y = __ldcg(row + j + 1);
+        if (j + 2 < n) v[u].z = __ldcg(row + j + 2);
       }
+    }
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int j = j0 + u * kThreads * 4;
-        if (j < n) {
-          const uint4 kv = make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z), score_key(v[u].w));
-          *reinterpret_cast<uint4*>(&fs.keys[j]) = kv;
-          hist_add(sh.hist, kv.x >> 20, true);
-          hist_add(sh.hist, kv.y >> 20, j + 1 < n);
-          hist_add(sh.hist, kv.z >> 20, j + 2 < n);
-          hist_add(sh.hist, kv.w >> 20, j + 3 < n);
-        }
+    for (int u = 0; u < kSliceVecs; ++u) {
+      const int j = (u * kThreads + t) * 4;
+      if (j < n) {
+        const uint4 kv = make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z), score_key(v[u].w));
+        *reinterpret_cast<uint4*>(&fs.keys[j]) = kv;
+        hist_add(sh.hist, kv.x >> 20, true);
+        hist_add(sh.hist, kv.y >> 20, j + 1 < n);
+        hist_add(sh.hist, kv.z >> 20, j + 2 < n);
+        hist_add(sh.hist, kv.w >> 20, j + 3 < n);
       }
     }
   }
   __syncthreads();
   cluster_sync();
-  // 2: this CTA's portion of the row histogram, and its total
+  // 2: CTA r sums bins [r P, (r+1) P) of the cluster's histograms (16-byte
+  // remote loads, consecutive across lanes) and their total; the portion
+  // holding the k-th key is found from the C totals, and every CTA selects
+  // the bin d1 inside it from that portion's sums
   const int P = kBins1 / C;
-  uint32_t mine = 0;
-  for (int j = t; j < P; j += kThreads) {
-    uint32_t sum = 0;
-    for (int q = 0; q < C; ++q) sum += ld_dsmem_u32(dsmem_addr(&sh.hist[r * P + j], static_cast<uint32_t>(q)));
-    fs.part[j] = sum;
-    mine += sum;
-  }
-  mine = __reduce_add_sync(0xffffffffu, mine);
-  if (lane == 0) fs.wsum[warp] = mine;
-  __syncthreads();
-  if (t == 0) {
-    uint32_t tot = 0;
-    for (int w = 0; w < kWarps; ++w) tot += fs.wsum[w];
-    fs.portion_total = tot;
+  {
+    const uint4* hist4 = reinterpret_cast<const uint4*>(sh.hist);
+    uint32_t mine = 0;
+    for (int j = t; j < P / 4; j += kThreads) {
+      uint4 hv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        hv[q] = q < C ? ld_dsmem_v4(dsmem_addr(&hist4[r * (P / 4) + j], static_cast<uint32_t>(q)))
+                      : make_uint4(0, 0, 0, 0);
+      uint4 sum;
+      sum.x = (hv[0].x + hv[1].x) + (hv[2].x + hv[3].x);
+      sum.y = (hv[0].y + hv[1].y) + (hv[2].y + hv[3].y);
+      sum.z = (hv[0].z + hv[1].z) + (hv[2].z + hv[3].z);
+      sum.w = (hv[0].w + hv[1].w) + (hv[2].w + hv[3].w);
+      reinterpret_cast<uint4*>(fs.part)[j] = sum;
+      mine += (sum.x + sum.y) + (sum.z + sum.w);
+    }
+    mine = __reduce_add_sync(0xffffffffu, mine);
+    if (lane == 0) fs.wsum[warp] = mine;
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t v = lane < kWarps ? fs.wsum[lane] : 0u;
+      v = __reduce_add_sync(0xffffffffu, v);
+      if (lane == 0) fs.portion_total = v;
+    }
   }
   __syncthreads();
   cluster_sync();
-  if (t == 0) {
-    // portions in descending bin order: the one holding the k-th largest key
-    uint32_t above = 0, pq = 0, krp = 1;
-    for (int q = C - 1; q >= 0; --q) {
-      const uint32_t tq = ld_dsmem_u32(dsmem_addr(&fs.portion_total, static_cast<uint32_t>(q)));
-      if (above + tq >= static_cast<uint32_t>(a.k)) {
-        pq = static_cast<uint32_t>(q);
-        krp = static_cast<uint32_t>(a.k) - above;
-        break;
-      }
-      above += tq;
+  if (warp == 0) {
+    // lane q < C: portion q's total; portions in descending bin order, the
+    // one holding the k-th largest key
+    const uint32_t tq = static_cast<uint32_t>(lane) < static_cast<uint32_t>(C)
+                            ? ld_dsmem_u32(dsmem_addr(&fs.portion_total, static_cast<uint32_t>(lane)))
+                            : 0u;
+    uint32_t above = tq;  // inclusive suffix sum over q' >= q
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t n2 = __shfl_down_sync(0xffffffffu, above, off);
+      if (lane + off < 32) above += n2;
     }
-    fs.pq = pq;
-    fs.krp = krp;
+    const uint32_t kk = static_cast<uint32_t>(a.k);
+    const bool holds = lane < C && above - tq < kk && kk <= above;
+    const uint32_t bal = __ballot_sync(0xffffffffu, holds);
+    const int q = bal ? __ffs(bal) - 1 : 0;
+    const uint32_t above_q = __shfl_sync(0xffffffffu, above - tq, q);
+    if (lane == 0) {
+      fs.pq = static_cast<uint32_t>(q);
+      fs.krp = bal ? kk - above_q : 1u;
+    }
   }
   __syncthreads();
   const uint32_t pq = fs.pq;
-  for (int j = t; j < P; j += kThreads) sh.hist[j] = ld_dsmem_u32(dsmem_addr(&fs.part[j], pq));
+  for (int j = t; j < P / 4; j += kThreads)
+    reinterpret_cast<uint4*>(sh.hist)[j] = ld_dsmem_v4(dsmem_addr(&reinterpret_cast<const uint4*>(fs.part)[j], pq));
   __syncthreads();
   select_digit(sh.hist, P, fs.krp, &sh.d, &sh.kr, sh.warp_tot);
   const uint32_t d1 = pq * static_cast<uint32_t>(P) + static_cast<uint32_t>(sh.d);
-  const uint32_t kr1 = sh.kr;                                     // rank of the k-th key inside bin d1
-  const uint32_t n_cand_row = sh.hist[sh.d];                      // keys in bin d1 (whole row)
+  const uint32_t kr1 = sh.kr;                   // rank of the k-th key inside bin d1
+  const uint32_t n_cand_row = sh.hist[sh.d];    // keys in bin d1 (whole row)
   const uint32_t n_above = static_cast<uint32_t>(a.k) - kr1;
-  // 3: each lane counts its keys above bin d1 and in bin d1 (packed
-  // above | cand << 16; a lane sees at most kFusedSlice / kThreads keys), one
-  // warp scan and one prefix over the warps and the cluster's lower-ranked
-  // CTAs give every lane its first position in both lists; the second sweep
-  // visits the lane's keys in the same order and writes each one there.
+  // 3: each lane classifies its keys (groups of four consecutive keys)
+  // against bin d1 -- above: key > the bin's top; candidate: key in the bin --
+  // and keeps one byte of hit bits per group (above | candidate << 4) in
+  // registers. One warp scan of the packed counts (above | cand << 16; a lane
+  // sees at most kFusedSlice / kThreads keys) and a prefix over the warps and
+  // the cluster's lower-ranked CTAs give every lane its first position in
+  // both lists; the second sweep visits only the hit bits, in the same order.
+  const uint32_t cand_lo = d1 << 20, cand_hi = cand_lo | 0xFFFFFu;
+  constexpr int kGroups = kFusedSlice / (kThreads * 4);  // groups of four keys per lane
   constexpr int kWarpKeys = 128 * kUnroll;
-  auto classify = [&](int j0, uint32_t& ma, uint32_t& mc, uint4& kv) {  // keys j0 .. j0+3 of the slice
-    kv = *reinterpret_cast<const uint4*>(&fs.keys[j0]);
-    const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
-    ma = mc = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t bin = kk[e] >> 20;
-      const bool valid = j0 + e < n;
-      ma |= (valid && bin > d1) ? (1u << e) : 0u;
-      mc |= (valid && bin == d1) ? (1u << e) : 0u;
-    }
+  auto group_first = [&](int gi) {  // first key of the lane's group gi (slice-relative)
+    return (gi / kUnroll) * (kThreads * 4 * kUnroll) + warp * kWarpKeys + (gi % kUnroll) * 128 + lane * 4;
   };
+  uint32_t hits[kGroups / 4];
   uint32_t lcnt = 0;
-  for (int base = warp * kWarpKeys; base < n; base += kThreads * 4 * kUnroll)
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      uint32_t ma, mc;
-      uint4 kv;
-      classify(base + u * 128 + lane * 4, ma, mc, kv);
-      lcnt += static_cast<uint32_t>(__popc(ma)) | (static_cast<uint32_t>(__popc(mc)) << 16);
-    }
+  for (int gi = 0; gi < kGroups; ++gi) {
+    const int j0 = group_first(gi);
+    const uint4 kv = *reinterpret_cast<const uint4*>(&fs.keys[j0]);
+    const int rem = n - j0;
+    const uint32_t vmask = rem >= 4 ? 0xFu : (rem > 0 ? (1u << rem) - 1u : 0u);
+    const uint32_t ma = ((kv.x > cand_hi ? 1u : 0u) | (kv.y > cand_hi ? 2u : 0u) | (kv.z > cand_hi ? 4u : 0u) |
+                         (kv.w > cand_hi ? 8u : 0u)) & vmask;
+    const uint32_t mc = (((kv.x - cand_lo) < 0x100000u ? 1u : 0u) | ((kv.y - cand_lo) < 0x100000u ? 2u : 0u) |
+                         ((kv.z - cand_lo) < 0x100000u ? 4u : 0u) | ((kv.w - cand_lo) < 0x100000u ? 8u : 0u)) &
+                        vmask;
+    if (gi % 4 == 0) hits[gi / 4] = 0u;
+    hits[gi / 4] |= (ma | (mc << 4)) << (8 * (gi % 4));
+    lcnt += static_cast<uint32_t>(__popc(ma)) | (static_cast<uint32_t>(__popc(mc)) << 16);
+  }
   uint32_t incl = lcnt;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -795,14 +817,19 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(const TopkArg
   }
   __syncthreads();
   cluster_sync();
-  if (t == 0) {
+  if (warp == 0) {
+    // lane q < r: counts of the lower-ranked CTA q
     uint32_t ba = 0, bc = 0;
-    for (uint32_t q = 0; q < r; ++q) {
-      ba += ld_dsmem_u32(dsmem_addr(&fs.na, q));
-      bc += ld_dsmem_u32(dsmem_addr(&fs.nc, q));
+    if (static_cast<uint32_t>(lane) < r) {
+      ba = ld_dsmem_u32(dsmem_addr(&fs.na, static_cast<uint32_t>(lane)));
+      bc = ld_dsmem_u32(dsmem_addr(&fs.nc, static_cast<uint32_t>(lane)));
     }
-    sh.base_above = ba;
-    sh.base_cand = bc;
+    ba = __reduce_add_sync(0xffffffffu, ba);
+    bc = __reduce_add_sync(0xffffffffu, bc);
+    if (lane == 0) {
+      sh.base_above = ba;
+      sh.base_cand = bc;
+    }
   }
   __syncthreads();
   {
@@ -810,33 +837,63 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(const TopkArg
     int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
     uint32_t* ckbuf = a.cand_key + static_cast<int64_t>(b) * a.cand_cap;
     const uint32_t first = fs.wsum[warp] + incl - lcnt;  // this lane's first positions (packed)
-    uint32_t pa = sh.base_above + (first & 0xffffu), pc = sh.base_cand + (first >> 16);
-    for (int base = warp * kWarpKeys; base < n; base += kThreads * 4 * kUnroll)
+    // This CTA's entries go to [base, base + count) of each list: staged in
+    // shared memory, then copied out with consecutive stores (or stored
+    // directly when a count exceeds the staging lists).
+    const uint32_t na = fs.na, nc = fs.nc;
+    const bool staged = na <= static_cast<uint32_t>(kLocalCap) && nc <= static_cast<uint32_t>(kLocalCap);
+    uint32_t pa = first & 0xffffu, pc = first >> 16;  // positions within this CTA's ranges
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int j0 = base + u * 128 + lane * 4;
-        uint32_t ma, mc;
-        uint4 kv;
-        classify(j0, ma, mc, kv);
-        if ((ma | mc) == 0u) continue;
-        const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int32_t pos = static_cast<int32_t>(lo + j0 + e);
-          if ((ma >> e) & 1u) {
-            if (pa < n_above) out[pa] = pos;
-            else record_status(a.status, IC_ERR_BAD_INDEX);  // cannot happen with consistent counts
-            ++pa;
-          }
-          if ((mc >> e) & 1u) {
-            if (pc < static_cast<uint32_t>(a.cand_cap)) {
-              cbuf[pc] = pos;
-              ckbuf[pc] = kk[e];
-            }
-            ++pc;
+    for (int gi = 0; gi < kGroups; ++gi) {
+      const uint32_t h = (hits[gi / 4] >> (8 * (gi % 4))) & 0xFFu;
+      if (h == 0u) continue;
+      const int j0 = group_first(gi);
+      uint32_t ma = h & 0xFu, mc = h >> 4;
+      while (ma) {
+        const int e = __ffs(ma) - 1;
+        const int32_t pos = static_cast<int32_t>(lo + j0 + e);
+        if (staged) {
+          sh.above[pa] = pos;
+        } else {
+          const uint32_t gp = sh.base_above + pa;
+          if (gp < n_above) out[gp] = pos;
+          else record_status(a.status, IC_ERR_BAD_INDEX);  // cannot happen with consistent counts
+        }
+        ++pa;
+        ma &= ma - 1u;
+      }
+      while (mc) {
+        const int e = __ffs(mc) - 1;
+        const int32_t pos = static_cast<int32_t>(lo + j0 + e);
+        if (staged) {
+          sh.cand[pc] = pos;
+          sh.cand_key[pc] = fs.keys[j0 + e];
+        } else {
+          const uint32_t gp = sh.base_cand + pc;
+          if (gp < static_cast<uint32_t>(a.cand_cap)) {
+            cbuf[gp] = pos;
+            ckbuf[gp] = fs.keys[j0 + e];
           }
         }
+        ++pc;
+        mc &= mc - 1u;
       }
+    }
+    if (staged) {
+      __syncthreads();
+      for (uint32_t j = t; j < na; j += kThreads) {
+        const uint32_t gp = sh.base_above + j;
+        if (gp < n_above) out[gp] = sh.above[j];
+        else record_status(a.status, IC_ERR_BAD_INDEX);  // cannot happen with consistent counts
+      }
+      for (uint32_t j = t; j < nc; j += kThreads) {
+        const uint32_t gp = sh.base_cand + j;
+        if (gp < static_cast<uint32_t>(a.cand_cap)) {
+          cbuf[gp] = sh.cand[j];
+          ckbuf[gp] = sh.cand_key[j];
+        }
+      }
+    }
   }
   // 4: every CTA's writes are visible to CTA 0, and no CTA reads another's
   // shared memory after this barrier
