@@ -241,7 +241,7 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
   if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) || (gate && !aligned16(gate)))
     return IC_ERR_INVALID_ARG;
   MlaLayout L = mla_layout(B, H, k);
-  if (ws_bytes < L.total) return IC_ERR_INVALID_ARG;
+  if (ws_bytes < L.total || !aligned16(ws)) return IC_ERR_INVALID_ARG;
   if (static_cast<int64_t>(B) * H >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return IC_ERR_CUDA;

@@ -177,6 +177,15 @@ IC_DEV void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
       : "memory");
 }
+// Global -> shared contiguous copy (TMA bulk, no tensor map): both addresses
+// 16-byte aligned, bytes a multiple of 16; completes `bytes` transactions on
+// bar.
+IC_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 // Shared -> global tile store of a 4-D tensor map (bulk-group completion);
 // rows outside the map's extent are not written.
 IC_DEV void tma_store_4d(const CUtensorMap* map, const void* src, int x, int y, int z, int w) {
@@ -199,6 +208,12 @@ IC_DEV void tma_prefetch_desc(const CUtensorMap* map) {
 // 16-byte copy global -> shared; src_bytes = 0 fills the destination with zeros.
 IC_DEV void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// The same copy with a hint that L2 fetch the whole 256-byte block around the
+// source from DRAM (the neighbouring bytes are read soon after).
+IC_DEV void cp_async16_l2_256(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
 }
 IC_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 // One arrival on `bar` once every cp.async this thread has issued so far has

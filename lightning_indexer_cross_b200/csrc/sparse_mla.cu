@@ -280,7 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
             if (j < TS) {
               const int tok = qk_tok[n];
               const __nv_bfloat16* src = tok >= 0 ? kvb + static_cast<int64_t>(tok) * kD + s * 64 + gcc * 8 : a.kv;
-              cp_async16(kv_u + sw128_offset(j, gcc), src, tok >= 0 ? 16u : 0u);
+              // a row's slices are read one stage apart: a 256-byte DRAM fetch
+              // brings the next slice into L2 with this one
+              cp_async16_l2_256(kv_u + sw128_offset(j, gcc), src, tok >= 0 ? 16u : 0u);
             }
           }
         } else {
@@ -633,6 +635,166 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const MlaArgs a) {
   else combine_half<false>(a, item >> 1, static_cast<int>(item & 1), lane);
 }
 
+constexpr int kCombThreads = 512;
+constexpr int kCombRowsPerBar = 16;  // one barrier for the CTA's rows
+
+// Row gw from its staged partials prow ([S][512]) and (m, l) pairs mr:
+// dims 8 q + 256 c, c < 2.
+template <bool F32>
+IC_DEV void combine_staged_row(const MlaArgs& a, const uint8_t* prow, const float2* mr, int64_t gw, float sink2,
+                               int q, const uint4 (&graw)[2]) {
+  constexpr int ES = F32 ? 4 : 2;
+  const int S = a.splits;
+  float M = sink2;
+  for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mr[s2].x);
+  float den = exp2f(sink2 - M);
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  // one split's contribution (a split with no valid row has weight 0)
+  auto add_split = [&](int s2) {
+    const float2 v = mr[s2];
+    const float wgt = v.x == -INFINITY ? 0.f : exp2f(v.x - M) * v.y;
+    den += wgt;
+    const uint8_t* ps = prow + static_cast<size_t>(s2) * kDv * ES;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      if constexpr (F32) {
+        const float4 x0 = ld_shared_v4f(ps + (8 * q + 256 * c) * 4);
+        const float4 x1 = ld_shared_v4f(ps + (8 * q + 256 * c) * 4 + 16);
+        const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[8 * c + e] = fmaf(wgt, xv[e], acc[8 * c + e]);
+      } else {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(ps + (8 * q + 256 * c) * 2);
+        const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[8 * c + e] = fmaf(wgt, bf16_lane(wd[e >> 1], e & 1), acc[8 * c + e]);
+      }
+    }
+  };
+  int s2 = 0;
+  for (; s2 + 1 < S; s2 += 2) {
+    add_split(s2);
+    add_split(s2 + 1);
+  }
+  if (s2 < S) add_split(s2);
+  const float inv = 1.f / den;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const uint32_t gwd[4] = {graw[c].x, graw[c].y, graw[c].z, graw[c].w};
+    float o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      o[e] = acc[8 * c + e] * inv;
+      if (a.gate) o[e] *= 1.f / (1.f + __expf(-bf16_lane(gwd[e >> 1], e & 1)));
+    }
+    if (a.out_f32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + gw * kDv + 8 * q + 256 * c);
+      dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+    } else {
+      uint4 pk;
+      pk.x = pack_bf16x2(o[0], o[1]);
+      pk.y = pack_bf16x2(o[2], o[3]);
+      pk.z = pack_bf16x2(o[4], o[5]);
+      pk.w = pack_bf16x2(o[6], o[7]);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + 8 * q + 256 * c) = pk;
+    }
+  }
+  if (a.lse && q == 0) a.lse[gw] = (M + log2f(den)) / kLog2e;
+}
+
+// The split combine with the partials staged by TMA: CTA c takes head rows
+// [c rpc, c rpc + rpc) of all queries (row = b H + h); one bulk copy per 32 KB
+// brings their partials (the S splits of a row are contiguous) into shared
+// memory with no register cost, so every row of the grid is in flight at
+// once (one barrier: per-row-pair barriers measured slower). Thread t
+// serves row t / 32 and dims 8 (t % 32) + 256 c, c < 2 (32 consecutive
+// threads read 512 consecutive bytes of a split row); two splits are reduced
+// per step.
+template <bool F32>
+__global__ void __launch_bounds__(kCombThreads) mla_combine_bulk_kernel(const MlaArgs a, int rpc) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int ES = F32 ? 4 : 2;
+  const int S = a.splits;
+  const int64_t rows = static_cast<int64_t>(a.B) * a.H;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * rpc;
+  const int nrows = static_cast<int>(rows - row0 < rpc ? rows - row0 : rpc);
+  const uint32_t row_bytes = static_cast<uint32_t>(S) * kDv * ES;
+  uint8_t* pbuf = smem;
+  float2* mlb = reinterpret_cast<float2*>(smem + static_cast<size_t>(rpc) * row_bytes);
+  // one barrier per kCombRowsPerBar rows
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(rpc) * row_bytes +
+                                               ((static_cast<size_t>(rpc) * S * 8 + 15) & ~size_t(15)));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 8);
+  const int t = threadIdx.x;
+  const int ngroups = (nrows + kCombRowsPerBar - 1) / kCombRowsPerBar;
+  if (t == 0) {
+    for (int i = 0; i < 8; ++i) mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();
+  if (nrows <= 0) return;
+  if (t == 0) {
+    const uint8_t* src = static_cast<const uint8_t*>(a.part_o) + row0 * row_bytes;
+    for (int gi = 0; gi < ngroups; ++gi) {
+      const int r0 = gi * kCombRowsPerBar;
+      const int nr = nrows - r0 < kCombRowsPerBar ? nrows - r0 : kCombRowsPerBar;
+      const uint32_t bytes = static_cast<uint32_t>(nr) * row_bytes;
+      mbar_arrive_expect_tx(&bars[gi], bytes);
+      const size_t off = static_cast<size_t>(r0) * row_bytes;
+      for (uint32_t o = 0; o < bytes; o += 32768u)
+        bulk_load(pbuf + off + o, src + off + o, bytes - o < 32768u ? bytes - o : 32768u, &bars[gi]);
+    }
+  }
+  const float2* ml = reinterpret_cast<const float2*>(a.part_ml);
+  for (int i = t; i < nrows * S; i += kCombThreads) mlb[i] = __ldcg(&ml[row0 * S + i]);
+  const int r = t >> 5, q = t & 31;
+  const bool active = r < nrows;
+  const int64_t gw = row0 + r;
+  uint4 graw[2];
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    graw[c] = make_uint4(0, 0, 0, 0);
+    if (active && a.gate) graw[c] = __ldg(reinterpret_cast<const uint4*>(a.gate + gw * kDv + 8 * q + 256 * c));
+  }
+  const float sink2 = active ? __ldg(&a.sink[gw % a.H]) * kLog2e : 0.f;
+  __syncthreads();  // (m, l) in shared memory
+  // this row's partials
+  const bool ok = active && mbar_wait(&bars[r / kCombRowsPerBar], 0u, abort_flag, a.status);
+  if (ok) combine_staged_row<F32>(a, pbuf + static_cast<size_t>(r) * row_bytes, mlb + r * S, gw, sink2, q, graw);
+  // every copy has landed (or its wait gave up) before the CTA exits
+  if (t == 0)
+    for (int gi = 0; gi < ngroups; ++gi) mbar_drain(&bars[gi], 0u);
+}
+
+// Rows per CTA of the staged combine: as many as fit two CTAs per SM (at most
+// 16); 0 if one row does not fit.
+int combine_rows_per_cta(int splits, bool f32, size_t* smem_bytes) {
+  static int sm_bytes = 0, reserved = 0;
+  if (sm_bytes == 0) {
+    int dev = 0, v = 0, rsv = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess) v = 0;
+    if (cudaDeviceGetAttribute(&rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) rsv = 1024;
+    reserved = rsv;
+    sm_bytes = v > 0 ? v : 1;
+  }
+  const size_t row_bytes = static_cast<size_t>(splits) * kDv * (f32 ? 4 : 2);
+  const size_t per_row = row_bytes + static_cast<size_t>(splits) * 8;
+  const size_t fixed = 16 + 80;  // (m, l) padding, barriers, abort flag
+  const int64_t usable = static_cast<int64_t>(sm_bytes) / 2 - reserved - static_cast<int64_t>(fixed);
+  int rpc = usable > 0 ? static_cast<int>(static_cast<size_t>(usable) / per_row) : 0;
+  if (rpc > 16) rpc = 16;
+  if (rpc < 1) return 0;
+  *smem_bytes = static_cast<size_t>(rpc) * row_bytes + ((static_cast<size_t>(rpc) * splits * 8 + 15) & ~size_t(15)) + 80;
+  return rpc;
+}
+
 template <int TS>
 cudaError_t launch_ts(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a, cudaStream_t stream,
                       bool pdl) {
@@ -675,9 +837,21 @@ cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, 
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  const int64_t warps = 2 * static_cast<int64_t>(a.B) * a.H;  // one per half row
-  const dim3 grid(static_cast<unsigned>((warps + 3) / 4));
-  e = launch_kernel(mla_combine_kernel, grid, dim3(128), 0, stream, true, a);
+  size_t cbytes = 0;
+  const int rpc = combine_rows_per_cta(a.splits, a.out_f32 != 0, &cbytes);
+  if (rpc > 0) {
+    auto kern = a.out_f32 ? mla_combine_bulk_kernel<true> : mla_combine_bulk_kernel<false>;
+    static bool done_b[2][64] = {{false}};
+    e = set_smem_once(kern, 232448, done_b[a.out_f32 ? 1 : 0]);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = static_cast<int64_t>(a.B) * a.H;
+    const dim3 grid(static_cast<unsigned>((rows + rpc - 1) / rpc));
+    e = launch_kernel(kern, grid, dim3(kCombThreads), cbytes, stream, true, a, rpc);
+  } else {
+    const int64_t warps = 2 * static_cast<int64_t>(a.B) * a.H;  // one per half row
+    const dim3 grid(static_cast<unsigned>((warps + 3) / 4));
+    e = launch_kernel(mla_combine_kernel, grid, dim3(128), 0, stream, true, a);
+  }
   if (e != cudaSuccess) return e;
   *launches += 2;
   return cudaGetLastError();

@@ -114,6 +114,11 @@ MLA_CASES = [
     (2, 2500, 16, 64, False, True, 10, torch.float32),
     (1, 9000, 130, 700, True, False, 0, torch.bfloat16),
     (8, 4000, 128, 2048, False, True, 0, torch.bfloat16),
+    # one query, 64-row units: a head row's partials over 64 / 128 splits do
+    # not fit the shared-memory staged combine, which falls back to the
+    # register-staged one
+    (1, 6000, 128, 4096, True, True, 0, torch.float32),
+    (1, 9000, 64, 8192, False, True, 5, torch.bfloat16),
 ]
 
 
