@@ -112,7 +112,9 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   a.G = per_query ? 1 : std::min(256 / HP, B);
   a.tiles = static_cast<int>(ceil_div<int64_t>(N, 128));
   const int64_t groups = ceil_div<int64_t>(B, a.G);
-  a.total_items = groups * a.tiles;
+  a.groups = static_cast<int>(groups);
+  a.pair = (!fp8 && !per_query && groups >= 2) ? 2 : 1;
+  a.total_items = ceil_div<int64_t>(groups, a.pair) * a.tiles;
   a.per_query = per_query ? 1 : 0;
   const int grid = static_cast<int>(std::min<int64_t>(num_sms(), a.total_items));
   cudaError_t e = ic::launch_indexer(map, a, HP, d_I, fp8, grid, stream, pdl);

@@ -8,7 +8,8 @@
 // Mapping. One tcgen05.mma per 16-wide slice of d_I computes a tile
 //   D[128 keys x n] = K_tile[128 x d_I] . Qg[n x d_I]^T,    n = G * HP
 // where Qg stacks the (padded) heads of G queries that read the same key
-// tile. Keys are the M side, so each TMEM lane holds one key's n head logits
+// tile. With one cache shared by all queries, two such groups (two TMEM
+// accumulators) use every key tile a CTA loads. Keys are the M side, so each TMEM lane holds one key's n head logits
 // and the epilogue thread owning that lane does ReLU, the w_h weighting and
 // the head sum in registers -- no cross-thread reduction. With one cache per
 // query G = 1 (n = HP, the decode case); with one cache shared by many
@@ -21,7 +22,7 @@
 //               shared-memory stages (128-byte swizzle, K-major).
 //   warp 1      TMEM owner and MMA issuer (one elected lane).
 //   warps 2..    epilogue: TMEM -> registers -> score row; also stage the
-//               query group's Q (swizzled, zero-padded heads) and weights.
+//               query groups' Q (swizzled, zero-padded heads) and weights.
 //               bf16 keys: warps 2..9, two per TMEM lane quadrant, each
 //               reducing one half of the columns; e4m3 keys: warps 2..5.
 //   warps 6..9  (e4m3 keys only) convert e4m3 tiles to bf16 in shared memory.
@@ -43,18 +44,24 @@ constexpr int kTileKeys = 128;
 constexpr int kMaxCols = 256;  // MMA N limit for M = 128
 constexpr int kEpiWarp0 = 2;
 
-template <int D_I, bool FP8>
+// PAIR: two query groups (two Q slots, one TMEM accumulator each) share every
+// key tile a CTA loads -- one cache shared by all queries; half the key-tile
+// traffic, two key stages instead of four.
+template <int D_I, bool FP8, bool PAIR>
 struct IdxCfg {
   static constexpr int kBlocks = D_I / 64;                        // 64-element (128 B) swizzle blocks
   static constexpr int kTileBytes = kTileKeys * D_I * 2;          // bf16 tile
   static constexpr int kRawBytes = FP8 ? kTileKeys * D_I : 0;     // e4m3 tile
-  static constexpr int kStages = FP8 ? 2 : (D_I == 128 ? 4 : 6);  // bf16 stages
+  static constexpr int kStages = FP8 ? 2 : (PAIR ? (D_I == 128 ? 2 : 4) : (D_I == 128 ? 4 : 6));  // bf16 stages
   static constexpr int kRawStages = FP8 ? 4 : 0;
-  static constexpr int kQBytes = kMaxCols * D_I * 2;
+  static constexpr int kQSlots = PAIR ? 2 : 1;
+  static constexpr int kQSlotBytes = kMaxCols * D_I * 2;
+  static constexpr int kQBytes = kQSlots * kQSlotBytes;
   // bf16 keys: 8 epilogue warps, two per TMEM lane quadrant, each reducing
   // one half of the columns (two warps per SM sub-partition hide each other's
-  // TMEM-load and FMA latencies). e4m3 keys: 4 epilogue warps (one per
-  // quadrant, whole rows) plus 4 converter warps.
+  // TMEM-load and FMA latencies; measured: four per quadrant at the 96
+  // registers of 18 warps spill and run slower). e4m3 keys: 4 epilogue warps
+  // (one per quadrant, whole rows) plus 4 converter warps.
   static constexpr int kEpiWarps = FP8 ? 4 : 8;
   static constexpr int kHalves = FP8 ? 1 : 2;
   static constexpr int kEpiThreads = kEpiWarps * 32;
@@ -64,17 +71,20 @@ struct IdxCfg {
   static constexpr int kOffRaw = kOffStages + kStages * kTileBytes;
   static constexpr int kOffQ = kOffRaw + kRawStages * kRawBytes;
   static constexpr int kOffW = kOffQ + kQBytes;
-  static constexpr int kOffNv = kOffW + kMaxCols * 4;
-  static constexpr int kOffBar = kOffNv + 16 * 8;
+  static constexpr int kOffNv = kOffW + kQSlots * kMaxCols * 4;
+  static constexpr int kOffBar = kOffNv + kQSlots * 16 * 8;
   static constexpr int kNumBars = 2 * kStages + 2 * kRawStages + 4 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static_assert(!(FP8 && PAIR), "e4m3 keys take one group per tile");
+  static_assert(kSmemBytes <= 232448, "fits one CTA per SM");
 };
 
-template <int D_I, int HP, bool FP8>
-__global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
+template <int D_I, int HP, bool FP8, bool PAIR>
+__global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
-  using C = IdxCfg<D_I, FP8>;
+  using C = IdxCfg<D_I, FP8, PAIR>;
+  constexpr int P = C::kQSlots;  // query groups per work item
   constexpr int GMAX = kMaxCols / HP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -98,7 +108,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   pdl_trigger();
 
-  // This CTA's contiguous share of the (group, tile) work list.
+  // This CTA's contiguous share of the work list: item (pair, tile) covers
+  // query groups P pair .. P pair + P - 1 (fewer at the end) on one key tile.
   const int64_t total = a.total_items;
   const int64_t lo = total * blockIdx.x / gridDim.x;
   const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
@@ -137,7 +148,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
     if (lane == 0) {
       int64_t it = 0;
       for (int64_t wi = lo; wi < hi; ++wi, ++it) {
-        const int grp = static_cast<int>(wi / a.tiles);
+        const int grp = static_cast<int>(wi / a.tiles) * P;  // first group of the item
         const int t = static_cast<int>(wi % a.tiles);
         const int z = a.per_query ? grp : 0;
         if constexpr (!FP8) {
@@ -173,9 +184,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
       const uint32_t q_addr = smem_u32(qs);
       int cur_grp = -1;
       uint32_t q_phase = 0;
-      int64_t it = 0;
-      for (int64_t wi = lo; wi < hi; ++wi, ++it) {
-        const int grp = static_cast<int>(wi / a.tiles);
+      int64_t it = 0, si = 0;  // items; (item, group) sub-items -> accumulator si & 1
+      bool ok = true;
+      for (int64_t wi = lo; wi < hi && ok; ++wi, ++it) {
+        const int grp = static_cast<int>(wi / a.tiles) * P;
+        const int ng = P == 1 ? 1 : (a.groups - grp < P ? a.groups - grp : P);
         if (grp != cur_grp) {
           if (!mbar_wait(q_ready, q_phase, abort_flag, a.status)) break;
           q_phase ^= 1;
@@ -183,22 +196,26 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
         }
         const int st = static_cast<int>(it % C::kStages);
         const uint32_t ph = static_cast<uint32_t>((it / C::kStages) & 1);
-        const int acc = static_cast<int>(it & 1);
-        const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
-        if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status)) break;
         if (!mbar_wait(&full[st], ph, abort_flag, a.status)) break;
-        tc_fence_after();
         const uint32_t a_addr = smem_u32(stages + st * C::kTileBytes);
-        const uint32_t d_tmem = tmem_base + acc * 256;
+        for (int sub = 0; sub < ng; ++sub, ++si) {
+          const int acc = static_cast<int>(si & 1);
+          const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
+          if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * 256;
+          const uint32_t qb = q_addr + sub * C::kQSlotBytes;
 #pragma unroll
-        for (int kk = 0; kk < D_I / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32;
-          const uint32_t qoff = (kk >> 2) * (kMaxCols * 128) + (kk & 3) * 32;
-          mma_bf16_ss(d_tmem, sw128_desc(a_addr + koff, 16, 1024), sw128_desc(q_addr + qoff, 16, 1024), idesc,
-                      kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D_I / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * (kMaxCols * 128) + (kk & 3) * 32;
+            mma_bf16_ss(d_tmem, sw128_desc(a_addr + koff, 16, 1024), sw128_desc(qb + qoff, 16, 1024), idesc,
+                        kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&acc_full[acc]);
         }
+        if (!ok) break;
         mma_commit(&empty[st]);
-        mma_commit(&acc_full[acc]);
       }
       // make sure nothing issued is still running before TMEM is released
       mma_commit(q_ready);
@@ -212,64 +229,73 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
     const int half = (warp - kEpiWarp0) >> 2;        // which half of the columns
     const int row = quad * 32 + lane;                // key row inside the tile
     int cur_grp = -1;
-    int64_t it = 0;
-    for (int64_t wi = lo; wi < hi; ++wi, ++it) {
-      const int grp = static_cast<int>(wi / a.tiles);
+    int64_t si = 0;  // (item, group) sub-items, as counted by the MMA issuer
+    bool got = true;
+    for (int64_t wi = lo; wi < hi && got; ++wi) {
+      const int grp = static_cast<int>(wi / a.tiles) * P;
+      const int ng = P == 1 ? 1 : (a.groups - grp < P ? a.groups - grp : P);
       const int t = static_cast<int>(wi % a.tiles);
       if (grp != cur_grp) {
-        // All MMAs of the previous group finished (their accumulators were
-        // drained below), so Q and the weights can be replaced.
+        // All MMAs of the previous item's groups finished (their accumulators
+        // were drained below), so Q and the weights can be replaced.
         if (*abort_flag) break;
         named_bar_sync(1, kNumEpiThreads);
-        const int b0 = grp * a.G;
-        constexpr int kChunksPerRow = D_I / 8;
-        // 16-byte chunks in batches of 8 loads per thread, all issued before
-        // their stores, so one memory latency covers a batch
-        constexpr int kBatch = FP8 ? 2 : 8;
-        const int total = ncols * kChunksPerRow;
-        for (int i0 = et; i0 < total; i0 += kBatch * kNumEpiThreads) {
-          uint4 v[kBatch];
+        for (int slot = 0; slot < ng; ++slot) {
+          const int b0 = (grp + slot) * a.G;
+          uint8_t* qslot = qs + slot * C::kQSlotBytes;
+          float* wslot = ws + slot * kMaxCols;
+          constexpr int kChunksPerRow = D_I / 8;
+          // 16-byte chunks in batches of 8 loads per thread, all issued
+          // before their stores, so one memory latency covers a batch
+          constexpr int kBatch = FP8 ? 2 : 8;
+          const int total = ncols * kChunksPerRow;
+          for (int i0 = et; i0 < total; i0 += kBatch * kNumEpiThreads) {
+            uint4 v[kBatch];
 #pragma unroll
-          for (int k = 0; k < kBatch; ++k) {
-            const int i = i0 + k * kNumEpiThreads;
-            v[k] = make_uint4(0, 0, 0, 0);
-            if (i < total) {
-              const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
-              const int g = r / HP, h = r % HP, b = b0 + g;
-              if (h < a.H_I && b < a.B)
-                v[k] = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * a.H_I + h) * D_I + c8 * 8));
+            for (int k = 0; k < kBatch; ++k) {
+              const int i = i0 + k * kNumEpiThreads;
+              v[k] = make_uint4(0, 0, 0, 0);
+              if (i < total) {
+                const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
+                const int g = r / HP, h = r % HP, b = b0 + g;
+                if (h < a.H_I && b < a.B)
+                  v[k] = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * a.H_I + h) * D_I + c8 * 8));
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+              const int i = i0 + k * kNumEpiThreads;
+              if (i < total) {
+                const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
+                st_shared_v4(smem_u32(qslot + (c8 >> 3) * (kMaxCols * 128) + sw128_offset(r, c8 & 7)), v[k]);
+              }
             }
           }
-#pragma unroll
-          for (int k = 0; k < kBatch; ++k) {
-            const int i = i0 + k * kNumEpiThreads;
-            if (i < total) {
-              const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
-              st_shared_v4(smem_u32(qs + (c8 >> 3) * (kMaxCols * 128) + sw128_offset(r, c8 & 7)), v[k]);
-            }
+          for (int i = et; i < kMaxCols; i += kNumEpiThreads) {
+            const int g = i / HP, h = i % HP, b = b0 + g;
+            wslot[i] = (g < a.G && h < a.H_I && b < a.B) ? a.w[static_cast<int64_t>(b) * a.H_I + h] : 0.f;
           }
-        }
-        for (int i = et; i < kMaxCols; i += kNumEpiThreads) {
-          const int g = i / HP, h = i % HP, b = b0 + g;
-          ws[i] = (g < a.G && h < a.H_I && b < a.B) ? a.w[static_cast<int64_t>(b) * a.H_I + h] : 0.f;
-        }
-        if (et < GMAX) {
-          const int b = b0 + et;
-          nvs[et] = (et < a.G && b < a.B) ? (a.n_valid ? a.n_valid[b] : a.N) : 0;
+          if (et < GMAX) {
+            const int b = b0 + et;
+            nvs[slot * 16 + et] = (et < a.G && b < a.B) ? (a.n_valid ? a.n_valid[b] : a.N) : 0;
+          }
         }
         fence_proxy_async_smem();
         named_bar_sync(1, kNumEpiThreads);
         if (et == 0) mbar_arrive(q_ready);
         cur_grp = grp;
       }
-      const int acc = static_cast<int>(it & 1);
-      const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
-      const bool got = mbar_wait(&acc_full[acc], aph, abort_flag, a.status);
+      for (int sub = 0; sub < ng; ++sub, ++si) {
+      const int acc = static_cast<int>(si & 1);
+      const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
+      got = mbar_wait(&acc_full[acc], aph, abort_flag, a.status);
       __syncwarp();  // tcgen05.ld below is warp-collective
       if (!got) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256;
-      const int b0 = grp * a.G;
+      const int b0 = (grp + sub) * a.G;
+      const float* wsl = ws + sub * kMaxCols;
+      const int64_t* nvsl = nvs + sub * 16;
       const int64_t s = static_cast<int64_t>(t) * kTileKeys + row;
       // One half of the columns = a contiguous run of whole queries.
       auto tile_half = [&](auto half_c) {
@@ -307,16 +333,23 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
           if constexpr (kPerWait == 2) {
             if (haveB) tmem_ld_wait64(rb);
           }
+          // the weights of 32 columns at a time: eight loads issued back to
+          // back, then used
           auto reduce64 = [&](const uint32_t (&rv)[64], int cbase) {
 #pragma unroll
-            for (int j4 = 0; j4 < 16; ++j4) {
-              const float4 wv = ld_shared_v4f(ws + cbase + 4 * j4);
-              const float wj[4] = {wv.x, wv.y, wv.z, wv.w};
+            for (int h32 = 0; h32 < 2; ++h32) {
+              float4 wv[8];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int j = j4 * 4 + e;
-                float& acc_ref = sum[(cbase + j) / HP - kQ0][j % NP];
-                acc_ref = fmaf(wj[e], fmaxf(__uint_as_float(rv[j]), 0.f), acc_ref);
+              for (int k = 0; k < 8; ++k) wv[k] = ld_shared_v4f(wsl + cbase + 32 * h32 + 4 * k);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float wj[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int j = 32 * h32 + 4 * k + e;
+                  float& acc_ref = sum[(cbase + j) / HP - kQ0][j % NP];
+                  acc_ref = fmaf(wj[e], fmaxf(__uint_as_float(rv[j]), 0.f), acc_ref);
+                }
               }
             }
           };
@@ -330,7 +363,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
         if (s < a.N) {
           float scale = 1.f;
           if constexpr (FP8) {
-            const int64_t zb = a.per_query ? grp : 0;
+            const int64_t zb = a.per_query ? grp + sub : 0;
             scale = a.k_scale[zb * a.scale_batch_stride + s];
           }
 #pragma unroll
@@ -340,7 +373,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
               float tot = 0.f;
 #pragma unroll
               for (int p = 0; p < NP; ++p) tot += sum[g][p];
-              const float val = (s < nvs[gg]) ? tot * scale : -INFINITY;
+              const float val = (s < nvsl[gg]) ? tot * scale : -INFINITY;
               a.scores[static_cast<int64_t>(b0 + gg) * a.N + s] = val;
             }
           }
@@ -351,6 +384,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
         else tile_half(std::integral_constant<int, 1>{});
       } else {
         tile_half(std::integral_constant<int, 0>{});
+      }
       }
     }
   } else if constexpr (FP8) {
@@ -404,11 +438,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8>::kThreads, 1)
   }
 }
 
-template <int D_I, int HP, bool FP8>
+template <int D_I, int HP, bool FP8, bool PAIR>
 cudaError_t launch_indexer_inst(const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t stream,
                                 bool pdl) {
-  using C = IdxCfg<D_I, FP8>;
-  auto kern = indexer_tc_kernel<D_I, HP, FP8>;
+  using C = IdxCfg<D_I, FP8, PAIR>;
+  auto kern = indexer_tc_kernel<D_I, HP, FP8, PAIR>;
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
@@ -416,13 +450,13 @@ cudaError_t launch_indexer_inst(const CUtensorMap& map, const IndexerArgs& a, in
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int D_I, bool FP8>
+template <int D_I, bool FP8, bool PAIR>
 cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t s, bool pdl) {
   switch (HP) {
-    case 16: return launch_indexer_inst<D_I, 16, FP8>(map, a, grid, s, pdl);
-    case 32: return launch_indexer_inst<D_I, 32, FP8>(map, a, grid, s, pdl);
-    case 64: return launch_indexer_inst<D_I, 64, FP8>(map, a, grid, s, pdl);
-    case 128: return launch_indexer_inst<D_I, 128, FP8>(map, a, grid, s, pdl);
+    case 16: return launch_indexer_inst<D_I, 16, FP8, PAIR>(map, a, grid, s, pdl);
+    case 32: return launch_indexer_inst<D_I, 32, FP8, PAIR>(map, a, grid, s, pdl);
+    case 64: return launch_indexer_inst<D_I, 64, FP8, PAIR>(map, a, grid, s, pdl);
+    case 128: return launch_indexer_inst<D_I, 128, FP8, PAIR>(map, a, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -430,18 +464,24 @@ cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const IndexerArgs& a, in
 }  // namespace
 
 int indexer_smem_bytes(int d_I, bool fp8) {
-  if (d_I == 64) return fp8 ? IdxCfg<64, true>::kSmemBytes : IdxCfg<64, false>::kSmemBytes;
-  return fp8 ? IdxCfg<128, true>::kSmemBytes : IdxCfg<128, false>::kSmemBytes;
+  if (d_I == 64) return fp8 ? IdxCfg<64, true, false>::kSmemBytes : IdxCfg<64, false, true>::kSmemBytes;
+  return fp8 ? IdxCfg<128, true, false>::kSmemBytes : IdxCfg<128, false, true>::kSmemBytes;
 }
 
 cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
                            cudaStream_t stream, bool pdl) {
-  if (d_I == 64)
-    return fp8 ? dispatch_hp<64, true>(HP, map, a, grid, stream, pdl)
-               : dispatch_hp<64, false>(HP, map, a, grid, stream, pdl);
-  if (d_I == 128)
-    return fp8 ? dispatch_hp<128, true>(HP, map, a, grid, stream, pdl)
-               : dispatch_hp<128, false>(HP, map, a, grid, stream, pdl);
+  if (fp8) {
+    if (d_I == 64) return dispatch_hp<64, true, false>(HP, map, a, grid, stream, pdl);
+    if (d_I == 128) return dispatch_hp<128, true, false>(HP, map, a, grid, stream, pdl);
+    return cudaErrorInvalidValue;
+  }
+  if (a.pair == 2) {
+    if (d_I == 64) return dispatch_hp<64, false, true>(HP, map, a, grid, stream, pdl);
+    if (d_I == 128) return dispatch_hp<128, false, true>(HP, map, a, grid, stream, pdl);
+    return cudaErrorInvalidValue;
+  }
+  if (d_I == 64) return dispatch_hp<64, false, false>(HP, map, a, grid, stream, pdl);
+  if (d_I == 128) return dispatch_hp<128, false, false>(HP, map, a, grid, stream, pdl);
   return cudaErrorInvalidValue;
 }
 

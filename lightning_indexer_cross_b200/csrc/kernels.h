@@ -82,7 +82,9 @@ struct IndexerArgs {
   int64_t N;
   int G;              // queries per group (share one key tile)
   int tiles;          // 128-key tiles per group
-  int64_t total_items;  // groups * tiles
+  int groups;         // ceil(B / G)
+  int pair;           // groups per work item: 2 (one cache shared by all queries, >= 2 groups) or 1
+  int64_t total_items;  // ceil(groups / pair) * tiles
   int per_query;      // 1: key cache z-coordinate = group (G == 1)
 };
 
