@@ -228,19 +228,6 @@ IC_DEV void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Per-warpgroup register budget (every warp of a warpgroup executes the same
-// one). Registers a decrease gives back go to a per-CTA pool that an increase
-// draws from, so the decreases and increases of a kernel must balance against
-// the registers the CTA was launched with.
-template <int N>
-IC_DEV void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-IC_DEV void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // ---------------------------------------------------------------- tcgen05
 IC_DEV void tmem_alloc(uint32_t* holder, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(holder)),

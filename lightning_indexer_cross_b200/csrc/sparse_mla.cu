@@ -43,21 +43,16 @@ constexpr int kD = 576;
 constexpr int kDv = 512;
 constexpr int kHeads = 128;      // heads per CTA (MMA M)
 constexpr int kQKChunks = kD / 64;
-// 16 warps in four warpgroups: warps 0-10 gather, warp 11 issues the MMAs,
-// warps 12-15 run the softmax and the output (one per TMEM lane quadrant,
-// quadrant = warp % 4). Launched at 128 registers per thread; warpgroups 0-2
-// drop to kLowRegs and warpgroup 3 rises to kHighRegs. (Measured on B200: a
-// CTA's random 16-byte gathers scale with the threads issuing them, about
-// 51 GB/s from 224 threads and 66 GB/s from 512.)
+// 16 warps (so at most 128 registers per thread): warps 0-10 gather, warp 11
+// issues the MMAs, warps 12-15 run the softmax and the output (one per TMEM
+// lane quadrant, quadrant = warp % 4). (Measured on B200: a CTA's random
+// 16-byte gathers scale with the threads issuing them, about 51 GB/s from 224
+// threads and 66 GB/s from 512.)
 constexpr int kGatherWarps = 11;
 constexpr int kGather = kGatherWarps * 32;
 constexpr int kMmaWarp = 11;
 constexpr int kEpiWarp0 = 12;
 constexpr int kThreads = 512;
-constexpr int kLaunchRegs = 65536 / kThreads;
-constexpr int kLowRegs = 96;
-constexpr int kHighRegs = 216;
-static_assert(3 * 128 * kLowRegs + 128 * kHighRegs <= kThreads * kLaunchRegs, "register split exceeds the CTA's");
 constexpr int kStages = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -186,8 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  if (warp < kEpiWarp0) setmaxnreg_dec<kLowRegs>();
-  else setmaxnreg_inc<kHighRegs>();
 
   if (warp < kGatherWarps) {
     // ------------------------------------------------------------ gather warps
@@ -803,17 +796,6 @@ cudaError_t launch_ts(const CUtensorMap& qmap, const CUtensorMap& omap, const Ml
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  // The register split draws on the registers the CTA is launched with: a
-  // build that launches with fewer than kLaunchRegs per thread would leave
-  // the increase waiting, so it is refused.
-  static int regs = 0;
-  if (regs == 0) {
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, kern);
-    if (e != cudaSuccess) return e;
-    regs = fa.numRegs;
-  }
-  if (regs < kLaunchRegs) return cudaErrorInvalidConfiguration;
   return launch_kernel(kern, dim3(a.ctas), dim3(kThreads), C::kSmemBytes, stream, pdl, qmap, omap, a);
 }
 
