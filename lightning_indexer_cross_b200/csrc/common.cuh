@@ -376,6 +376,17 @@ IC_DEV float4 ld_shared_v4f(const void* p) {
 }
 
 // Element e (0 = low half, 1 = high half) of a packed bf16 pair, as float.
+// d = a * b + c on two fp32 lanes at once (sm_100 packed FMA), round to
+// nearest per lane.
+IC_DEV float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\tmov.b64 pc, {%6, %7};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
 IC_DEV float bf16_lane(uint32_t w, int e) { return __uint_as_float(e ? (w & 0xffff0000u) : (w << 16)); }
 IC_DEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -304,11 +304,18 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         constexpr int kC0 = H * kChunks;
         constexpr int kQ = GMAX / C::kHalves;                 // queries of this half
         constexpr int kQ0 = H * kQ;
-        // NP partial sums per query keep the FMA dependency chains short
+        // Four partial sums per query keep the FMA dependency chains short:
+        // for 64 or more heads two packed pairs (columns 4i, 4i+1 and 4i+2,
+        // 4i+3; one packed FMA per two columns), else NP scalars (more
+        // queries per warp; packed pairs would spill).
+        constexpr bool kPacked = HP >= 64;
         constexpr int NP = HP >= 64 ? 4 : (HP == 32 ? 2 : 1);
-        float sum[kQ][NP];
+        float2 sum2[kPacked ? kQ : 1][2];
+        float sum[kPacked ? 1 : kQ][NP];
 #pragma unroll
-        for (int g = 0; g < kQ; ++g)
+        for (int g = 0; g < (kPacked ? kQ : 1); ++g) sum2[g][0] = sum2[g][1] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < (kPacked ? 1 : kQ); ++g)
 #pragma unroll
           for (int p = 0; p < NP; ++p) sum[g][p] = 0.f;
         // The half's columns come in as two 64-column TMEM loads issued back
@@ -343,12 +350,22 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
               for (int k = 0; k < 8; ++k) wv[k] = ld_shared_v4f(wsl + cbase + 32 * h32 + 4 * k);
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
-                const float wj[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
+                const int j = 32 * h32 + 4 * k;  // 4 columns of one query (HP is a multiple of 16)
+                if constexpr (kPacked) {
+                  float2 (&acc)[2] = sum2[(cbase + j) / HP - kQ0];
+                  const float2 x01 =
+                      make_float2(fmaxf(__uint_as_float(rv[j]), 0.f), fmaxf(__uint_as_float(rv[j + 1]), 0.f));
+                  const float2 x23 =
+                      make_float2(fmaxf(__uint_as_float(rv[j + 2]), 0.f), fmaxf(__uint_as_float(rv[j + 3]), 0.f));
+                  acc[0] = ffma2(make_float2(wv[k].x, wv[k].y), x01, acc[0]);
+                  acc[1] = ffma2(make_float2(wv[k].z, wv[k].w), x23, acc[1]);
+                } else {
+                  const float wj[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int j = 32 * h32 + 4 * k + e;
-                  float& acc_ref = sum[(cbase + j) / HP - kQ0][j % NP];
-                  acc_ref = fmaf(wj[e], fmaxf(__uint_as_float(rv[j]), 0.f), acc_ref);
+                  for (int e = 0; e < 4; ++e) {
+                    float& acc_ref = sum[(cbase + j + e) / HP - kQ0][(j + e) % NP];
+                    acc_ref = fmaf(wj[e], fmaxf(__uint_as_float(rv[j + e]), 0.f), acc_ref);
+                  }
                 }
               }
             }
@@ -371,8 +388,12 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
             const int gg = kQ0 + g;
             if (gg < a.G && b0 + gg < a.B) {
               float tot = 0.f;
+              if constexpr (kPacked) {
+                tot = (sum2[g][0].x + sum2[g][0].y) + (sum2[g][1].x + sum2[g][1].y);
+              } else {
 #pragma unroll
-              for (int p = 0; p < NP; ++p) tot += sum[g][p];
+                for (int p = 0; p < NP; ++p) tot += sum[g][p];
+              }
               const float val = (s < nvsl[gg]) ? tot * scale : -INFINITY;
               a.scores[static_cast<int64_t>(b0 + gg) * a.N + s] = val;
             }
