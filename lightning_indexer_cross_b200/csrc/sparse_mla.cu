@@ -10,22 +10,25 @@
 //
 // Main kernel: persistent, one CTA per SM; a work unit is (split of TS <= 256
 // selected rows, query, block of 128 heads). Tensor memory holds 512 fp32
-// columns per lane, and the 128 x 512 output alone fills it, so each unit is
-// worked in two phases:
+// columns per lane, and the 128 x 512 output alone fills it, so its two
+// 256-column halves swap roles from one unit to the next. With A the half
+// the unit's logits use and B the other:
 //   QK   S[128 heads x TS] = Q . KV^T over 9 slices of 64 dims (tcgen05,
-//        M = 128 heads, N = TS rows) into TMEM columns [0, TS);
-//   soft the epilogue warps read S (one head per TMEM lane), take the exact
-//        max over the unit's rows, write P = 2^{z log2e - m} as bf16 into
-//        shared memory in the K-major layout of an MMA A operand;
-//   PV   O_lo = P . V[:, 0:256] into columns [256, 512), then
-//        O_hi = P . V[:, 256:512] into columns [0, 256) (S is dead by then);
+//        M = 128 heads, N = TS rows) into half A;
+//   soft the epilogue warps read S (one head per TMEM lane), write
+//        P = 2^{z log2e - ref} as bf16 into shared memory in the K-major
+//        layout of an MMA A operand;
+//   PV   O[:, 0:256] = P . V[:, 0:256] into half B, then
+//        O[:, 256:512] = P . V[:, 256:512] into half A (S is dead by then);
 //        V rows are the same gathered rows, read again as an MN-major B
 //        operand (64 rows x 256 dims per stage).
 // Each unit writes a normalised partial (m, l, O / l): O / l as 32-head x
-// 128-byte tiles staged in swizzled shared memory and written by TMA stores,
-// O_hi first so the next unit's QK can start while O_lo is written. The
-// combine kernel merges the splits, adds e^{sink} once to the denominator,
-// applies the gate and writes out / lse.
+// 128-byte tiles staged in swizzled shared memory and written by TMA stores.
+// Half B is read out while the MMAs of half A run, and the next unit's
+// logits go into it (its A is this unit's B), so the next QK does not wait
+// for the whole output to be read out. The combine kernel merges the splits,
+// adds e^{sink} once to the denominator, applies the gate and writes out /
+// lse.
 //
 // Warp roles (16 warps): 0-10 gather every stage of every unit (one ring of
 // three stages), 11 issues the MMAs, 12-15 run the softmax and the output.
@@ -66,16 +69,22 @@ struct MlaCfg {
   static constexpr int kOutSlots = kPBytes / (4 * 4096) < 4 ? kPBytes / (4 * 4096) : 4;
   static constexpr int kOffStages = 0;
   static constexpr int kOffP = kStages * kStageBytes;
-  static constexpr int kOffIdx = kOffP + kPBytes;         // [2][TS] selected rows, double-buffered
+  // one 4 KB output tile per epilogue warp for the first output half (the P
+  // buffer is still being read by the second half's MMAs)
+  static constexpr int kOffTiles = kOffP + kPBytes;
+  static constexpr int kOffIdx = kOffTiles + 4 * 4096;    // [2][TS] selected rows, double-buffered
   static constexpr int kOffMask = kOffIdx + 2 * TS * 4;   // [2][TS / 32] validity bits
   static constexpr int kOffBar = kOffMask + 2 * (TS / 32) * 4;
-  // full[kStages], empty[kStages], s_full, p_ready, o_full, o_hi_free, retire, idx_ready[2], idx_free[2]
-  static constexpr int kNumBars = 2 * kStages + 9;
+  // full[kStages], empty[kStages], s_full, p_ready, o1_full, o2_full, o1_free, o2_free, retire,
+  // idx_ready[2], idx_free[2]
+  static constexpr int kNumBars = 2 * kStages + 11;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // dynamic shared memory starts 1024-byte aligned (checked at entry)
+  static constexpr int kSmemBytes = kOffMisc + 16;
   static constexpr int kNumSt = kQKChunks + 2 * (TS / 64);
   static_assert(kOutSlots >= 1, "at least one output tile per warp");
   static_assert(kOffBar % 8 == 0, "mbarrier alignment");
+  static_assert(kOffTiles % 1024 == 0, "swizzled tiles 1024-byte aligned");
   static_assert(kSmemBytes <= 232448, "fits one CTA per SM");
 };
 
@@ -131,20 +140,29 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
                                                                    const __grid_constant__ CUtensorMap omap,
                                                                    const MlaArgs a) {
   using C = MlaCfg<TS>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the swizzled layouts need a 1024-byte-aligned base; the layout leaves no
+  // room to align it here, so a misaligned window is reported, not used
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) record_status(a.status, IC_ERR_UNSUPPORTED);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* stages = smem + C::kOffStages;
   uint8_t* ps = smem + C::kOffP;
+  uint8_t* tiles1 = smem + C::kOffTiles;
   int32_t* idx_s = reinterpret_cast<int32_t*>(smem + C::kOffIdx);
   uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + C::kOffMask);  // bit j of word w: row 32w+j valid
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = full + kStages;
-  uint64_t* s_full = empty + kStages;  // S of the current unit in TMEM
+  uint64_t* s_full = empty + kStages;  // S of the current unit in TMEM (half A)
   uint64_t* p_ready = s_full + 1;      // P in shared memory, S read
-  uint64_t* o_full = p_ready + 1;      // O of the current unit in TMEM
-  uint64_t* o_hi_free = o_full + 1;    // TMEM columns [0, 256) read out
-  uint64_t* retire = o_hi_free + 1;    // every MMA of this CTA retired
+  uint64_t* o1_full = p_ready + 1;     // output dims [0, 256) in TMEM half B
+  uint64_t* o2_full = o1_full + 1;     // output dims [256, 512) in TMEM half A
+  uint64_t* o1_free = o2_full + 1;     // half B read out
+  uint64_t* o2_free = o1_free + 1;     // half A read out
+  uint64_t* retire = o2_free + 1;      // every MMA of this CTA retired
   uint64_t* idx_ready = retire + 1;    // [2] selected rows of a unit in shared memory
   uint64_t* idx_free = idx_ready + 2;  // [2] the softmax is done with a unit's validity bits
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -162,8 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     }
     mbar_init(s_full, 1);
     mbar_init(p_ready, 128);  // the four epilogue warps
-    mbar_init(o_full, 1);
-    mbar_init(o_hi_free, 128);
+    mbar_init(o1_full, 1);
+    mbar_init(o2_full, 1);
+    mbar_init(o1_free, 128);
+    mbar_init(o2_free, 128);
     mbar_init(retire, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&idx_ready[i], kGather);
@@ -304,8 +324,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       bool ok = true;
       int g = 0;
       for (int i = 0, u = blockIdx.x; u < a.units && ok; ++i, u += a.ctas) {
-        // S lands in columns [0, TS): the previous unit's O_hi must be read out
-        if (i > 0 && !mbar_wait(o_hi_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status)) {
+        // TMEM halves: S and output dims [256, 512) in half A, output dims
+        // [0, 256) in half B; the next unit's A is this unit's B, read out
+        // first, while this unit's second output half is still being formed
+        const uint32_t col_a = (i & 1) ? 256u : 0u, col_b = 256u - col_a;
+        if (i > 0 && !mbar_wait(o1_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status)) {
           ok = false;
           break;
         }
@@ -318,13 +341,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           const uint32_t base = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tmem_base, sw128_desc(base + kk * 32, 16, 1024),
+            mma_bf16_ss(tmem_base + col_a, sw128_desc(base + kk * 32, 16, 1024),
                         sw128_desc(base + kHeads * 128 + kk * 32, 16, 1024), idesc_qk, (s | kk) != 0);
           mma_commit(&empty[st]);
         }
         if (!ok) break;
         mma_commit(s_full);
         if (!mbar_wait(p_ready, static_cast<uint32_t>(i & 1), abort_flag, a.status)) { ok = false; break; }
+        // half B held the previous unit's second output half
+        if (i > 0 && !mbar_wait(o2_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         for (int s = kQKChunks; s < C::kNumSt; ++s, ++g) {
           const int st = g % kStages;
@@ -333,16 +361,17 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           tc_fence_after();
           const int p = s - kQKChunks;
           const int jh = p / (TS / 64), tc = p % (TS / 64);
-          const uint32_t d_tmem = tmem_base + (jh == 0 ? 256u : 0u);
+          const uint32_t d_tmem = tmem_base + (jh == 0 ? col_b : col_a);
           const uint32_t base = smem_u32(stages + st * C::kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_ss(d_tmem, sw128_desc(p_addr + tc * (kHeads * 128) + kk * 32, 16, 1024),
                         sw128_desc(base + kk * 2048, 8192, 1024), idesc_pv, (tc | kk) != 0);
           mma_commit(&empty[st]);
+          if (p == TS / 64 - 1) mma_commit(o1_full);
         }
         if (!ok) break;
-        mma_commit(o_full);
+        mma_commit(o2_full);
       }
       // every MMA issued has retired before TMEM is released
       mma_commit(retire);
@@ -352,12 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
     // ------------------------------------------------------------ softmax + output
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // head row within the block
-    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t tlane = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const float c2 = a.sm_scale * kLog2e;
     uint8_t* tiles = ps + quad * (C::kOutSlots * 4096);
     bool ok = true;
     for (int i = 0, u = blockIdx.x; u < a.units && ok; ++i, u += a.ctas) {
       const Unit w = unit_of(a, u);
+      const uint32_t col_a = (i & 1) ? 256u : 0u, col_b = 256u - col_a;
+      const uint32_t taddr = tlane + col_a;  // S (and later output dims [256, 512))
       const uint32_t* vm = vmask + (i & 1) * (TS / 32);
       ok = mbar_wait(&idx_ready[i & 1], static_cast<uint32_t>((i >> 1) & 1), abort_flag, a.status) &&
            mbar_wait(s_full, static_cast<uint32_t>(i & 1), abort_flag, a.status);
@@ -440,25 +471,17 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       fence_proxy_async_smem();
       mbar_arrive(p_ready);
       mbar_arrive(&idx_free[i & 1]);
-      ok = mbar_wait(o_full, static_cast<uint32_t>(i & 1), abort_flag, a.status);
-      __syncwarp();
-      if (!ok) break;
-      tc_fence_after();
       // O / l (0 when no row was valid) as 32-head x 128-byte tiles in
-      // 128-byte-swizzled shared memory (the P buffer: every PV MMA has
-      // retired), each written out by one TMA store; heads past H fall outside
-      // the map and are not written. O_hi sits in TMEM columns [0, 256) and is
-      // read first, so the next unit's QK can start; O_lo in [256, 512).
+      // 128-byte-swizzled shared memory, each written out by one TMA store;
+      // heads past H fall outside the map and are not written. Dims
+      // [0, 256) (TMEM half B) are read out as soon as their MMAs retire,
+      // through this warp's own tile (the P buffer is still read by the
+      // second half's MMAs), and then free half B for the next unit's
+      // logits; dims [256, 512) (half A) go through four tiles of the P
+      // buffer once every PV MMA has retired.
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const int head0 = w.hb * kHeads + quad * 32;
-      int nt = 0;  // tiles issued by this warp in this unit
-      auto put_tile = [&](const uint32_t (&wd)[32], int x) {
-        const int slot = nt % C::kOutSlots;
-        if (nt >= C::kOutSlots) {
-          if (lane == 0) bulk_wait_read<C::kOutSlots - 1>();  // the slot's previous store has read it
-          __syncwarp();
-        }
-        uint8_t* tile = tiles + slot * 4096;
+      auto put_tile = [&](const uint32_t (&wd)[32], int x, uint8_t* tile) {
         const uint32_t tb = smem_u32(tile);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
@@ -470,41 +493,60 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
           tma_store_4d(&omap, tile, x, w.sp, head0, w.b);
           bulk_commit();
         }
-        ++nt;
       };
-      // dims [256 t', ...): half 1 (O_hi, columns [0, 256)) first, then half 0
+      uint8_t* own_tile = tiles1 + quad * 4096;
+      int nt = 0;  // tiles of the P buffer issued by this warp in this unit
 #pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        const int half = 1 - hh;
-        const uint32_t col0 = half ? 0u : 256u;
+      for (int half = 0; half < 2; ++half) {
+        ok = mbar_wait(half == 0 ? o1_full : o2_full, static_cast<uint32_t>(i & 1), abort_flag, a.status);
+        __syncwarp();
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tcol = tlane + (half == 0 ? col_b : col_a);
+        auto place = [&](const uint32_t (&wd)[32], int x) {
+          uint8_t* tile;
+          if (half == 0) {
+            if (lane == 0) bulk_wait_read<0>();  // this warp's tile is read out
+            __syncwarp();
+            tile = own_tile;
+          } else {
+            const int slot = nt % C::kOutSlots;
+            if (nt >= C::kOutSlots) {
+              if (lane == 0) bulk_wait_read<C::kOutSlots - 1>();  // the slot's previous store has read it
+              __syncwarp();
+            }
+            tile = tiles + slot * 4096;
+            ++nt;
+          }
+          put_tile(wd, x, tile);
+        };
         if (a.out_f32) {
 #pragma unroll 1
           for (int t = 0; t < 8; ++t) {  // 32 dims per tile
             uint32_t rv[32];
-            tmem_ld32_issue(taddr + col0 + 32u * t, rv);
+            tmem_ld32_issue(tcol + 32u * t, rv);
             tmem_ld_wait(rv);
 #pragma unroll
             for (int j = 0; j < 32; ++j) rv[j] = __float_as_uint(__uint_as_float(rv[j]) * inv_l);
-            put_tile(rv, half * 256 + 32 * t);
+            place(rv, half * 256 + 32 * t);
           }
         } else {
 #pragma unroll 1
           for (int t = 0; t < 4; ++t) {  // 64 dims per tile
             uint32_t rv[64];
-            tmem_ld64_issue(taddr + col0 + 64u * t, rv);
+            tmem_ld64_issue(tcol + 64u * t, rv);
             tmem_ld_wait64(rv);
             uint32_t wd[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               wd[j] = pack_bf16x2(__uint_as_float(rv[2 * j]) * inv_l, __uint_as_float(rv[2 * j + 1]) * inv_l);
-            put_tile(wd, half * 256 + 64 * t);
+            place(wd, half * 256 + 64 * t);
           }
         }
-        if (hh == 0) {
-          tc_fence_before();
-          mbar_arrive(o_hi_free);
-        }
+        tc_fence_before();
+        mbar_arrive(half == 0 ? o1_free : o2_free);
       }
+      if (!ok) break;
       if (lane == 0) bulk_wait_read<0>();  // the tiles (the next unit's P buffer) are read out
       __syncwarp();
       const int head = w.hb * kHeads + r;
