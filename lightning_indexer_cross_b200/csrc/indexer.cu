@@ -323,56 +323,88 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         // 32 columns.
         static_assert(kChunks == 4 || kChunks == 8, "half = 128 or 256 columns");
         constexpr int kLoads = kChunks / 2;  // 64-column loads of this half
-        // whole rows (one warp per quadrant): two loads in flight per wait;
-        // half rows (two warps per quadrant): one load at a time, the other
-        // warp of the sub-partition covers the latency
-        constexpr int kPerWait = C::kHalves == 1 ? 2 : 1;
+        constexpr int kPerWait = C::kHalves == 1 ? 2 : 1;  // 64-column loads per wait (whole rows)
+        // w * ReLU(logit) for 32 columns starting at cbase (their weights:
+        // kWBatch 16-byte loads issued back to back, then used)
+        constexpr int kWBatch = 8;
+        auto reduce32 = [&](const auto& rvv, int off, int cbase) {
 #pragma unroll
-        for (int pass = 0; pass < kLoads; pass += kPerWait) {
-          const int cA = (kC0 + 2 * pass) * 32, cB = cA + 64;
-          const bool haveA = cA < ncols, haveB = kPerWait == 2 && cB < ncols && pass + 1 < kLoads;
-          uint32_t ra[64], rb[kPerWait == 2 ? 64 : 1];
-          if (haveA) tmem_ld64_issue(taddr + cA, ra);
-          if constexpr (kPerWait == 2) {
-            if (haveB) tmem_ld64_issue(taddr + cB, rb);
-          }
-          if (haveA) tmem_ld_wait64(ra);
-          if constexpr (kPerWait == 2) {
-            if (haveB) tmem_ld_wait64(rb);
-          }
-          // the weights of 32 columns at a time: eight loads issued back to
-          // back, then used
-          auto reduce64 = [&](const uint32_t (&rv)[64], int cbase) {
+          for (int k0 = 0; k0 < 8; k0 += kWBatch) {
+          float4 wv[8];
 #pragma unroll
-            for (int h32 = 0; h32 < 2; ++h32) {
-              float4 wv[8];
+          for (int k = k0; k < k0 + kWBatch; ++k) wv[k] = ld_shared_v4f(wsl + cbase + 4 * k);
 #pragma unroll
-              for (int k = 0; k < 8; ++k) wv[k] = ld_shared_v4f(wsl + cbase + 32 * h32 + 4 * k);
+          for (int k = k0; k < k0 + kWBatch; ++k) {
+            const int j = 4 * k;  // 4 columns of one query (HP is a multiple of 16)
+            if constexpr (kPacked) {
+              float2 (&acc)[2] = sum2[(cbase + j) / HP - kQ0];
+              const float2 x01 = make_float2(fmaxf(__uint_as_float(rvv[off + j]), 0.f),
+                                             fmaxf(__uint_as_float(rvv[off + j + 1]), 0.f));
+              const float2 x23 = make_float2(fmaxf(__uint_as_float(rvv[off + j + 2]), 0.f),
+                                             fmaxf(__uint_as_float(rvv[off + j + 3]), 0.f));
+              acc[0] = ffma2(make_float2(wv[k].x, wv[k].y), x01, acc[0]);
+              acc[1] = ffma2(make_float2(wv[k].z, wv[k].w), x23, acc[1]);
+            } else {
+              const float wj[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int j = 32 * h32 + 4 * k;  // 4 columns of one query (HP is a multiple of 16)
-                if constexpr (kPacked) {
-                  float2 (&acc)[2] = sum2[(cbase + j) / HP - kQ0];
-                  const float2 x01 =
-                      make_float2(fmaxf(__uint_as_float(rv[j]), 0.f), fmaxf(__uint_as_float(rv[j + 1]), 0.f));
-                  const float2 x23 =
-                      make_float2(fmaxf(__uint_as_float(rv[j + 2]), 0.f), fmaxf(__uint_as_float(rv[j + 3]), 0.f));
-                  acc[0] = ffma2(make_float2(wv[k].x, wv[k].y), x01, acc[0]);
-                  acc[1] = ffma2(make_float2(wv[k].z, wv[k].w), x23, acc[1]);
-                } else {
-                  const float wj[4] = {wv[k].x, wv[k].y, wv[k].z, wv[k].w};
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    float& acc_ref = sum[(cbase + j + e) / HP - kQ0][(j + e) % NP];
-                    acc_ref = fmaf(wj[e], fmaxf(__uint_as_float(rv[j + e]), 0.f), acc_ref);
-                  }
-                }
+              for (int e = 0; e < 4; ++e) {
+                float& acc_ref = sum[(cbase + j + e) / HP - kQ0][(j + e) % NP];
+                acc_ref = fmaf(wj[e], fmaxf(__uint_as_float(rvv[off + j + e]), 0.f), acc_ref);
               }
             }
-          };
-          if (haveA) reduce64(ra, (kC0 + 2 * pass) * 32);
-          if constexpr (kPerWait == 2) {
-            if (haveB) reduce64(rb, (kC0 + 2 * pass) * 32 + 64);
+          }
+          }
+        };
+        if constexpr (kPerWait == 1) {
+          const int c0 = kC0 * 32;
+          if (c0 + kChunks * 32 <= ncols) {
+            // every column of the half is present: 32-column TMEM loads, the
+            // next one in flight while the current one is reduced
+            uint32_t r0[32], r1[32];
+            tmem_ld32_issue(taddr + c0, r0);
+            tmem_ld_wait(r0);
+#pragma unroll
+            for (int c = 0; c < kChunks; c += 2) {
+              tmem_ld32_issue(taddr + c0 + (c + 1) * 32, r1);
+              reduce32(r0, 0, c0 + c * 32);
+              tmem_ld_wait(r1);
+              if (c + 2 < kChunks) tmem_ld32_issue(taddr + c0 + (c + 2) * 32, r0);
+              reduce32(r1, 0, c0 + (c + 1) * 32);
+              if (c + 2 < kChunks) tmem_ld_wait(r0);
+            }
+          } else {
+            // a partial half: one 64-column load at a time
+#pragma unroll
+            for (int pass = 0; pass < kLoads; ++pass) {
+              const int cA = c0 + 64 * pass;
+              if (cA < ncols) {
+                uint32_t ra[64];
+                tmem_ld64_issue(taddr + cA, ra);
+                tmem_ld_wait64(ra);
+                reduce32(ra, 0, cA);
+                reduce32(ra, 32, cA + 32);
+              }
+            }
+          }
+        } else {
+          // whole rows: two 64-column loads in flight per wait
+#pragma unroll
+          for (int pass = 0; pass < kLoads; pass += 2) {
+            const int cA = (kC0 + 2 * pass) * 32, cB = cA + 64;
+            const bool haveA = cA < ncols, haveB = cB < ncols && pass + 1 < kLoads;
+            uint32_t ra[64], rb[64];
+            if (haveA) tmem_ld64_issue(taddr + cA, ra);
+            if (haveB) tmem_ld64_issue(taddr + cB, rb);
+            if (haveA) tmem_ld_wait64(ra);
+            if (haveB) tmem_ld_wait64(rb);
+            if (haveA) {
+              reduce32(ra, 0, cA);
+              reduce32(ra, 32, cA + 32);
+            }
+            if (haveB) {
+              reduce32(rb, 0, cB);
+              reduce32(rb, 32, cB + 32);
+            }
           }
         }
         tc_fence_before();
