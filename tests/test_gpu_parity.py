@@ -183,6 +183,24 @@ def test_sparse_mla_wide_logit_spread(cuda_dev):
     np.testing.assert_allclose(lse.double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-2)
 
 
+@pytest.mark.parametrize("odt", [torch.bfloat16, torch.float32])
+def test_sparse_mla_three_units_per_cta(cuda_dev, odt):
+    """48 queries x 8 splits = 384 work units on a persistent grid of (at
+    most) one CTA per SM: CTAs take up to three units, so the row-index
+    double buffer and both TMEM half assignments are reused. Sampled queries
+    against the oracle (with some -1 rows and a ragged last split)."""
+    B, N, H, k = 48, 6000, 128, 2000
+    q, kv, idx, sink, g = W.attention_case(B, N, H, k, shared=True, gate=True, n_invalid=9, seed=41,
+                                           device=cuda_dev)
+    out, lse = _ops().sparse_mla_decode(q, kv, idx, sink, g, out_dtype=odt)
+    torch.cuda.synchronize()
+    for b in (0, 17, 31, 46, 47):
+        ref, ref_lse = oracle.sparse_mla(q[b:b + 1], kv, idx[b:b + 1], sink, g[b:b + 1])
+        err = attn_row_error(out[b:b + 1], ref)
+        assert err <= ATTN_TOL[odt], f"query {b}: attention row error {err:.3e}"
+        np.testing.assert_allclose(lse[b:b + 1].double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-3)
+
+
 def test_sparse_mla_bad_index_is_reported_and_skipped(cuda_dev):
     from lightning_indexer_cross_b200 import _abi
     ops = _ops()
