@@ -183,6 +183,27 @@ def test_sparse_mla_wide_logit_spread(cuda_dev):
     np.testing.assert_allclose(lse.double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-2)
 
 
+def test_sparse_mla_holes_and_wide_spread_256_row_splits(cuda_dev):
+    """256-row splits (16 queries x 8 splits fill the SMs) with -1 rows inside
+    the lists: whole first 32-row chunks of two splits are empty (the
+    exponent reference starts at 0), a third split has scattered holes, the
+    rest are all valid; a large softmax scale pushes many rows past the
+    first pass's range, so the pass is redone with the row max."""
+    B, N, H, k = 16, 5000, 128, 2048
+    q, kv, idx, sink, g = W.attention_case(B, N, H, k, shared=True, gate=True, seed=45, device=cuda_dev)
+    idx[:, 256:296] = -1
+    idx[:, 3 * 256:3 * 256 + 32] = -1
+    idx[:, 5 * 256 + 7:6 * 256:13] = -1
+    for scale in (None, 3.0):
+        out, lse = _ops().sparse_mla_decode(q, kv, idx, sink, g, sm_scale=scale, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        for b in (0, 9, 15):
+            ref, ref_lse = oracle.sparse_mla(q[b:b + 1], kv, idx[b:b + 1], sink, g[b:b + 1], scale)
+            err = attn_row_error(out[b:b + 1], ref)
+            assert err <= ATTN_TOL[torch.float32], f"scale {scale}, query {b}: attention row error {err:.3e}"
+            np.testing.assert_allclose(lse[b:b + 1].double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-2)
+
+
 @pytest.mark.parametrize("odt", [torch.bfloat16, torch.float32])
 def test_sparse_mla_three_units_per_cta(cuda_dev, odt):
     """48 queries x 8 splits = 384 work units on a persistent grid of (at
