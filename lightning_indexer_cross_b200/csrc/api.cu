@@ -96,6 +96,18 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
                    fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
+  const int HP = indexer_hp(H_I);
+  const int G = per_query ? 1 : std::min(256 / HP, B);
+  // queries: (d_I, H_I, B); a (64, HP, G) box is one 64-dim block of a query
+  // group's stacked heads, heads past H_I and queries past B read as zeros
+  CUtensorMap qmap;
+  const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(d_I), static_cast<cuuint64_t>(H_I), static_cast<cuuint64_t>(B)};
+  const cuuint64_t qstrides[2] = {static_cast<cuuint64_t>(d_I) * 2, static_cast<cuuint64_t>(H_I) * d_I * 2};
+  const cuuint32_t qbox[3] = {64, static_cast<cuuint32_t>(HP), static_cast<cuuint32_t>(G)};
+  r = enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), qdims, qstrides, qbox, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
 
   ic::IndexerArgs a{};
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -108,8 +120,7 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   a.B = B;
   a.H_I = H_I;
   a.N = N;
-  const int HP = indexer_hp(H_I);
-  a.G = per_query ? 1 : std::min(256 / HP, B);
+  a.G = G;
   a.tiles = static_cast<int>(ceil_div<int64_t>(N, 128));
   const int64_t groups = ceil_div<int64_t>(B, a.G);
   a.groups = static_cast<int>(groups);
@@ -117,7 +128,7 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   a.total_items = ceil_div<int64_t>(groups, a.pair) * a.tiles;
   a.per_query = per_query ? 1 : 0;
   const int grid = static_cast<int>(std::min<int64_t>(num_sms(), a.total_items));
-  cudaError_t e = ic::launch_indexer(map, a, HP, d_I, fp8, grid, stream, pdl);
+  cudaError_t e = ic::launch_indexer(map, qmap, a, HP, d_I, fp8, grid, stream, pdl);
   if (e != cudaSuccess) return IC_ERR_CUDA;
   g_launches += 1;
   return IC_OK;

@@ -82,7 +82,8 @@ struct IdxCfg {
 
 template <int D_I, int HP, bool FP8, bool PAIR>
 __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
-    indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerArgs a) {
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                      const IndexerArgs a) {
   using C = IdxCfg<D_I, FP8, PAIR>;
   constexpr int P = C::kQSlots;  // query groups per work item
   constexpr int GMAX = kMaxCols / HP;
@@ -132,7 +133,10 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&kmap);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&qmap);
+  }
   pdl_wait();
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -240,37 +244,21 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         // were drained below), so Q and the weights can be replaced.
         if (*abort_flag) break;
         named_bar_sync(1, kNumEpiThreads);
+        // Q of each slot: one TMA load per 64-dim block of the box (d_I 64,
+        // HP heads, G queries), written in the 128-byte-swizzled K-major
+        // layout the MMA reads; heads past H_I and queries past B are zero
+        // filled. The MMA issuer waits for the bytes on q_ready.
+        if (et == 0) {
+          mbar_arrive_expect_tx(q_ready, static_cast<uint32_t>(ng * C::kBlocks * HP * a.G * 128));
+          for (int slot = 0; slot < ng; ++slot)
+#pragma unroll
+            for (int bk = 0; bk < C::kBlocks; ++bk)
+              tma_load_3d(qs + slot * C::kQSlotBytes + bk * (kMaxCols * 128), &qmap, q_ready, bk * 64, 0,
+                          (grp + slot) * a.G);
+        }
         for (int slot = 0; slot < ng; ++slot) {
           const int b0 = (grp + slot) * a.G;
-          uint8_t* qslot = qs + slot * C::kQSlotBytes;
           float* wslot = ws + slot * kMaxCols;
-          constexpr int kChunksPerRow = D_I / 8;
-          // 16-byte chunks in batches of 8 loads per thread, all issued
-          // before their stores, so one memory latency covers a batch
-          constexpr int kBatch = FP8 ? 2 : 8;
-          const int total = ncols * kChunksPerRow;
-          for (int i0 = et; i0 < total; i0 += kBatch * kNumEpiThreads) {
-            uint4 v[kBatch];
-#pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-              const int i = i0 + k * kNumEpiThreads;
-              v[k] = make_uint4(0, 0, 0, 0);
-              if (i < total) {
-                const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
-                const int g = r / HP, h = r % HP, b = b0 + g;
-                if (h < a.H_I && b < a.B)
-                  v[k] = __ldg(reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * a.H_I + h) * D_I + c8 * 8));
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-              const int i = i0 + k * kNumEpiThreads;
-              if (i < total) {
-                const int r = i / kChunksPerRow, c8 = i % kChunksPerRow;
-                st_shared_v4(smem_u32(qslot + (c8 >> 3) * (kMaxCols * 128) + sw128_offset(r, c8 & 7)), v[k]);
-              }
-            }
-          }
           for (int i = et; i < kMaxCols; i += kNumEpiThreads) {
             const int g = i / HP, h = i % HP, b = b0 + g;
             wslot[i] = (g < a.G && h < a.H_I && b < a.B) ? a.w[static_cast<int64_t>(b) * a.H_I + h] : 0.f;
@@ -280,9 +268,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
             nvs[slot * 16 + et] = (et < a.G && b < a.B) ? (a.n_valid ? a.n_valid[b] : a.N) : 0;
           }
         }
-        fence_proxy_async_smem();
         named_bar_sync(1, kNumEpiThreads);
-        if (et == 0) mbar_arrive(q_ready);
         cur_grp = grp;
       }
       for (int sub = 0; sub < ng; ++sub, ++si) {
@@ -492,24 +478,25 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
 }
 
 template <int D_I, int HP, bool FP8, bool PAIR>
-cudaError_t launch_indexer_inst(const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t stream,
-                                bool pdl) {
+cudaError_t launch_indexer_inst(const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int grid,
+                                cudaStream_t stream, bool pdl) {
   using C = IdxCfg<D_I, FP8, PAIR>;
   auto kern = indexer_tc_kernel<D_I, HP, FP8, PAIR>;
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  e = launch_kernel(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, pdl, map, a);
+  e = launch_kernel(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, pdl, map, qmap, a);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D_I, bool FP8, bool PAIR>
-cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const IndexerArgs& a, int grid, cudaStream_t s, bool pdl) {
+cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int grid,
+                        cudaStream_t s, bool pdl) {
   switch (HP) {
-    case 16: return launch_indexer_inst<D_I, 16, FP8, PAIR>(map, a, grid, s, pdl);
-    case 32: return launch_indexer_inst<D_I, 32, FP8, PAIR>(map, a, grid, s, pdl);
-    case 64: return launch_indexer_inst<D_I, 64, FP8, PAIR>(map, a, grid, s, pdl);
-    case 128: return launch_indexer_inst<D_I, 128, FP8, PAIR>(map, a, grid, s, pdl);
+    case 16: return launch_indexer_inst<D_I, 16, FP8, PAIR>(map, qmap, a, grid, s, pdl);
+    case 32: return launch_indexer_inst<D_I, 32, FP8, PAIR>(map, qmap, a, grid, s, pdl);
+    case 64: return launch_indexer_inst<D_I, 64, FP8, PAIR>(map, qmap, a, grid, s, pdl);
+    case 128: return launch_indexer_inst<D_I, 128, FP8, PAIR>(map, qmap, a, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -521,20 +508,20 @@ int indexer_smem_bytes(int d_I, bool fp8) {
   return fp8 ? IdxCfg<128, true, false>::kSmemBytes : IdxCfg<128, false, true>::kSmemBytes;
 }
 
-cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
-                           cudaStream_t stream, bool pdl) {
+cudaError_t launch_indexer(const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int HP, int d_I,
+                           bool fp8, int grid, cudaStream_t stream, bool pdl) {
   if (fp8) {
-    if (d_I == 64) return dispatch_hp<64, true, false>(HP, map, a, grid, stream, pdl);
-    if (d_I == 128) return dispatch_hp<128, true, false>(HP, map, a, grid, stream, pdl);
+    if (d_I == 64) return dispatch_hp<64, true, false>(HP, map, qmap, a, grid, stream, pdl);
+    if (d_I == 128) return dispatch_hp<128, true, false>(HP, map, qmap, a, grid, stream, pdl);
     return cudaErrorInvalidValue;
   }
   if (a.pair == 2) {
-    if (d_I == 64) return dispatch_hp<64, false, true>(HP, map, a, grid, stream, pdl);
-    if (d_I == 128) return dispatch_hp<128, false, true>(HP, map, a, grid, stream, pdl);
+    if (d_I == 64) return dispatch_hp<64, false, true>(HP, map, qmap, a, grid, stream, pdl);
+    if (d_I == 128) return dispatch_hp<128, false, true>(HP, map, qmap, a, grid, stream, pdl);
     return cudaErrorInvalidValue;
   }
-  if (d_I == 64) return dispatch_hp<64, false, false>(HP, map, a, grid, stream, pdl);
-  if (d_I == 128) return dispatch_hp<128, false, false>(HP, map, a, grid, stream, pdl);
+  if (d_I == 64) return dispatch_hp<64, false, false>(HP, map, qmap, a, grid, stream, pdl);
+  if (d_I == 128) return dispatch_hp<128, false, false>(HP, map, qmap, a, grid, stream, pdl);
   return cudaErrorInvalidValue;
 }
 

@@ -89,8 +89,10 @@ struct IndexerArgs {
 };
 
 int indexer_smem_bytes(int d_I, bool fp8);
-cudaError_t launch_indexer(const CUtensorMap& map, const IndexerArgs& a, int HP, int d_I, bool fp8, int grid,
-                           cudaStream_t stream, bool pdl);
+// map: the key cache (d_I, N, batch), 128-key boxes; qmap: the queries (d_I, H_I, B)
+// with (64, HP, G) boxes, both 128-byte swizzled (e4m3 keys: unswizzled rows).
+cudaError_t launch_indexer(const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int HP, int d_I,
+                           bool fp8, int grid, cudaStream_t stream, bool pdl);
 
 // 32-bit words of per-row top-k control state (one 128-byte line per row,
 // so rows do not contend for the same line in L2).
