@@ -344,19 +344,21 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         if constexpr (kPerWait == 1) {
           const int c0 = kC0 * 32;
           if (c0 + kChunks * 32 <= ncols) {
-            // every column of the half is present: 32-column TMEM loads, the
+            // every column of the half is present: 64-column TMEM loads, the
             // next one in flight while the current one is reduced
-            uint32_t r0[32], r1[32];
-            tmem_ld32_issue(taddr + c0, r0);
-            tmem_ld_wait(r0);
+            uint32_t ra[64], rb[64];
+            tmem_ld64_issue(taddr + c0, ra);
+            tmem_ld_wait64(ra);
 #pragma unroll
-            for (int c = 0; c < kChunks; c += 2) {
-              tmem_ld32_issue(taddr + c0 + (c + 1) * 32, r1);
-              reduce32(r0, 0, c0 + c * 32);
-              tmem_ld_wait(r1);
-              if (c + 2 < kChunks) tmem_ld32_issue(taddr + c0 + (c + 2) * 32, r0);
-              reduce32(r1, 0, c0 + (c + 1) * 32);
-              if (c + 2 < kChunks) tmem_ld_wait(r0);
+            for (int c = 0; c < kLoads; c += 2) {
+              tmem_ld64_issue(taddr + c0 + (c + 1) * 64, rb);
+              reduce32(ra, 0, c0 + c * 64);
+              reduce32(ra, 32, c0 + c * 64 + 32);
+              tmem_ld_wait64(rb);
+              if (c + 2 < kLoads) tmem_ld64_issue(taddr + c0 + (c + 2) * 64, ra);
+              reduce32(rb, 0, c0 + (c + 1) * 64);
+              reduce32(rb, 32, c0 + (c + 1) * 64 + 32);
+              if (c + 2 < kLoads) tmem_ld_wait64(ra);
             }
           } else {
             // a partial half: one 64-column load at a time
