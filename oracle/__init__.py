@@ -20,3 +20,11 @@ from .indexcache_oracle import (  # noqa: F401
     validate_schedule,
     governing_full_layer,
 )
+from .cache_append_oracle import (  # noqa: F401
+    layernorm_bias,
+    encode_e4m3,
+    rope_interleaved,
+    quantize_key_e4m3,
+    cache_append,
+    rope_query,
+)
