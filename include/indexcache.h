@@ -213,6 +213,48 @@ ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule
 size_t ic_layer_stack_workspace_size(const ic_stack_shape_t* shape);
 
 /* ---------------------------------------------------------------------------
+ * ic_cache_append -- the cache-append step for T new tokens, run before the
+ * decode step (Hy4-preview porting issue: "Indexer" bullet, the indexer key
+ * goes through a LayerNorm with bias; "RoPE is interleaved" bullet,
+ * is_neox_style=False: adjacent pairs of the 64 rotary dims rotate).
+ *
+ * Token t writes row r = pos[t] of cache c (c = t where a batch stride is
+ * nonzero, the single shared cache where it is 0):
+ *   y = (k_raw[t] - mean) / sqrt(var + ln_eps) * ln_gamma + ln_beta
+ *       (mean and population variance over the d_I dims)
+ *   k_dtype IC_BF16:     key row = bf16(y)  (round to nearest even)
+ *   k_dtype IC_FP8_E4M3: key_scale[r] = max|y| / 448 (1 if y is all zero),
+ *                        key row = e4m3(y / key_scale[r]), round to nearest
+ *                        even, saturating at +-448
+ *   kv row  = kv_raw[t] with each rotary pair i < 32 of dims [512, 576)
+ *             (a, b) = (x[512+2i], x[513+2i]) -> (a cos - b sin, a sin + b cos),
+ *             angle = r * rope_base^(-2i/64), result rounded to bf16
+ * If q is not NULL, the rotary dims of every head of query b < B are
+ * rotated the same way in place by the angle of position q_pos[b].
+ *
+ *   k_raw      [T, d_I] bf16.  ln_gamma, ln_beta [d_I] fp32.
+ *   key_cache  [N, d_I] bf16 or e4m3 bytes per cache, caches k_batch_stride
+ *              elements apart; key_scale [N] fp32 per cache,
+ *              scale_batch_stride apart (e4m3 only; NULL for bf16).
+ *   kv_raw     [T, 576] bf16.  kv_cache [N, 576] bf16 per cache,
+ *              kv_batch_stride elements apart.
+ *   pos        [T] int64 device.  A row outside [0, N) is not written and
+ *              the status word records IC_ERR_BAD_INDEX.
+ *   q          [B, H, 576] bf16 or NULL.  q_pos [B] int64 device.
+ *   Supported: T >= 1, N >= 1, d_I in {64, 128}; ln_eps >= 0 and
+ *   rope_base > 0, both finite. Pointers 16-byte aligned. Two tokens of one
+ *   call must not write the same row. The caller owns every buffer.
+ *   workspace >= ic_cache_append_workspace_size() bytes (status word).
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_cache_append(const void* k_raw, const float* ln_gamma, const float* ln_beta, float ln_eps,
+                            ic_dtype_t k_dtype, void* key_cache, float* key_scale, int64_t k_batch_stride,
+                            int64_t scale_batch_stride, const void* kv_raw, void* kv_cache,
+                            int64_t kv_batch_stride, const int64_t* pos, int T, int d_I, int64_t N,
+                            float rope_base, void* q, const int64_t* q_pos, int B, int H, void* workspace,
+                            size_t ws_bytes, ic_stream_t stream);
+size_t ic_cache_append_workspace_size(void);
+
+/* ---------------------------------------------------------------------------
  * ic_last_device_status -- synchronises `stream`, then reads and clears the
  * device status word at the start of `workspace` (any of the workspaces
  * above). Returns IC_OK, IC_ERR_TIMEOUT or IC_ERR_BAD_INDEX (or IC_ERR_CUDA

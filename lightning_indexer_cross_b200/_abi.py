@@ -35,6 +35,8 @@ EXPORTED = [
     "ic_sparse_mla_workspace_size",
     "ic_layer_stack",
     "ic_layer_stack_workspace_size",
+    "ic_cache_append",
+    "ic_cache_append_workspace_size",
     "ic_last_device_status",
     "ic_last_launch_count",
 ]
@@ -95,6 +97,10 @@ _stack = _sig("ic_layer_stack", _i,
               [ctypes.POINTER(ic_layer_t), _i, ctypes.c_char_p, ctypes.POINTER(ic_stack_shape_t), _p, _p, _p,
                _sz, _p])
 _stack_ws = _sig("ic_layer_stack_workspace_size", _sz, [ctypes.POINTER(ic_stack_shape_t)])
+_append = _sig("ic_cache_append", _i,
+               [_p, _p, _p, _f, _i, _p, _p, _i64, _i64, _p, _p, _i64, _p, _i, _i, _i64, _f, _p, _p, _i, _i, _p, _sz,
+                _p])
+_append_ws = _sig("ic_cache_append_workspace_size", _sz, [])
 _last_status = _sig("ic_last_device_status", _i, [_p, _p])
 _last_launches = _sig("ic_last_launch_count", _i, [])
 
@@ -151,6 +157,18 @@ def ic_layer_stack(layers, L, schedule: bytes, shape, index_buf, idx_trace, work
 
 def ic_layer_stack_workspace_size(shape) -> int:
     return int(_stack_ws(ctypes.byref(shape)))
+
+
+def ic_cache_append(k_raw, ln_gamma, ln_beta, ln_eps, k_dtype, key_cache, key_scale, k_batch_stride,
+                    scale_batch_stride, kv_raw, kv_cache, kv_batch_stride, pos, T, d_I, N, rope_base, q, q_pos, B,
+                    H, workspace, ws_bytes, stream) -> None:
+    _check(_append(k_raw, ln_gamma, ln_beta, ln_eps, k_dtype, key_cache, key_scale, k_batch_stride,
+                   scale_batch_stride, kv_raw, kv_cache, kv_batch_stride, pos, T, d_I, N, rope_base, q, q_pos, B, H,
+                   workspace, ws_bytes, stream), "ic_cache_append")
+
+
+def ic_cache_append_workspace_size() -> int:
+    return int(_append_ws())
 
 
 def ic_last_device_status(workspace, stream) -> int:

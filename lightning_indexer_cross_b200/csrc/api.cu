@@ -2,6 +2,7 @@
 // any launch), workspace layouts, TMA descriptor encoding, and the F/S layer
 // stack driver (Hy4-preview porting issue, "Indexer" bullet: shared layers
 // reuse the last preceding full layer's top-k).
+#include <cmath>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -468,6 +469,66 @@ ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule
     }
   }
   g_launches = total;
+  return IC_OK;
+}
+
+size_t ic_cache_append_workspace_size(void) { return kStatusBytes; }
+
+ic_status_t ic_cache_append(const void* k_raw, const float* ln_gamma, const float* ln_beta, float ln_eps,
+                            ic_dtype_t k_dtype, void* key_cache, float* key_scale, int64_t k_batch_stride,
+                            int64_t scale_batch_stride, const void* kv_raw, void* kv_cache,
+                            int64_t kv_batch_stride, const int64_t* pos, int T, int d_I, int64_t N,
+                            float rope_base, void* q, const int64_t* q_pos, int B, int H, void* workspace,
+                            size_t ws_bytes, ic_stream_t stream) {
+  g_launches = 0;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
+  if (!k_raw || !ln_gamma || !ln_beta || !key_cache || !kv_raw || !kv_cache || !pos) return IC_ERR_INVALID_ARG;
+  if (T < 1 || N < 1) return IC_ERR_INVALID_ARG;
+  if (k_dtype != IC_BF16 && k_dtype != IC_FP8_E4M3) return IC_ERR_UNSUPPORTED;
+  if (d_I != 64 && d_I != 128) return IC_ERR_UNSUPPORTED;
+  const bool fp8 = k_dtype == IC_FP8_E4M3;
+  if (fp8 != (key_scale != nullptr)) return IC_ERR_INVALID_ARG;
+  if (!(ln_eps >= 0.f) || !std::isfinite(ln_eps) || !(rope_base > 0.f) || !std::isfinite(rope_base))
+    return IC_ERR_INVALID_ARG;
+  if (!aligned16(k_raw) || !aligned16(key_cache) || !aligned16(kv_raw) || !aligned16(kv_cache) ||
+      (q && !aligned16(q)))
+    return IC_ERR_INVALID_ARG;
+  const int64_t esz = fp8 ? 1 : 2;
+  if (k_batch_stride < 0 || scale_batch_stride < 0 || kv_batch_stride < 0) return IC_ERR_INVALID_ARG;
+  // nonzero strides: token t writes cache t, which must not overlap cache t+1
+  if (k_batch_stride != 0 && (k_batch_stride < N * d_I || (k_batch_stride * esz) % 16 != 0))
+    return IC_ERR_INVALID_ARG;
+  if (kv_batch_stride != 0 && (kv_batch_stride < N * 576 || (kv_batch_stride * 2) % 16 != 0))
+    return IC_ERR_INVALID_ARG;
+  if (fp8 && scale_batch_stride != 0 && scale_batch_stride < N) return IC_ERR_INVALID_ARG;
+  if (q && (!q_pos || B < 1 || H < 1)) return IC_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) + (q ? B : 0) >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+
+  ic::AppendArgs a{};
+  a.k_raw = static_cast<const __nv_bfloat16*>(k_raw);
+  a.gamma = ln_gamma;
+  a.beta = ln_beta;
+  a.eps = ln_eps;
+  a.fp8 = fp8 ? 1 : 0;
+  a.key_cache = key_cache;
+  a.key_scale = key_scale;
+  a.k_bs = k_batch_stride;
+  a.s_bs = fp8 ? scale_batch_stride : 0;
+  a.kv_bs = kv_batch_stride;
+  a.kv_raw = static_cast<const __nv_bfloat16*>(kv_raw);
+  a.kv_cache = static_cast<__nv_bfloat16*>(kv_cache);
+  a.pos = pos;
+  a.T = T;
+  a.d_I = d_I;
+  a.N = N;
+  a.log2_base = std::log2(static_cast<double>(rope_base));
+  a.q = static_cast<__nv_bfloat16*>(q);
+  a.q_pos = q_pos;
+  a.B = q ? B : 0;
+  a.H = q ? H : 0;
+  a.status = static_cast<int*>(workspace);
+  if (ic::launch_cache_append(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;
+  g_launches = 1;
   return IC_OK;
 }
 

@@ -163,4 +163,27 @@ int mla_smem_bytes(int ts);
 cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a,
                               cudaStream_t stream, bool pdl, int* launches);
 
+// ---------------------------------------------------------------- cache append
+struct AppendArgs {
+  const __nv_bfloat16* k_raw;    // [T, d_I] indexer keys before the norm
+  const float* gamma;            // [d_I] LayerNorm weight
+  const float* beta;             // [d_I] LayerNorm bias
+  float eps;
+  int fp8;                       // key cache holds e4m3 codes + per-token scales
+  void* key_cache;               // bf16 elements or e4m3 bytes
+  float* key_scale;              // e4m3 only
+  int64_t k_bs, s_bs, kv_bs;     // per-token cache strides (elements; 0 = one shared cache)
+  const __nv_bfloat16* kv_raw;   // [T, 576] latent rows, rotary dims unrotated
+  __nv_bfloat16* kv_cache;
+  const int64_t* pos;            // [T] destination row = position
+  int T, d_I;
+  int64_t N;                     // rows per cache
+  double log2_base;              // log2 of the RoPE base
+  __nv_bfloat16* q;              // [B, H, 576] rotated in place, or null
+  const int64_t* q_pos;          // [B]
+  int B, H;
+  int* status;
+};
+cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t stream);
+
 }  // namespace ic

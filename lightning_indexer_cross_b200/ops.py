@@ -101,6 +101,40 @@ def sparse_mla_decode(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sink
     return out, lse
 
 
+def cache_append(k_raw: torch.Tensor, ln_gamma: torch.Tensor, ln_beta: torch.Tensor, kv_raw: torch.Tensor,
+                 pos: torch.Tensor, key_cache: torch.Tensor, kv_cache: torch.Tensor,
+                 key_scale: Optional[torch.Tensor] = None, ln_eps: float = 1e-6, rope_base: float = 10000.0,
+                 q: Optional[torch.Tensor] = None, q_pos: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Append T new tokens: LayerNorm-with-bias of k_raw [T, d_I] into row pos[t] of key_cache (bf16, or
+    uint8 e4m3 codes with per-token key_scale), kv_raw [T, 576] into kv_cache with its rotary dims
+    [512, 576) rotated (interleaved pairs) to pos[t]; if q [B, H, 576] is given, its rotary dims are
+    rotated in place to q_pos[b]. Caches are [C, N, ...] with C == 1 (one shared cache) or C == T (token t
+    writes cache t). Returns the workspace (its status word records out-of-range rows)."""
+    _need_cuda(k_raw, ln_gamma, ln_beta, kv_raw, pos, key_cache, kv_cache, key_scale, q, q_pos)
+    T, d_I = k_raw.shape
+    C, N, dk = key_cache.shape
+    assert k_raw.dtype == torch.bfloat16 and kv_raw.dtype == torch.bfloat16 and kv_cache.dtype == torch.bfloat16
+    assert ln_gamma.dtype == torch.float32 and ln_beta.dtype == torch.float32 and pos.dtype == torch.int64
+    assert dk == d_I and kv_raw.shape == (T, D_QK) and kv_cache.shape == (C, N, D_QK) and C in (1, T)
+    fp8 = key_cache.dtype == torch.uint8
+    assert key_cache.dtype in (torch.bfloat16, torch.uint8) and (key_scale is not None) == fp8
+    B = H = 0
+    if q is not None:
+        B, H, D = q.shape
+        assert D == D_QK and q.dtype == torch.bfloat16 and q_pos is not None and q_pos.dtype == torch.int64
+    if workspace is None:
+        workspace = new_workspace(_abi.ic_cache_append_workspace_size(), k_raw.device)
+    kbs = key_cache.stride(0) if C > 1 else 0
+    sbs = key_scale.stride(0) if (fp8 and C > 1) else 0
+    kvbs = kv_cache.stride(0) if C > 1 else 0
+    _abi.ic_cache_append(_ptr(k_raw), _ptr(ln_gamma), _ptr(ln_beta), ln_eps,
+                         _abi.IC_FP8_E4M3 if fp8 else _abi.IC_BF16, _ptr(key_cache), _ptr(key_scale), kbs, sbs,
+                         _ptr(kv_raw), _ptr(kv_cache), kvbs, _ptr(pos), T, d_I, N, rope_base, _ptr(q), _ptr(q_pos),
+                         B, H, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    return workspace
+
+
 class LayerStack:
     """Holds the per-layer pointer table, the shape struct, the index buffer
     and the workspace of one decode stack, so that a step is one C call."""

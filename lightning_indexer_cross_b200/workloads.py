@@ -302,3 +302,43 @@ def attention_case(B, N, H, k, shared=False, gate=True, n_invalid=0, seed=13, de
         if n_invalid:
             idx[b, k - n_invalid:] = -1
     return q, kv, idx, sink, gt
+
+
+def append_case(T, N, d_I, per_token=False, fp8=False, B=0, H=128, seed=14, device="cpu"):
+    """Inputs of the cache-append step: T new tokens' raw indexer keys
+    [T, d_I] bf16 (mean offset and spread so the norm has work to do),
+    LayerNorm weight ~ 1 + N(0, 0.1) and bias ~ N(0, 0.1) fp32, raw latent
+    rows [T, 576] bf16, destination rows (distinct for one shared cache;
+    0 and N-1 always among them), caches [C, N, ...] pre-filled with random
+    bytes (C = T per-token caches, else 1), and optionally queries
+    [B, H, 576] bf16 with positions q_pos [B] (0, 1, N-1 and 1000003 first)."""
+    g = _gen(seed, device)
+    k_raw = (_randn((T, d_I), g, device, 2.0) + 0.5).to(torch.bfloat16)
+    gamma = 1.0 + _randn((d_I,), g, device, 0.1)
+    beta = _randn((d_I,), g, device, 0.1)
+    kv_raw = _randn((T, D_QK), g, device).to(torch.bfloat16)
+    if per_token:
+        pos = torch.randint(0, N, (T,), generator=g, device=device)
+        pos[0] = 0
+        if T > 1:
+            pos[T - 1] = N - 1
+    else:  # distinct rows: 0, T - 2 others from [1, N - 2], N - 1
+        assert T <= N and (T == 1 or N >= 2)
+        mid = torch.randperm(max(N - 2, 0), generator=g, device=device)[:max(T - 2, 0)] + 1
+        ends = [torch.zeros(1, dtype=mid.dtype, device=device)]
+        pos = torch.cat(ends + ([mid, torch.full((1,), N - 1, dtype=mid.dtype, device=device)] if T > 1 else []))
+    pos = pos.to(torch.int64)
+    C = T if per_token else 1
+    kc_bytes = torch.randint(0, 256, (C, N, d_I * (1 if fp8 else 2)), generator=g, device=device, dtype=torch.uint8)
+    key_cache = kc_bytes if fp8 else kc_bytes.view(torch.bfloat16)
+    # finite bf16 filler for the latent cache (random bytes could be NaN)
+    kv_cache = _randn((C, N, D_QK), g, device).to(torch.bfloat16)
+    key_scale = _rand((C, N), g, device) if fp8 else None
+    q = q_pos = None
+    if B:
+        q = _randn((B, H, D_QK), g, device).to(torch.bfloat16)
+        q_pos = torch.randint(0, 1 << 20, (B,), generator=g, device=device).to(torch.int64)
+        for i, v in enumerate([0, 1, N - 1, 1000003][:B]):
+            q_pos[i] = v
+    return dict(k_raw=k_raw, gamma=gamma, beta=beta, kv_raw=kv_raw, pos=pos, key_cache=key_cache,
+                kv_cache=kv_cache, key_scale=key_scale, q=q, q_pos=q_pos)

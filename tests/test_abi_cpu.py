@@ -93,6 +93,35 @@ def test_sparse_mla_rejects_bad_arguments(abi):
     assert call(wsb=64) == abi.IC_ERR_INVALID_ARG
 
 
+def test_cache_append_rejects_bad_arguments(abi):
+    # every case below must fail validation: the pointers are host memory
+    p, keep = _fake()
+    call = lambda **kw: abi._append(*[kw.get(n, d) for n, d in [
+        ("kr", p), ("g", p), ("b", p), ("eps", 1e-6), ("dt", abi.IC_BF16), ("kc", p), ("ks", None), ("kbs", 0),
+        ("sbs", 0), ("kvr", p), ("kvc", p), ("kvbs", 0), ("pos", p), ("T", 4), ("d", 128), ("N", 100),
+        ("base", 10000.0), ("q", None), ("qp", None), ("B", 0), ("H", 0), ("ws", p), ("wsb", 256), ("st", None)]])
+    assert call(kr=None) == abi.IC_ERR_INVALID_ARG
+    assert call(pos=None) == abi.IC_ERR_INVALID_ARG
+    assert call(T=0) == abi.IC_ERR_INVALID_ARG
+    assert call(N=0) == abi.IC_ERR_INVALID_ARG
+    assert call(d=96) == abi.IC_ERR_UNSUPPORTED
+    assert call(dt=abi.IC_F32) == abi.IC_ERR_UNSUPPORTED
+    assert call(dt=abi.IC_FP8_E4M3) == abi.IC_ERR_INVALID_ARG  # e4m3 keys need their scales
+    assert call(ks=p) == abi.IC_ERR_INVALID_ARG                 # bf16 keys take none
+    assert call(eps=-1.0) == abi.IC_ERR_INVALID_ARG
+    assert call(eps=float("inf")) == abi.IC_ERR_INVALID_ARG
+    assert call(base=0.0) == abi.IC_ERR_INVALID_ARG
+    assert call(base=float("nan")) == abi.IC_ERR_INVALID_ARG
+    assert call(kc=ctypes.c_void_p(p.value + 8)) == abi.IC_ERR_INVALID_ARG  # misaligned
+    assert call(kbs=100 * 128 - 1) == abi.IC_ERR_INVALID_ARG   # caches would overlap
+    assert call(kvbs=576) == abi.IC_ERR_INVALID_ARG
+    assert call(q=p) == abi.IC_ERR_INVALID_ARG                  # q needs q_pos, B and H
+    assert call(q=p, qp=p, B=2, H=0) == abi.IC_ERR_INVALID_ARG
+    assert call(wsb=16) == abi.IC_ERR_INVALID_ARG
+    assert call(ws=None) == abi.IC_ERR_INVALID_ARG
+    assert abi.ic_cache_append_workspace_size() >= 4
+
+
 @pytest.mark.parametrize("sched", [b"SFFF", b"FXSS", b"FS", b"FSSSS", b"", b"fsss"])
 def test_stack_rejects_bad_schedules(abi, sched):
     p, keep = _fake()
