@@ -313,6 +313,10 @@ def run_native(args):
 
     # ------------------------------------------------------------------ per-kernel timing
     kern = time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst)
+    try:  # reported beside the step, never part of it; a failure here is recorded, not fatal
+        kern["cache_append"] = time_cache_append(dev, hbm_gbs)
+    except Exception as e:  # noqa: BLE001
+        kern["cache_append"] = {"error": f"{type(e).__name__}: {e}"}
     clk.stop()
     clocks = clk.summary()
 
@@ -468,6 +472,37 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
                        "distinct_rows_per_layer": mla_rows,
                        "roofline": roofline(mla_bytes, mla_flops, t_mla)},
     }
+
+
+def time_cache_append(dev, hbm_gbs):
+    """The cache-append step that precedes each decode step (not inside the
+    step's timed region): one launch per layer writes the 32 queries' new
+    tokens into a 131072-row shared cache (bf16 LayerNorm'd keys, latent rows
+    with rotated rotary dims) and rotates the 32 queries' rotary dims, timed
+    like the other kernels (graph of L launches, events on their stream)."""
+    import torch
+    from lightning_indexer_cross_b200 import _abi, ops, workloads as Wl
+    stream = torch.cuda.Stream(device=dev)
+    c = Wl.append_case(B, N, D_I, per_token=False, fp8=False, B=B, H=H, seed=70, device=dev)
+    ws = ops.new_workspace(_abi.ic_cache_append_workspace_size(), dev)
+
+    def app(i):
+        ops.cache_append(c["k_raw"], c["gamma"], c["beta"], c["kv_raw"], c["pos"], c["key_cache"], c["kv_cache"],
+                         q=c["q"], q_pos=c["q_pos"], workspace=ws)
+
+    for i in range(3):
+        app(i)
+    torch.cuda.synchronize()
+    us = _time_loop(app, L, stream)
+    if _abi.ic_last_device_status(ops._ptr(ws), ops._stream_ptr()) != _abi.IC_OK:
+        raise RuntimeError("device status not OK after the cache-append launches")
+    # algorithmic bytes per launch: key rows in and out, latent rows in and
+    # out, the queries' rotary dims in and out, LayerNorm parameters, rows
+    bytes_ = (B * (D_I * 2 * 2 + D_QK * 2 * 2) + B * H * (D_QK - D_V) * 2 * 2 + 2 * D_I * 4 + 2 * B * 8)
+    ach = bytes_ / (us * 1e-6) / 1e9
+    return {"us": us, "launches": L, "tokens_per_launch": B,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s", "frac": ach / hbm_gbs,
+                         "algorithmic_bytes": bytes_, "algorithmic_flops": 0.0}}
 
 
 def time_e2e(wl, st, args, dev, world):
