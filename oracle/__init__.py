@@ -28,3 +28,4 @@ from .cache_append_oracle import (  # noqa: F401
     cache_append,
     rope_query,
 )
+from .gate_oracle import decompress, decompressed_gate  # noqa: F401
