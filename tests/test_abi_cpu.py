@@ -156,6 +156,16 @@ def test_ops_refuse_cpu_tensors(abi):
     q = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.indexer_score(q, torch.zeros(1, 4), torch.zeros(1, 10, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        ops.topk(torch.zeros(1, 10), 4)
+    with pytest.raises(ValueError):
+        ops.sparse_mla_decode(torch.zeros(1, 8, 576, dtype=torch.bfloat16),
+                              torch.zeros(1, 10, 576, dtype=torch.bfloat16),
+                              torch.zeros(1, 4, dtype=torch.int32), torch.zeros(8))
+    with pytest.raises(ValueError):
+        ops.cache_append(torch.zeros(2, 64, dtype=torch.bfloat16), torch.ones(64), torch.zeros(64),
+                         torch.zeros(2, 576, dtype=torch.bfloat16), torch.zeros(2, dtype=torch.int64),
+                         torch.zeros(1, 10, 64, dtype=torch.bfloat16), torch.zeros(1, 10, 576, dtype=torch.bfloat16))
 
 
 def test_layer_struct_matches_header(abi):
