@@ -255,6 +255,28 @@ ic_status_t ic_cache_append(const void* k_raw, const float* ln_gamma, const floa
 size_t ic_cache_append_workspace_size(void);
 
 /* ---------------------------------------------------------------------------
+ * ic_decompress_gate -- the output gate in the decompressed space
+ * (Hy4-preview porting issue, gate bullet: the elementwise sigmoid gate
+ * multiplies the decompressed per-head attention output, after the value
+ * up-projection wv_b and before o_proj).
+ *
+ *   v[b,h,:]   = wv_b[h] @ o_latent[b,h,:]      (512 -> d_v per head)
+ *   out[b,h,:] = sigmoid(gate[b,h,:]) * v[b,h,:]   (gate NULL: out = v)
+ *
+ *   o_latent  [B, H, 512] bf16: the ungated sparse-attention output
+ *             (ic_sparse_mla_decode with gate NULL and out_dtype IC_BF16).
+ *   wv_b      [H, d_v, 512] bf16 (out x in per head).
+ *   gate      [B, H, d_v] bf16 gate logits, or NULL.
+ *   out       [B, H, d_v], bf16 (IC_BF16) or fp32 (IC_F32).
+ *   Supported: d_v = 128; B, H >= 1. Pointers 16-byte aligned.
+ *   workspace >= ic_decompress_gate_workspace_size() bytes (status word).
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_decompress_gate(const void* o_latent, const void* wv_b, const void* gate, int B, int H, int d_v,
+                               ic_dtype_t out_dtype, void* out, void* workspace, size_t ws_bytes,
+                               ic_stream_t stream);
+size_t ic_decompress_gate_workspace_size(void);
+
+/* ---------------------------------------------------------------------------
  * ic_last_device_status -- synchronises `stream`, then reads and clears the
  * device status word at the start of `workspace` (any of the workspaces
  * above). Returns IC_OK, IC_ERR_TIMEOUT or IC_ERR_BAD_INDEX (or IC_ERR_CUDA

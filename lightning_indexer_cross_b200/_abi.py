@@ -37,6 +37,8 @@ EXPORTED = [
     "ic_layer_stack_workspace_size",
     "ic_cache_append",
     "ic_cache_append_workspace_size",
+    "ic_decompress_gate",
+    "ic_decompress_gate_workspace_size",
     "ic_last_device_status",
     "ic_last_launch_count",
 ]
@@ -101,6 +103,8 @@ _append = _sig("ic_cache_append", _i,
                [_p, _p, _p, _f, _i, _p, _p, _i64, _i64, _p, _p, _i64, _p, _i, _i, _i64, _f, _p, _p, _i, _i, _p, _sz,
                 _p])
 _append_ws = _sig("ic_cache_append_workspace_size", _sz, [])
+_gate = _sig("ic_decompress_gate", _i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz, _p])
+_gate_ws = _sig("ic_decompress_gate_workspace_size", _sz, [])
 _last_status = _sig("ic_last_device_status", _i, [_p, _p])
 _last_launches = _sig("ic_last_launch_count", _i, [])
 
@@ -169,6 +173,15 @@ def ic_cache_append(k_raw, ln_gamma, ln_beta, ln_eps, k_dtype, key_cache, key_sc
 
 def ic_cache_append_workspace_size() -> int:
     return int(_append_ws())
+
+
+def ic_decompress_gate(o_latent, wv_b, gate, B, H, d_v, out_dtype, out, workspace, ws_bytes, stream) -> None:
+    _check(_gate(o_latent, wv_b, gate, B, H, d_v, out_dtype, out, workspace, ws_bytes, stream),
+           "ic_decompress_gate")
+
+
+def ic_decompress_gate_workspace_size() -> int:
+    return int(_gate_ws())
 
 
 def ic_last_device_status(workspace, stream) -> int:

@@ -532,6 +532,53 @@ ic_status_t ic_cache_append(const void* k_raw, const float* ln_gamma, const floa
   return IC_OK;
 }
 
+size_t ic_decompress_gate_workspace_size(void) { return kStatusBytes; }
+
+ic_status_t ic_decompress_gate(const void* o_latent, const void* wv_b, const void* gate, int B, int H, int d_v,
+                               ic_dtype_t out_dtype, void* out, void* workspace, size_t ws_bytes,
+                               ic_stream_t stream) {
+  g_launches = 0;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
+  if (!o_latent || !wv_b || !out || B < 1 || H < 1) return IC_ERR_INVALID_ARG;
+  if (d_v != 128) return IC_ERR_UNSUPPORTED;
+  if (out_dtype != IC_BF16 && out_dtype != IC_F32) return IC_ERR_UNSUPPORTED;
+  if (!aligned16(o_latent) || !aligned16(wv_b) || !aligned16(out) || (gate && !aligned16(gate)))
+    return IC_ERR_INVALID_ARG;
+  if (ceil_div<int64_t>(B, 128) * H >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return IC_ERR_CUDA;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  // wv_b (512, d_v, H): one box = 64 latent dims of a head's 128 weight rows
+  CUtensorMap wmap;
+  const cuuint64_t wdims[3] = {512, static_cast<cuuint64_t>(d_v), static_cast<cuuint64_t>(H)};
+  const cuuint64_t wstrides[2] = {512 * 2, static_cast<cuuint64_t>(d_v) * 512 * 2};
+  const cuuint32_t wbox[3] = {64, 128, 1};
+  CUresult r = enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(wv_b), wdims, wstrides, wbox,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
+  // latent outputs (512, H, B): one box = 64 latent dims of one head for 128
+  // queries (queries past B read as zeros)
+  CUtensorMap omap;
+  const cuuint64_t odims[3] = {512, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t ostrides[2] = {512 * 2, static_cast<cuuint64_t>(H) * 512 * 2};
+  const cuuint32_t obox[3] = {64, 1, 128};
+  r = enc(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(o_latent), odims, ostrides, obox, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
+  ic::GateArgs a{};
+  a.gate = static_cast<const __nv_bfloat16*>(gate);
+  a.out = out;
+  a.out_f32 = out_dtype == IC_F32 ? 1 : 0;
+  a.B = B;
+  a.H = H;
+  a.status = static_cast<int*>(workspace);
+  if (ic::launch_gate(wmap, omap, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;
+  g_launches = 1;
+  return IC_OK;
+}
+
 ic_status_t ic_last_device_status(void* workspace, ic_stream_t stream) {
   if (!workspace) return IC_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;

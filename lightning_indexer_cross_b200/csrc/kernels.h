@@ -186,4 +186,18 @@ struct AppendArgs {
 };
 cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t stream);
 
+// ---------------------------------------------------------------- output gate
+struct GateArgs {
+  const __nv_bfloat16* gate;  // [B, H, 128] or null (identity)
+  void* out;                  // [B, H, 128] bf16 or fp32
+  int out_f32;
+  int B, H;
+  int* status;
+};
+int gate_smem_bytes();
+// wmap: 3-D tensor map over wv_b (512, 128, H), box 64 x 128 x 1; omap: 3-D
+// over the latent outputs (512, H, B), box 64 x 1 x 128; both bf16 with the
+// 128-byte swizzle.
+cudaError_t launch_gate(const CUtensorMap& wmap, const CUtensorMap& omap, const GateArgs& a, cudaStream_t stream);
+
 }  // namespace ic

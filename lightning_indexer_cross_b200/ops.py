@@ -101,6 +101,26 @@ def sparse_mla_decode(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sink
     return out, lse
 
 
+def decompress_gate(o_latent: torch.Tensor, wv_b: torch.Tensor, gate: Optional[torch.Tensor] = None,
+                    out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[b,h] = sigmoid(gate[b,h]) * (wv_b[h] @ o_latent[b,h]): o_latent [B,H,512] bf16 (ungated attention
+    output), wv_b [H,128,512] bf16, gate [B,H,128] bf16 or None."""
+    _need_cuda(o_latent, wv_b, gate, out)
+    B, H, K = o_latent.shape
+    Hw, d_v, Kw = wv_b.shape
+    assert K == D_V and Kw == D_V and Hw == H
+    assert o_latent.dtype == torch.bfloat16 and wv_b.dtype == torch.bfloat16
+    assert gate is None or (gate.shape == (B, H, d_v) and gate.dtype == torch.bfloat16)
+    if out is None:
+        out = torch.empty((B, H, d_v), dtype=out_dtype, device=o_latent.device)
+    if workspace is None:
+        workspace = new_workspace(_abi.ic_decompress_gate_workspace_size(), o_latent.device)
+    _abi.ic_decompress_gate(_ptr(o_latent), _ptr(wv_b), _ptr(gate), B, H, d_v,
+                            _abi.IC_F32 if out.dtype == torch.float32 else _abi.IC_BF16, _ptr(out), _ptr(workspace),
+                            workspace.numel(), _stream_ptr(stream))
+    return out
+
 def cache_append(k_raw: torch.Tensor, ln_gamma: torch.Tensor, ln_beta: torch.Tensor, kv_raw: torch.Tensor,
                  pos: torch.Tensor, key_cache: torch.Tensor, kv_cache: torch.Tensor,
                  key_scale: Optional[torch.Tensor] = None, ln_eps: float = 1e-6, rope_base: float = 10000.0,

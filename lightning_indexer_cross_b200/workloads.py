@@ -342,3 +342,15 @@ def append_case(T, N, d_I, per_token=False, fp8=False, B=0, H=128, seed=14, devi
             q_pos[i] = v
     return dict(k_raw=k_raw, gamma=gamma, beta=beta, kv_raw=kv_raw, pos=pos, key_cache=key_cache,
                 kv_cache=kv_cache, key_scale=key_scale, q=q, q_pos=q_pos)
+
+
+def gate_case(B, H, d_v=128, gate=True, seed=15, device="cpu"):
+    """Inputs of the decompressed-space gate: ungated latent attention
+    outputs [B, H, 512] bf16 ~ N(0, 1), per-head up-projections
+    [H, d_v, 512] bf16 ~ N(0, 1)/sqrt(512) (synthetic weights), gate logits
+    [B, H, d_v] bf16 ~ N(0, 1) or None."""
+    g = _gen(seed, device)
+    o = _randn((B, H, D_LATENT), g, device).to(torch.bfloat16)
+    w = _randn((H, d_v, D_LATENT), g, device, 1.0 / math.sqrt(D_LATENT)).to(torch.bfloat16)
+    gl = _randn((B, H, d_v), g, device).to(torch.bfloat16) if gate else None
+    return o, w, gl

@@ -122,6 +122,24 @@ def test_cache_append_rejects_bad_arguments(abi):
     assert abi.ic_cache_append_workspace_size() >= 4
 
 
+def test_decompress_gate_rejects_bad_arguments(abi):
+    # every case below must fail validation: the pointers are host memory
+    p, keep = _fake()
+    call = lambda **kw: abi._gate(*[kw.get(n, d) for n, d in [
+        ("o", p), ("w", p), ("g", None), ("B", 4), ("H", 8), ("dv", 128), ("od", abi.IC_BF16), ("out", p),
+        ("ws", p), ("wsb", 256), ("st", None)]])
+    assert call(o=None) == abi.IC_ERR_INVALID_ARG
+    assert call(out=None) == abi.IC_ERR_INVALID_ARG
+    assert call(B=0) == abi.IC_ERR_INVALID_ARG
+    assert call(H=0) == abi.IC_ERR_INVALID_ARG
+    assert call(dv=64) == abi.IC_ERR_UNSUPPORTED
+    assert call(od=abi.IC_FP8_E4M3) == abi.IC_ERR_UNSUPPORTED
+    assert call(w=ctypes.c_void_p(p.value + 2)) == abi.IC_ERR_INVALID_ARG  # misaligned
+    assert call(g=ctypes.c_void_p(p.value + 8)) == abi.IC_ERR_INVALID_ARG
+    assert call(wsb=8) == abi.IC_ERR_INVALID_ARG
+    assert abi.ic_decompress_gate_workspace_size() >= 4
+
+
 @pytest.mark.parametrize("sched", [b"SFFF", b"FXSS", b"FS", b"FSSSS", b"", b"fsss"])
 def test_stack_rejects_bad_schedules(abi, sched):
     p, keep = _fake()
