@@ -111,7 +111,6 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
 
   ic::IndexerArgs a{};
-  a.q = static_cast<const __nv_bfloat16*>(q);
   a.w = w;
   a.k_scale = k_scale;
   a.scale_batch_stride = per_query ? scale_batch_stride : 0;

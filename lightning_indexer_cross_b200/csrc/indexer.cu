@@ -22,7 +22,8 @@
 //               shared-memory stages (128-byte swizzle, K-major).
 //   warp 1      TMEM owner and MMA issuer (one elected lane).
 //   warps 2..    epilogue: TMEM -> registers -> score row; also stage the
-//               query groups' Q (swizzled, zero-padded heads) and weights.
+//               query groups' head weights, and one of their threads issues
+//               the TMA loads of the groups' Q (swizzled, zero-padded heads).
 //               bf16 keys: warps 2..9, two per TMEM lane quadrant, each
 //               reducing one half of the columns; e4m3 keys: warps 2..5.
 //   warps 6..9  (e4m3 keys only) convert e4m3 tiles to bf16 in shared memory.

@@ -71,7 +71,7 @@ inline cudaError_t launch_kernel_cluster(void (*kern)(KArgs...), dim3 grid, dim3
 }
 
 struct IndexerArgs {
-  const __nv_bfloat16* q;      // [B, H_I, d_I]
+  // q [B, H_I, d_I] is read through its tensor map
   const float* w;              // [B, H_I]
   const float* k_scale;        // e4m3 keys: per-token scale
   int64_t scale_batch_stride;  // elements between queries' scales
