@@ -288,6 +288,23 @@ ic_status_t ic_last_device_status(void* workspace, ic_stream_t stream);
  * (for launch accounting in benchmarks). */
 int ic_last_launch_count(void);
 
+/* ---------------------------------------------------------------------------
+ * ic_set_wait_limit_ns / ic_wait_limit_ns -- bound of the waits inside the
+ * kernels (no counterpart in the pages; part of the failure handling).
+ *
+ * Every wait a kernel makes on a copy, an MMA or another warp of its CTA
+ * gives up after this many nanoseconds: the kernel then records
+ * IC_ERR_TIMEOUT in the status word, writes no further output, lets its own
+ * copies and MMAs in flight finish (each of those waits bounded by 2 s) and
+ * frees its tensor memory before returning, so the context stays usable.
+ * The default is 2 s. The value is process-wide and read when a call
+ * enqueues its kernels (calls already enqueued keep theirs). 0 makes every
+ * wait that is not already satisfied when first tested give up at once:
+ * meant for tests of the failure path; outputs of such calls are undefined.
+ * ------------------------------------------------------------------------- */
+void ic_set_wait_limit_ns(uint64_t ns);
+uint64_t ic_wait_limit_ns(void);
+
 #ifdef __cplusplus
 }
 #endif

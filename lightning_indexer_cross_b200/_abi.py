@@ -41,6 +41,8 @@ EXPORTED = [
     "ic_decompress_gate_workspace_size",
     "ic_last_device_status",
     "ic_last_launch_count",
+    "ic_set_wait_limit_ns",
+    "ic_wait_limit_ns",
 ]
 
 
@@ -107,6 +109,8 @@ _gate = _sig("ic_decompress_gate", _i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz,
 _gate_ws = _sig("ic_decompress_gate_workspace_size", _sz, [])
 _last_status = _sig("ic_last_device_status", _i, [_p, _p])
 _last_launches = _sig("ic_last_launch_count", _i, [])
+_set_wait = _sig("ic_set_wait_limit_ns", None, [ctypes.c_uint64])
+_get_wait = _sig("ic_wait_limit_ns", ctypes.c_uint64, [])
 
 
 def ic_status_string(code: int) -> str:
@@ -190,6 +194,16 @@ def ic_last_device_status(workspace, stream) -> int:
 
 def ic_last_launch_count() -> int:
     return int(_last_launches())
+
+
+def ic_set_wait_limit_ns(ns: int) -> None:
+    """Bound (ns) of every wait inside kernels enqueued from now on; 0 gives up
+    any wait not already satisfied (failure-path tests)."""
+    _set_wait(int(ns))
+
+
+def ic_wait_limit_ns() -> int:
+    return int(_get_wait())
 
 
 def raw_function(name: str):

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -17,6 +18,9 @@
 namespace {
 
 thread_local int g_launches = 0;
+
+// Bound of the waits inside the kernels (ic_set_wait_limit_ns).
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
 
 constexpr size_t kStatusBytes = 256;  // status word + padding (keeps regions aligned)
 
@@ -127,6 +131,7 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   a.pair = (!fp8 && !per_query && groups >= 2) ? 2 : 1;
   a.total_items = ceil_div<int64_t>(groups, a.pair) * a.tiles;
   a.per_query = per_query ? 1 : 0;
+  a.wait_ns = ic::wait_limit_ns();
   const int grid = static_cast<int>(std::min<int64_t>(num_sms(), a.total_items));
   cudaError_t e = ic::launch_indexer(map, qmap, a, HP, d_I, fp8, grid, stream, pdl);
   if (e != cudaSuccess) return IC_ERR_CUDA;
@@ -137,6 +142,8 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
 }  // namespace
 
 namespace ic {
+
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ top-k
 TopkLayout topk_layout(int B, int64_t N) {
@@ -309,6 +316,7 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
   a.out_f32 = out_dtype == IC_F32 ? 1 : 0;
   a.lse = lse;
   a.status = status;
+  a.wait_ns = ic::wait_limit_ns();
   int launches = 0;
   cudaError_t e = ic::launch_sparse_mla(qmap, omap, a, stream, pdl, &launches);
   if (e != cudaSuccess) return IC_ERR_CUDA;
@@ -351,6 +359,10 @@ const char* ic_status_string(ic_status_t s) {
 }
 
 int ic_last_launch_count(void) { return g_launches; }
+
+void ic_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns, std::memory_order_relaxed); }
+
+uint64_t ic_wait_limit_ns(void) { return g_wait_ns.load(std::memory_order_relaxed); }
 
 size_t ic_indexer_workspace_size(void) { return kStatusBytes; }
 
@@ -573,6 +585,7 @@ ic_status_t ic_decompress_gate(const void* o_latent, const void* wv_b, const voi
   a.B = B;
   a.H = H;
   a.status = static_cast<int*>(workspace);
+  a.wait_ns = ic::wait_limit_ns();
   if (ic::launch_gate(wmap, omap, a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;
   g_launches = 1;
   return IC_OK;

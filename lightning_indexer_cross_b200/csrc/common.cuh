@@ -35,9 +35,10 @@ IC_DEV uint64_t globaltimer_ns() {
   return t;
 }
 
-// Every wait inside a kernel gives up after this long, records
-// IC_ERR_TIMEOUT and lets the kernel wind down instead of spinning forever.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+// Bound of the waits a kernel makes while winding down after an abort (its
+// own copies and MMAs landing). The ordinary waits take their bound from the
+// kernel's arguments (ic_set_wait_limit_ns, 2 s by default).
+constexpr uint64_t kDrainLimitNs = 2000000000ull;  // 2 s
 
 IC_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -119,18 +120,41 @@ IC_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same condition.
+IC_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+IC_DEV void give_up(volatile int* abort_flag, int* status) {
+  *abort_flag = 1;
+  record_status(status, IC_ERR_TIMEOUT);
+}
+
 // Wait until the phase with the given parity has completed. Returns false if
-// the CTA-wide abort flag is raised or the wait limit passes (then the abort
-// flag is raised and IC_ERR_TIMEOUT recorded).
-IC_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status) {
+// the CTA-wide abort flag is raised or limit_ns passes (then the abort flag
+// is raised and IC_ERR_TIMEOUT recorded). limit_ns = 0: a phase that has not
+// completed at the first, non-blocking test is given up at once.
+IC_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status, uint64_t limit_ns) {
+  if (limit_ns == 0) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (!*abort_flag) give_up(abort_flag, status);
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
-      record_status(status, IC_ERR_TIMEOUT);
+    if (globaltimer_ns() - t0 > limit_ns) {
+      give_up(abort_flag, status);
       return false;
     }
   }
@@ -140,7 +164,7 @@ IC_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, 
 IC_DEV void mbar_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+    if (globaltimer_ns() - t0 > kDrainLimitNs) return;
   }
 }
 

@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (; s < kSlices; ++s) {
         const int st = s % kStages;
         const uint32_t ph = static_cast<uint32_t>((s / kStages) & 1);
-        if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status)) break;
+        if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
         mbar_arrive_expect_tx(&full[st], kStageBytes);
         uint8_t* base = stages + st * kStageBytes;
         tma_load_3d(base, &wmap, &full[st], s * 64, 0, h);                // W_h rows, dims [64 s, 64 s + 64)
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(kDv, n_mma, false, false);
       for (int s = 0; s < kSlices; ++s) {
         const int st = s % kStages;
-        if (!mbar_wait(&full[st], static_cast<uint32_t>((s / kStages) & 1), abort_flag, a.status)) break;
+        if (!mbar_wait(&full[st], static_cast<uint32_t>((s / kStages) & 1), abort_flag, a.status, a.wait_ns)) break;
         tc_fence_after();
         const uint32_t wa = smem_u32(stages + st * kStageBytes);
         const uint32_t ob = wa + kSliceBytes;
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
     const int d = quad * 32 + lane;
-    bool got = mbar_wait(acc_full, 0u, abort_flag, a.status);
+    bool got = mbar_wait(acc_full, 0u, abort_flag, a.status, a.wait_ns);
     __syncwarp();  // tcgen05.ld below is warp-collective
     got = got && !*abort_flag;
     got = __all_sync(0xffffffffu, got);
@@ -148,6 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    // every MMA issued has completed before its accumulator is freed (the
+    // issuer commits acc_full on every path, including after an abort)
+    if (lane == 0) mbar_drain(acc_full, 0u);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, kTileQ);

@@ -74,7 +74,7 @@ struct IdxCfg {
   static constexpr int kOffW = kOffQ + kQBytes;
   static constexpr int kOffNv = kOffW + kQSlots * kMaxCols * 4;
   static constexpr int kOffBar = kOffNv + kQSlots * 16 * 8;
-  static constexpr int kNumBars = 2 * kStages + 2 * kRawStages + 4 + 1;
+  static constexpr int kNumBars = 2 * kStages + 2 * kRawStages + 4 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(!(FP8 && PAIR), "e4m3 keys take one group per tile");
@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   uint64_t* acc_full = raw_empty + C::kRawStages; // [2]
   uint64_t* acc_empty = acc_full + 2;             // [2]
   uint64_t* q_ready = acc_empty + 2;              // [1]
+  uint64_t* mma_done = q_ready + 1;               // [1] every MMA issued has completed
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       mbar_init(&acc_empty[i], C::kEpiThreads);
     }
     mbar_init(q_ready, 1);
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -159,7 +161,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         if constexpr (!FP8) {
           const int st = static_cast<int>(it % C::kStages);
           const uint32_t ph = static_cast<uint32_t>((it / C::kStages) & 1);
-          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status)) break;
+          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
           mbar_arrive_expect_tx(&full[st], C::kTileBytes);
 #pragma unroll
           for (int bk = 0; bk < C::kBlocks; ++bk)
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         } else {
           const int st = static_cast<int>(it % C::kRawStages);
           const uint32_t ph = static_cast<uint32_t>((it / C::kRawStages) & 1);
-          if (!mbar_wait(&raw_empty[st], ph ^ 1, abort_flag, a.status)) break;
+          if (!mbar_wait(&raw_empty[st], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
           mbar_arrive_expect_tx(&raw_full[st], C::kRawBytes);
           tma_load_3d(raw + st * C::kRawBytes, &kmap, &raw_full[st], 0, t * kTileKeys, z);
         }
@@ -195,18 +197,18 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         const int grp = static_cast<int>(wi / a.tiles) * P;
         const int ng = P == 1 ? 1 : (a.groups - grp < P ? a.groups - grp : P);
         if (grp != cur_grp) {
-          if (!mbar_wait(q_ready, q_phase, abort_flag, a.status)) break;
+          if (!mbar_wait(q_ready, q_phase, abort_flag, a.status, a.wait_ns)) break;
           q_phase ^= 1;
           cur_grp = grp;
         }
         const int st = static_cast<int>(it % C::kStages);
         const uint32_t ph = static_cast<uint32_t>((it / C::kStages) & 1);
-        if (!mbar_wait(&full[st], ph, abort_flag, a.status)) break;
+        if (!mbar_wait(&full[st], ph, abort_flag, a.status, a.wait_ns)) break;
         const uint32_t a_addr = smem_u32(stages + st * C::kTileBytes);
         for (int sub = 0; sub < ng; ++sub, ++si) {
           const int acc = static_cast<int>(si & 1);
           const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
-          if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + acc * 256;
           const uint32_t qb = q_addr + sub * C::kQSlotBytes;
@@ -223,8 +225,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         mma_commit(&empty[st]);
       }
       // make sure nothing issued is still running before TMEM is released
-      mma_commit(q_ready);
-      mbar_drain(q_ready, q_phase);
+      mma_commit(mma_done);
+      mbar_drain(mma_done, 0u);
     }
   } else if (warp < kEpiWarp0 + C::kEpiWarps) {
     // ------------------------------------------------------------ epilogue
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       for (int sub = 0; sub < ng; ++sub, ++si) {
       const int acc = static_cast<int>(si & 1);
       const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
-      got = mbar_wait(&acc_full[acc], aph, abort_flag, a.status);
+      got = mbar_wait(&acc_full[acc], aph, abort_flag, a.status, a.wait_ns);
       __syncwarp();  // tcgen05.ld below is warp-collective
       if (!got) break;
       tc_fence_after();
@@ -438,8 +440,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       const uint32_t rph = static_cast<uint32_t>((it / C::kRawStages) & 1);
       const int bs = static_cast<int>(it % C::kStages);
       const uint32_t bph = static_cast<uint32_t>((it / C::kStages) & 1);
-      if (!mbar_wait(&raw_full[rs], rph, abort_flag, a.status)) break;
-      if (!mbar_wait(&empty[bs], bph ^ 1, abort_flag, a.status)) break;
+      if (!mbar_wait(&raw_full[rs], rph, abort_flag, a.status, a.wait_ns)) break;
+      if (!mbar_wait(&empty[bs], bph ^ 1, abort_flag, a.status, a.wait_ns)) break;
       const uint8_t* src = raw + rs * C::kRawBytes;
       uint8_t* dst = stages + bs * C::kTileBytes;
       constexpr int kChunks16 = D_I / 16;  // 16-element e4m3 chunks per row

@@ -14,6 +14,10 @@
 
 namespace ic {
 
+// Bound, in nanoseconds, of every wait inside the kernels enqueued from now
+// on (set with ic_set_wait_limit_ns).
+uint64_t wait_limit_ns();
+
 // Raise a kernel's dynamic shared-memory limit once per device (never again
 // afterwards, so later calls are safe inside CUDA-graph capture). `done` is
 // the caller's per-kernel flag array: kernels of one signature share a
@@ -86,6 +90,7 @@ struct IndexerArgs {
   int pair;           // groups per work item: 2 (one cache shared by all queries, >= 2 groups) or 1
   int64_t total_items;  // ceil(groups / pair) * tiles
   int per_query;      // 1: key cache z-coordinate = group (G == 1)
+  uint64_t wait_ns;   // bound of every wait (0: give up unless already complete)
 };
 
 int indexer_smem_bytes(int d_I, bool fp8);
@@ -153,6 +158,7 @@ struct MlaArgs {
   int out_f32;
   float* lse;                // [B, H] or null
   int* status;
+  uint64_t wait_ns;          // bound of every wait (0: give up unless already complete)
 };
 int mla_smem_bytes(int ts);
 // qmap: 2-D tensor map over q viewed as [B*H rows, 576] bf16, box 64 x 128,
@@ -193,6 +199,7 @@ struct GateArgs {
   int out_f32;
   int B, H;
   int* status;
+  uint64_t wait_ns;           // bound of every wait (0: give up unless already complete)
 };
 int gate_smem_bytes();
 // wmap: 3-D tensor map over wv_b (512, 128, H), box 64 x 128 x 1; omap: 3-D

@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       int32_t* ids = idx_s + (i & 1) * TS;
       uint32_t* vm = vmask + (i & 1) * (TS / 32);
       // the softmax of unit i - 2 is done with this buffer's validity bits
-      if (i >= 2 && !mbar_wait(&idx_free[i & 1], static_cast<uint32_t>(((i >> 1) - 1) & 1), abort_flag, a.status)) {
+      if (i >= 2 && !mbar_wait(&idx_free[i & 1], static_cast<uint32_t>(((i >> 1) - 1) & 1), abort_flag, a.status, a.wait_ns)) {
         ok = false;
         break;
       }
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       }
       mbar_arrive(&idx_ready[i & 1]);
       if (u + a.ctas < a.units) load_rows(u + a.ctas, nxt);
-      if (!mbar_wait(&idx_ready[i & 1], static_cast<uint32_t>((i >> 1) & 1), abort_flag, a.status)) {
+      if (!mbar_wait(&idx_ready[i & 1], static_cast<uint32_t>((i >> 1) & 1), abort_flag, a.status, a.wait_ns)) {
         ok = false;
         break;
       }
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       const __nv_bfloat16* kvb = a.kv + static_cast<int64_t>(w.b) * a.kv_batch_stride;
       for (int s = 0; s < C::kNumSt; ++s, ++g) {
         const int st = g % kStages;
-        if (!mbar_wait(&empty[st], static_cast<uint32_t>((g / kStages) & 1) ^ 1u, abort_flag, a.status)) {
+        if (!mbar_wait(&empty[st], static_cast<uint32_t>((g / kStages) & 1) ^ 1u, abort_flag, a.status, a.wait_ns)) {
           ok = false;
           break;
         }
@@ -328,14 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         // [0, 256) in half B; the next unit's A is this unit's B, read out
         // first, while this unit's second output half is still being formed
         const uint32_t col_a = (i & 1) ? 256u : 0u, col_b = 256u - col_a;
-        if (i > 0 && !mbar_wait(o1_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status)) {
+        if (i > 0 && !mbar_wait(o1_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status, a.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int s = 0; s < kQKChunks; ++s, ++g) {
           const int st = g % kStages;
-          if (!mbar_wait(&full[st], (g / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait(&full[st], (g / kStages) & 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
           fence_proxy_async_smem();
           tc_fence_after();
           const uint32_t base = smem_u32(stages + st * C::kStageBytes);
@@ -347,16 +347,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
         }
         if (!ok) break;
         mma_commit(s_full);
-        if (!mbar_wait(p_ready, static_cast<uint32_t>(i & 1), abort_flag, a.status)) { ok = false; break; }
+        if (!mbar_wait(p_ready, static_cast<uint32_t>(i & 1), abort_flag, a.status, a.wait_ns)) { ok = false; break; }
         // half B held the previous unit's second output half
-        if (i > 0 && !mbar_wait(o2_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status)) {
+        if (i > 0 && !mbar_wait(o2_free, static_cast<uint32_t>((i - 1) & 1), abort_flag, a.status, a.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int s = kQKChunks; s < C::kNumSt; ++s, ++g) {
           const int st = g % kStages;
-          if (!mbar_wait(&full[st], (g / kStages) & 1, abort_flag, a.status)) { ok = false; break; }
+          if (!mbar_wait(&full[st], (g / kStages) & 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
           fence_proxy_async_smem();
           tc_fence_after();
           const int p = s - kQKChunks;
@@ -390,8 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       const uint32_t col_a = (i & 1) ? 256u : 0u, col_b = 256u - col_a;
       const uint32_t taddr = tlane + col_a;  // S (and later output dims [256, 512))
       const uint32_t* vm = vmask + (i & 1) * (TS / 32);
-      ok = mbar_wait(&idx_ready[i & 1], static_cast<uint32_t>((i >> 1) & 1), abort_flag, a.status) &&
-           mbar_wait(s_full, static_cast<uint32_t>(i & 1), abort_flag, a.status);
+      ok = mbar_wait(&idx_ready[i & 1], static_cast<uint32_t>((i >> 1) & 1), abort_flag, a.status, a.wait_ns) &&
+           mbar_wait(s_full, static_cast<uint32_t>(i & 1), abort_flag, a.status, a.wait_ns);
       __syncwarp();  // tcgen05.ld is warp-collective
       if (!ok) break;
       tc_fence_after();
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_mla_kernel(const __grid_co
       int nt = 0;  // tiles of the P buffer issued by this warp in this unit
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
-        ok = mbar_wait(half == 0 ? o1_full : o2_full, static_cast<uint32_t>(i & 1), abort_flag, a.status);
+        ok = mbar_wait(half == 0 ? o1_full : o2_full, static_cast<uint32_t>(i & 1), abort_flag, a.status, a.wait_ns);
         __syncwarp();
         if (!ok) break;
         tc_fence_after();
@@ -800,7 +800,7 @@ __global__ void __launch_bounds__(kCombThreads) mla_combine_bulk_kernel(const Ml
   const float sink2 = active ? __ldg(&a.sink[gw % a.H]) * kLog2e : 0.f;
   __syncthreads();  // (m, l) in shared memory
   // this row's partials
-  const bool ok = active && mbar_wait(&bars[r / kCombRowsPerBar], 0u, abort_flag, a.status);
+  const bool ok = active && mbar_wait(&bars[r / kCombRowsPerBar], 0u, abort_flag, a.status, a.wait_ns);
   if (ok) combine_staged_row<F32>(a, pbuf + static_cast<size_t>(r) * row_bytes, mlb + r * S, gw, sink2, q, graw);
   // every copy has landed (or its wait gave up) before the CTA exits
   if (t == 0)

@@ -34,6 +34,23 @@ def _need_cuda(*ts):
             raise ValueError("lightning_indexer_cross_b200 ops need CUDA tensors (no CPU path exists)")
 
 
+def _need_dense(*ts):
+    """Tensors handed to the library as raw pointers are read with dense
+    row-major strides."""
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("lightning_indexer_cross_b200 ops need contiguous tensors")
+
+
+def _need_dense_rows(*ts):
+    """Caches may sit apart by a batch stride (dim 0) but are dense within."""
+    for t in ts:
+        if t is None:
+            continue
+        if not t[0].is_contiguous() or (t.shape[0] > 1 and t.stride(0) < t[0].numel()):
+            raise ValueError("lightning_indexer_cross_b200 ops need caches dense within each batch entry")
+
+
 def new_workspace(nbytes: int, device) -> torch.Tensor:
     """Zeroed byte workspace (the status word must start at IC_OK)."""
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
@@ -43,15 +60,19 @@ def indexer_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: Op
                   n_valid: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """scores[b,s] = sum_h w[b,h] ReLU(q[b,h] . k[s]). k: [Bk,N,d_I] bf16 or uint8 (e4m3 codes)."""
-    _need_cuda(q, w, k, k_scale, n_valid)
+    _need_cuda(q, w, k, k_scale, n_valid, scores)
+    _need_dense(q, w, n_valid, scores)
+    _need_dense_rows(k, k_scale)
     B, H_I, d_I = q.shape
     Bk, N, dk = k.shape
     assert dk == d_I and Bk in (1, B)
     fp8 = k.dtype == torch.uint8
     assert q.dtype == torch.bfloat16 and w.dtype == torch.float32
     assert k.dtype in (torch.bfloat16, torch.uint8)
+    assert k_scale is None or (fp8 and k_scale.dtype == torch.float32 and k_scale.shape == (Bk, N))
     if scores is None:
         scores = torch.empty((B, N), dtype=torch.float32, device=q.device)
+    assert scores.shape == (B, N) and scores.dtype == torch.float32
     if workspace is None:
         workspace = new_workspace(_abi.ic_indexer_workspace_size(), q.device)
     kbs = k.stride(0) if Bk > 1 else 0
@@ -64,10 +85,13 @@ def indexer_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: Op
 
 def topk(scores: torch.Tensor, k: int, n_valid: Optional[torch.Tensor] = None,
          idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    _need_cuda(scores, n_valid)
+    _need_cuda(scores, n_valid, idx)
+    _need_dense(scores, n_valid, idx)
     B, N = scores.shape
+    assert scores.dtype == torch.float32
     if idx is None:
         idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    assert idx.shape == (B, k) and idx.dtype == torch.int32
     if workspace is None:
         workspace = new_workspace(_abi.ic_topk_workspace_size(B, N, k), scores.device)
     _abi.ic_topk(_ptr(scores), B, N, _ptr(n_valid), k, _ptr(idx), _ptr(workspace), workspace.numel(),
@@ -80,17 +104,25 @@ def sparse_mla_decode(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, sink
                       out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
                       lse: Optional[torch.Tensor] = None, want_lse: bool = True,
                       workspace: Optional[torch.Tensor] = None, stream=None):
-    _need_cuda(q, kv, idx, sink, gate)
+    _need_cuda(q, kv, idx, sink, gate, out, lse)
+    _need_dense(q, idx, sink, gate, out, lse)
+    _need_dense_rows(kv)
     B, H, D = q.shape
     Bkv, N, Dk = kv.shape
     assert D == D_QK and Dk == D_QK and Bkv in (1, B)
+    assert q.dtype == torch.bfloat16 and kv.dtype == torch.bfloat16 and idx.dtype == torch.int32
+    assert sink.shape == (H,) and sink.dtype == torch.float32
+    assert gate is None or (gate.shape == (B, H, D_V) and gate.dtype == torch.bfloat16)
     k = idx.shape[1]
+    assert idx.shape == (B, k)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(D_QK)
     if out is None:
         out = torch.empty((B, H, D_V), dtype=out_dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    assert out.shape == (B, H, D_V) and out.dtype in (torch.bfloat16, torch.float32)
+    assert lse is None or (lse.shape == (B, H) and lse.dtype == torch.float32)
     if workspace is None:
         workspace = new_workspace(_abi.ic_sparse_mla_workspace_size(B, H, k), q.device)
     od = _abi.IC_F32 if out.dtype == torch.float32 else _abi.IC_BF16
@@ -107,6 +139,7 @@ def decompress_gate(o_latent: torch.Tensor, wv_b: torch.Tensor, gate: Optional[t
     """out[b,h] = sigmoid(gate[b,h]) * (wv_b[h] @ o_latent[b,h]): o_latent [B,H,512] bf16 (ungated attention
     output), wv_b [H,128,512] bf16, gate [B,H,128] bf16 or None."""
     _need_cuda(o_latent, wv_b, gate, out)
+    _need_dense(o_latent, wv_b, gate, out)
     B, H, K = o_latent.shape
     Hw, d_v, Kw = wv_b.shape
     assert K == D_V and Kw == D_V and Hw == H
@@ -114,12 +147,14 @@ def decompress_gate(o_latent: torch.Tensor, wv_b: torch.Tensor, gate: Optional[t
     assert gate is None or (gate.shape == (B, H, d_v) and gate.dtype == torch.bfloat16)
     if out is None:
         out = torch.empty((B, H, d_v), dtype=out_dtype, device=o_latent.device)
+    assert out.shape == (B, H, d_v) and out.dtype in (torch.bfloat16, torch.float32)
     if workspace is None:
         workspace = new_workspace(_abi.ic_decompress_gate_workspace_size(), o_latent.device)
     _abi.ic_decompress_gate(_ptr(o_latent), _ptr(wv_b), _ptr(gate), B, H, d_v,
                             _abi.IC_F32 if out.dtype == torch.float32 else _abi.IC_BF16, _ptr(out), _ptr(workspace),
                             workspace.numel(), _stream_ptr(stream))
     return out
+
 
 def cache_append(k_raw: torch.Tensor, ln_gamma: torch.Tensor, ln_beta: torch.Tensor, kv_raw: torch.Tensor,
                  pos: torch.Tensor, key_cache: torch.Tensor, kv_cache: torch.Tensor,
@@ -132,6 +167,8 @@ def cache_append(k_raw: torch.Tensor, ln_gamma: torch.Tensor, ln_beta: torch.Ten
     rotated in place to q_pos[b]. Caches are [C, N, ...] with C == 1 (one shared cache) or C == T (token t
     writes cache t). Returns the workspace (its status word records out-of-range rows)."""
     _need_cuda(k_raw, ln_gamma, ln_beta, kv_raw, pos, key_cache, kv_cache, key_scale, q, q_pos)
+    _need_dense(k_raw, ln_gamma, ln_beta, kv_raw, pos, q, q_pos)
+    _need_dense_rows(key_cache, kv_cache, key_scale)
     T, d_I = k_raw.shape
     C, N, dk = key_cache.shape
     assert k_raw.dtype == torch.bfloat16 and kv_raw.dtype == torch.bfloat16 and kv_cache.dtype == torch.bfloat16

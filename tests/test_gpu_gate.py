@@ -8,8 +8,7 @@ import torch
 from oracle import gate_oracle as G
 from lightning_indexer_cross_b200 import workloads as W
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skip(reason="ic_decompress_gate has not yet run on a GPU; enabled once it has")]
+pytestmark = pytest.mark.gpu
 
 # bf16 inputs, fp32 accumulation over 512 products: far below 1e-4 of the
 # row's largest value; a bf16 output adds its rounding (2^-9)
