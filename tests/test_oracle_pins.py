@@ -156,28 +156,52 @@ def test_topk_neg_inf_ranked_last():
 
 
 # ---------------------------------------------------------------- planted tokens
+def _planted_z(s_row, planted):
+    """z-scores of the planted positions against the unplanted scores."""
+    mask = np.ones(s_row.shape[0], bool)
+    mask[planted] = False
+    return (s_row[planted] - s_row[mask].mean()) / s_row[mask].std()
+
+
 def test_planted_tokens_recovered_tiny_workload():
+    """Tiny recipe: planted keys "aligned to q, score +4 sigma". The oracle's
+    scores put every planted token at 3.9..4.1 standard deviations above the
+    mean of the 4088 unplanted ones, and top-256 keeps all 8."""
     wl = W.tiny("cpu")
     lay = wl.layers[0]
     s = O.indexer_scores(lay.q_idx, lay.w, lay.k_idx)
     planted = wl.planted[0].numpy()
-    mask = np.ones(wl.N, bool)
-    mask[planted] = False
-    mu, sd = s[0, mask].mean(), s[0, mask].std()
-    assert np.all(s[0, planted] >= mu + 4 * sd)
+    z = _planted_z(s[0], planted)
+    assert np.all((z >= 3.9) & (z <= 4.1)), z
     top = set(O.topk_indices(s, wl.topk)[0])
     assert set(planted) <= top
 
 
-def test_planted_tokens_recovered_long_context_shape_small():
-    # the long-context recipe at a reduced N, both key variants
+def test_planted_tokens_long_context_recipe_small():
+    """The long-context recipe at a reduced N, bf16 and e4m3 keys: planted
+    z-scores in [3.9, 4.1] (for e4m3 on the stored, quantised keys) and
+    every planted token recovered."""
     for fp8 in (False, True):
-        wl = W.long_context("cpu", N=8192, B=2, H=8, fp8=fp8, n_planted=16)
+        wl = W.long_context("cpu", N=32768, B=2, H=8, fp8=fp8, n_planted=16)
         lay = wl.layers[0]
         s = O.indexer_scores(lay.q_idx, lay.w, lay.k_idx, lay.k_scale, keys_are_e4m3=fp8)
         for b in range(wl.B):
+            z = _planted_z(s[b], wl.planted[b].numpy())
+            assert np.all((z >= 3.9) & (z <= 4.1)), (fp8, b, z)
             top = set(O.topk_indices(s[b:b + 1], wl.topk)[0])
             assert set(wl.planted[b].numpy()) <= top
+
+
+def test_planting_moments_match_the_oracle_scores_of_random_keys():
+    """The closed-form mean and standard deviation used to place planted keys
+    agree with the oracle's scores of 65536 keys drawn from the recipe's
+    distribution (no planted keys), within sampling error."""
+    q, w, k, _, _ = W.indexer_case(3, 65536, 64, 128, seed=77)
+    s = O.indexer_scores(q, w, k)
+    mu, sd = W.unplanted_score_moments(q, w, 1.0 / np.sqrt(128))
+    for b in range(3):
+        assert abs(s[b].mean() - float(mu[b])) <= 0.02 * float(sd[b])
+        assert abs(s[b].std() / float(sd[b]) - 1.0) <= 0.02
 
 
 # ---------------------------------------------------------------- sparse MLA
