@@ -141,7 +141,9 @@ ic_status_t ic_topk_noalloc(const float* scores, int B, int64_t N, const int64_t
  *   q     [B, H, 576] bf16 (RoPE already applied to dims 512..575).
  *   kv    latent cache of query b at kv + b*kv_batch_stride elements,
  *         [N, 576] bf16; kv_batch_stride = 0: one cache shared by all.
- *   idx   [B, k] int32.   sink [H] fp32.   gate [B, H, 512] bf16 or NULL.
+ *   idx   [B, k] int32.   sink [H] fp32 (may be -inf: no sink term; a row
+ *         with no valid selected token then gets out = 0, lse = -inf).
+ *   gate  [B, H, 512] bf16 or NULL.
  *   out   [B, H, 512], bf16 (out_dtype IC_BF16) or fp32 (IC_F32).
  *   lse   [B, H] fp32 natural-log sum, or NULL.
  *   Supported: any H >= 1 (heads run in blocks of 128); k >= 1;
@@ -275,6 +277,63 @@ ic_status_t ic_decompress_gate(const void* o_latent, const void* wv_b, const voi
                                ic_dtype_t out_dtype, void* out, void* workspace, size_t ws_bytes,
                                ic_stream_t stream);
 size_t ic_decompress_gate_workspace_size(void);
+
+/* ---------------------------------------------------------------------------
+ * Context-parallel decode: the N cached tokens split over G ranks, rank r
+ * holding the contiguous shard [lo_r, hi_r) of the positions (Hy4 IndexCache
+ * explainer, TL;DR and Jargon "Sparse attention": the indexer scores the
+ * whole cached past, which is what grows with a 1M-token context). The
+ * exchanges between the ranks are collectives the caller issues (NCCL); the
+ * library provides the steps around them. Per F layer and rank:
+ *   1. ic_indexer_score and ic_topk over the shard (local positions);
+ *   2. ic_cp_candidates: (score, global position) of each local top-k entry;
+ *   3. all-gather of the candidates over the ranks -> [B, G*k];
+ *   4. ic_cp_merge_topk: the global top-k (every rank gets the same set: the
+ *      k best of a row are among the k best of their own shard), and the
+ *      row's positions inside this rank's shard;
+ * and per layer:
+ *   5. ic_sparse_mla_decode over the local positions with the sink -inf
+ *      (no sink term), gate NULL, fp32 output and lse;
+ *   6. all-gather of the partial outputs and lse over the ranks;
+ *   7. ic_cp_combine: out = sum_r e^{lse_r} o_r / (e^{sink} + sum_r e^{lse_r}),
+ *      then the gate -- the single-GPU result up to rounding.
+ *
+ * ic_cp_candidates
+ *   scores [B, N_local] fp32 (the shard's scores), idx [B, k] int32 (shard
+ *   positions or -1). Writes cand_score [B, k] (the score, -inf for -1) and
+ *   cand_idx [B, k] (offset + position, -1 for -1). A position outside
+ *   [-1, N_local) is treated as -1 and recorded as IC_ERR_BAD_INDEX in the
+ *   workspace's status word (>= ic_cp_workspace_size() bytes).
+ *
+ * ic_cp_merge_topk
+ *   Candidates of G segments (one per rank, as an all-gather lays them
+ *   out), segment g at cand_score + g*seg_stride and cand_idx +
+ *   g*seg_stride, each [B, kin]; G*kin <= 16384. Writes to idx_global
+ *   [B, k] the global positions of the k candidates with the highest
+ *   scores, ties toward the lower global position (the single-GPU tie rule),
+ *   -1 padding when a row has fewer than k candidates with a position; and,
+ *   if idx_local is not NULL, idx_local[b, j] = idx_global - lo when that
+ *   lies in [lo, hi), else -1. Order within a row is unspecified (the same
+ *   on every rank). G*kin > 16384: IC_ERR_UNSUPPORTED.
+ *
+ * ic_cp_combine
+ *   Rank r's normalised output [B, H, 512] fp32 at part_out + r*out_stride
+ *   and natural-log sum [B, H] fp32 at part_lse + r*lse_stride (-inf: no
+ *   row), from step 5; when G > 1, out_stride a multiple of 4 and
+ *   >= B*H*512, lse_stride >= B*H. sink [H], gate [B, H, 512] bf16 or NULL. Writes out [B, H, 512]
+ *   (bf16 or fp32) and, if not NULL, lse [B, H] (log of the whole
+ *   denominator).
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_cp_candidates(const float* scores, const int32_t* idx, int B, int64_t N_local, int k,
+                             int64_t offset, float* cand_score, int32_t* cand_idx, void* workspace,
+                             size_t ws_bytes, ic_stream_t stream);
+size_t ic_cp_workspace_size(void);
+ic_status_t ic_cp_merge_topk(const float* cand_score, const int32_t* cand_idx, int64_t seg_stride, int G, int B,
+                             int kin, int k, int64_t lo, int64_t hi, int32_t* idx_global, int32_t* idx_local,
+                             ic_stream_t stream);
+ic_status_t ic_cp_combine(const float* part_out, int64_t out_stride, const float* part_lse, int64_t lse_stride, int G,
+                          int B, int H, const float* sink, const void* gate, ic_dtype_t out_dtype, void* out,
+                          float* lse, ic_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * ic_last_device_status -- synchronises `stream`, then reads and clears the

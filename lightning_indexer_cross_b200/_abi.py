@@ -43,6 +43,10 @@ EXPORTED = [
     "ic_last_launch_count",
     "ic_set_wait_limit_ns",
     "ic_wait_limit_ns",
+    "ic_cp_candidates",
+    "ic_cp_workspace_size",
+    "ic_cp_merge_topk",
+    "ic_cp_combine",
 ]
 
 
@@ -109,6 +113,10 @@ _gate = _sig("ic_decompress_gate", _i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _sz,
 _gate_ws = _sig("ic_decompress_gate_workspace_size", _sz, [])
 _last_status = _sig("ic_last_device_status", _i, [_p, _p])
 _last_launches = _sig("ic_last_launch_count", _i, [])
+_cp_cand = _sig("ic_cp_candidates", _i, [_p, _p, _i, _i64, _i, _i64, _p, _p, _p, _sz, _p])
+_cp_ws = _sig("ic_cp_workspace_size", _sz, [])
+_cp_merge = _sig("ic_cp_merge_topk", _i, [_p, _p, _i64, _i, _i, _i, _i, _i64, _i64, _p, _p, _p])
+_cp_combine = _sig("ic_cp_combine", _i, [_p, _i64, _p, _i64, _i, _i, _i, _p, _p, _i, _p, _p, _p])
 _set_wait = _sig("ic_set_wait_limit_ns", None, [ctypes.c_uint64])
 _get_wait = _sig("ic_wait_limit_ns", ctypes.c_uint64, [])
 
@@ -194,6 +202,29 @@ def ic_last_device_status(workspace, stream) -> int:
 
 def ic_last_launch_count() -> int:
     return int(_last_launches())
+
+
+def ic_cp_candidates(scores, idx, B, N_local, k, offset, cand_score, cand_idx, workspace, ws_bytes, stream) -> None:
+    _check(_cp_cand(scores, idx, B, N_local, k, offset, cand_score, cand_idx, workspace, ws_bytes, stream),
+           "ic_cp_candidates")
+
+
+def ic_cp_workspace_size() -> int:
+    return int(_cp_ws())
+
+
+def ic_cp_merge_topk(cand_score, cand_idx, seg_stride, G, B, kin, k, lo, hi, idx_global, idx_local, stream) -> None:
+    _check(_cp_merge(cand_score, cand_idx, seg_stride, G, B, kin, k, lo, hi, idx_global, idx_local, stream),
+           "ic_cp_merge_topk")
+
+
+def ic_cp_combine(part_out, out_stride, part_lse, lse_stride, G, B, H, sink, gate, out_dtype, out, lse,
+                  stream) -> None:
+    _check(_cp_combine(part_out, out_stride, part_lse, lse_stride, G, B, H, sink, gate, out_dtype, out, lse, stream),
+           "ic_cp_combine")
+
+
+IC_CP_MAX_CANDIDATES = 16384
 
 
 def ic_set_wait_limit_ns(ns: int) -> None:

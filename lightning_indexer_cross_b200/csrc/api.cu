@@ -591,6 +591,86 @@ ic_status_t ic_decompress_gate(const void* o_latent, const void* wv_b, const voi
   return IC_OK;
 }
 
+size_t ic_cp_workspace_size(void) { return kStatusBytes; }
+
+ic_status_t ic_cp_candidates(const float* scores, const int32_t* idx, int B, int64_t N_local, int k,
+                             int64_t offset, float* cand_score, int32_t* cand_idx, void* workspace, size_t ws_bytes,
+                             ic_stream_t stream) {
+  g_launches = 0;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
+  if (!scores || !idx || !cand_score || !cand_idx) return IC_ERR_INVALID_ARG;
+  if (B < 1 || k < 1 || N_local < 1 || offset < 0 || offset + N_local >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * k >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  ic::CpCandArgs a{};
+  a.scores = scores;
+  a.idx = idx;
+  a.B = B;
+  a.k = k;
+  a.N_local = N_local;
+  a.offset = offset;
+  a.cand_score = cand_score;
+  a.cand_idx = cand_idx;
+  a.status = static_cast<int*>(workspace);
+  if (ic::launch_cp_candidates(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;
+  g_launches = 1;
+  return IC_OK;
+}
+
+ic_status_t ic_cp_merge_topk(const float* cand_score, const int32_t* cand_idx, int64_t seg_stride, int G, int B,
+                             int kin, int k, int64_t lo, int64_t hi, int32_t* idx_global, int32_t* idx_local,
+                             ic_stream_t stream) {
+  g_launches = 0;
+  if (!cand_score || !cand_idx || !idx_global) return IC_ERR_INVALID_ARG;
+  if (G < 1 || B < 1 || kin < 1 || k < 1 || lo < 0 || hi < lo || hi >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  if (G > 1 && seg_stride < static_cast<int64_t>(B) * kin) return IC_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(G) * kin > ic::kCpMaxCand) return IC_ERR_UNSUPPORTED;
+  ic::CpMergeArgs a{};
+  a.cand_score = cand_score;
+  a.cand_idx = cand_idx;
+  a.seg_stride = seg_stride;
+  a.G = G;
+  a.B = B;
+  a.kin = kin;
+  a.k = k;
+  a.lo = lo;
+  a.hi = hi;
+  a.idx_global = idx_global;
+  a.idx_local = idx_local;
+  if (ic::launch_cp_merge_topk(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;
+  g_launches = 1;
+  return IC_OK;
+}
+
+ic_status_t ic_cp_combine(const float* part_out, int64_t out_stride, const float* part_lse, int64_t lse_stride, int G,
+                          int B, int H, const float* sink, const void* gate, ic_dtype_t out_dtype, void* out,
+                          float* lse, ic_stream_t stream) {
+  g_launches = 0;
+  if (!part_out || !part_lse || !sink || !out) return IC_ERR_INVALID_ARG;
+  if (G < 1 || B < 1 || H < 1) return IC_ERR_INVALID_ARG;
+  if (out_dtype != IC_BF16 && out_dtype != IC_F32) return IC_ERR_UNSUPPORTED;
+  if (!aligned16(part_out) || !aligned16(out) || (gate && !aligned16(gate))) return IC_ERR_INVALID_ARG;
+  const int64_t rows = static_cast<int64_t>(B) * H;
+  if (rows >= (int64_t(1) << 31)) return IC_ERR_INVALID_ARG;
+  // every segment holds one rank's [B, H, 512] output (16-byte aligned) and [B, H] lse
+  if (G > 1 && (out_stride < rows * 512 || out_stride % 4 != 0 || lse_stride < rows)) return IC_ERR_INVALID_ARG;
+  ic::CpCombineArgs a{};
+  a.part_out = part_out;
+  a.part_lse = part_lse;
+  a.out_stride = out_stride;
+  a.lse_stride = lse_stride;
+  a.G = G;
+  a.B = B;
+  a.H = H;
+  a.sink = sink;
+  a.gate = static_cast<const __nv_bfloat16*>(gate);
+  a.out = out;
+  a.out_f32 = out_dtype == IC_F32 ? 1 : 0;
+  a.lse = lse;
+  if (ic::launch_cp_combine(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;
+  g_launches = 1;
+  return IC_OK;
+}
+
 ic_status_t ic_last_device_status(void* workspace, ic_stream_t stream) {
   if (!workspace) return IC_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return IC_ERR_CUDA;

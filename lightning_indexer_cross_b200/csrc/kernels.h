@@ -207,4 +207,45 @@ int gate_smem_bytes();
 // 128-byte swizzle.
 cudaError_t launch_gate(const CUtensorMap& wmap, const CUtensorMap& omap, const GateArgs& a, cudaStream_t stream);
 
+// ---------------------------------------------------------------- context parallel
+// Candidates per row the merge holds in shared memory (G ranks x k).
+constexpr int kCpMaxCand = 16384;
+
+struct CpCandArgs {
+  const float* scores;   // [B, N_local] this rank's shard scores
+  const int32_t* idx;    // [B, k] local top-k (shard positions, -1 padding)
+  int B, k;
+  int64_t N_local;
+  int64_t offset;        // global position of the shard's first token
+  float* cand_score;     // [B, k]
+  int32_t* cand_idx;     // [B, k] global positions (-1 padding)
+  int* status;
+};
+cudaError_t launch_cp_candidates(const CpCandArgs& a, cudaStream_t stream);
+
+struct CpMergeArgs {
+  const float* cand_score;  // [G][B, kin] segments seg_stride elements apart
+  const int32_t* cand_idx;  // the same layout: global positions (-1 padding)
+  int64_t seg_stride;
+  int G, B, kin, k;
+  int64_t lo, hi;           // this rank's shard [lo, hi) of the global positions
+  int32_t* idx_global;      // [B, k]
+  int32_t* idx_local;       // [B, k] positions inside the shard, -1 elsewhere (or null)
+};
+cudaError_t launch_cp_merge_topk(const CpMergeArgs& a, cudaStream_t stream);
+
+struct CpCombineArgs {
+  const float* part_out;      // [G][B, H, 512] each rank's normalised partial output
+  const float* part_lse;      // [G][B, H] each rank's natural-log sum (-inf: no row)
+  int64_t out_stride;         // elements between ranks' outputs
+  int64_t lse_stride;         // elements between ranks' lse arrays
+  int G, B, H;
+  const float* sink;          // [H]
+  const __nv_bfloat16* gate;  // [B, H, 512] or null
+  void* out;                  // [B, H, 512]
+  int out_f32;
+  float* lse;                 // [B, H] or null
+};
+cudaError_t launch_cp_combine(const CpCombineArgs& a, cudaStream_t stream);
+
 }  // namespace ic

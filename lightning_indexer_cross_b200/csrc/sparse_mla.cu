@@ -588,7 +588,8 @@ IC_DEV void combine_half(const MlaArgs& a, int64_t gw, int half, int lane) {
   uint4 graw = make_uint4(0, 0, 0, 0);  // 8 bf16 gate logits, unpacked at the end
   if (a.gate) graw = __ldg(reinterpret_cast<const uint4*>(a.gate + gw * kDv + d0));
   const float sink2 = a.sink[h] * kLog2e;
-  float M = sink2, den = 1.f;  // the sink's term e^{sink - M}, M = sink so far
+  // the sink's term e^{sink - M}, M = sink so far (no term for a sink of -inf)
+  float M = sink2, den = sink2 == -INFINITY ? 0.f : 1.f;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -613,7 +614,7 @@ IC_DEV void combine_half(const MlaArgs& a, int64_t gw, int half, int lane) {
     float Mc = M;
 #pragma unroll
     for (int u = 0; u < CH; ++u) Mc = fmaxf(Mc, mlv[u].x);
-    const float sc = exp2f(M - Mc);
+    const float sc = M == Mc ? 1.f : exp2f(M - Mc);  // (M = Mc = -inf: nothing to rescale)
     den *= sc;
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] *= sc;
@@ -635,7 +636,7 @@ IC_DEV void combine_half(const MlaArgs& a, int64_t gw, int half, int lane) {
       }
     }
   }
-  const float inv = 1.f / den;
+  const float inv = den > 0.f ? 1.f / den : 0.f;  // (no valid row and no sink: out = 0)
   const uint32_t gwd[4] = {graw.x, graw.y, graw.z, graw.w};
   float o[8];
 #pragma unroll
@@ -655,7 +656,7 @@ IC_DEV void combine_half(const MlaArgs& a, int64_t gw, int half, int lane) {
     pk.w = pack_bf16x2(o[6], o[7]);
     *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + d0) = pk;
   }
-  if (a.lse && half == 0 && lane == 0) a.lse[gw] = (M + log2f(den)) / kLog2e;
+  if (a.lse && half == 0 && lane == 0) a.lse[gw] = den > 0.f ? (M + log2f(den)) / kLog2e : -INFINITY;
 }
 
 // The split combine: one warp per half of a (query, head) row, after the
@@ -682,7 +683,7 @@ IC_DEV void combine_staged_row(const MlaArgs& a, const uint8_t* prow, const floa
   const int S = a.splits;
   float M = sink2;
   for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mr[s2].x);
-  float den = exp2f(sink2 - M);
+  float den = sink2 == -INFINITY ? 0.f : exp2f(sink2 - M);  // (no term for a sink of -inf)
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
@@ -714,7 +715,7 @@ IC_DEV void combine_staged_row(const MlaArgs& a, const uint8_t* prow, const floa
     add_split(s2 + 1);
   }
   if (s2 < S) add_split(s2);
-  const float inv = 1.f / den;
+  const float inv = den > 0.f ? 1.f / den : 0.f;  // (no valid row and no sink: out = 0)
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
     const uint32_t gwd[4] = {graw[c].x, graw[c].y, graw[c].z, graw[c].w};
@@ -737,7 +738,7 @@ IC_DEV void combine_staged_row(const MlaArgs& a, const uint8_t* prow, const floa
       *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + gw * kDv + 8 * q + 256 * c) = pk;
     }
   }
-  if (a.lse && q == 0) a.lse[gw] = (M + log2f(den)) / kLog2e;
+  if (a.lse && q == 0) a.lse[gw] = den > 0.f ? (M + log2f(den)) / kLog2e : -INFINITY;
 }
 
 // The split combine with the partials staged by TMA: CTA c takes head rows

@@ -192,6 +192,71 @@ def cache_append(k_raw: torch.Tensor, ln_gamma: torch.Tensor, ln_beta: torch.Ten
     return workspace
 
 
+def cp_candidates(scores: torch.Tensor, idx: torch.Tensor, offset: int, cand_score: Optional[torch.Tensor] = None,
+                  cand_idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None):
+    """(score, global position) of each local top-k entry of a shard: scores [B, N_local] fp32, idx [B, k]
+    int32 shard positions (-1 padding), offset = global position of the shard's first token."""
+    _need_cuda(scores, idx, cand_score, cand_idx)
+    _need_dense(scores, idx, cand_score, cand_idx)
+    B, N_local = scores.shape
+    k = idx.shape[1]
+    assert scores.dtype == torch.float32 and idx.dtype == torch.int32 and idx.shape[0] == B
+    if cand_score is None:
+        cand_score = torch.empty((B, k), dtype=torch.float32, device=scores.device)
+    if cand_idx is None:
+        cand_idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    assert cand_score.shape == (B, k) and cand_idx.shape == (B, k)
+    assert cand_score.dtype == torch.float32 and cand_idx.dtype == torch.int32
+    if workspace is None:
+        workspace = new_workspace(_abi.ic_cp_workspace_size(), scores.device)
+    _abi.ic_cp_candidates(_ptr(scores), _ptr(idx), B, N_local, k, int(offset), _ptr(cand_score), _ptr(cand_idx),
+                          _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    return cand_score, cand_idx
+
+
+def cp_merge_topk(cand_score: torch.Tensor, cand_idx: torch.Tensor, k: int, lo: int = 0, hi: int = 0,
+                  idx_global: Optional[torch.Tensor] = None, idx_local: Optional[torch.Tensor] = None,
+                  want_local: bool = True, stream=None):
+    """Global top-k of the gathered candidates [G, B, kin] (fp32 scores, int32 global positions): ties toward
+    the lower global position; also the positions inside the shard [lo, hi) (-1 elsewhere)."""
+    _need_cuda(cand_score, cand_idx, idx_global, idx_local)
+    _need_dense(cand_score, cand_idx, idx_global, idx_local)
+    G, B, kin = cand_score.shape
+    assert cand_idx.shape == (G, B, kin) and cand_score.dtype == torch.float32 and cand_idx.dtype == torch.int32
+    if idx_global is None:
+        idx_global = torch.empty((B, k), dtype=torch.int32, device=cand_score.device)
+    if idx_local is None and want_local:
+        idx_local = torch.empty((B, k), dtype=torch.int32, device=cand_score.device)
+    assert idx_global.shape == (B, k) and (idx_local is None or idx_local.shape == (B, k))
+    _abi.ic_cp_merge_topk(_ptr(cand_score), _ptr(cand_idx), B * kin, G, B, kin, k, int(lo), int(hi),
+                          _ptr(idx_global), _ptr(idx_local), _stream_ptr(stream))
+    return idx_global, idx_local
+
+
+def cp_combine(part_out: torch.Tensor, part_lse: torch.Tensor, sink: torch.Tensor,
+               gate: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
+               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = False,
+               stream=None):
+    """Merge the ranks' partial attention outputs part_out [G, B, H, 512] fp32 (normalised, no sink) and
+    part_lse [G, B, H] fp32: the sink added once, then the gate [B, H, 512] bf16."""
+    _need_cuda(part_out, part_lse, sink, gate, out, lse)
+    _need_dense(part_out, part_lse, sink, gate, out, lse)
+    G, B, H, D = part_out.shape
+    assert D == D_V and part_lse.shape == (G, B, H) and part_out.dtype == torch.float32
+    assert part_lse.dtype == torch.float32 and sink.shape == (H,) and sink.dtype == torch.float32
+    assert gate is None or (gate.shape == (B, H, D_V) and gate.dtype == torch.bfloat16)
+    if out is None:
+        out = torch.empty((B, H, D_V), dtype=out_dtype, device=part_out.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=part_out.device)
+    assert out.shape == (B, H, D_V) and out.dtype in (torch.bfloat16, torch.float32)
+    _abi.ic_cp_combine(_ptr(part_out), B * H * D_V, _ptr(part_lse), B * H, G, B, H, _ptr(sink), _ptr(gate),
+                       _abi.IC_F32 if out.dtype == torch.float32 else _abi.IC_BF16, _ptr(out), _ptr(lse),
+                       _stream_ptr(stream))
+    return out, lse
+
+
 class LayerStack:
     """Holds the per-layer pointer table, the shape struct, the index buffer
     and the workspace of one decode stack, so that a step is one C call."""
