@@ -313,10 +313,18 @@ def run_native(args):
 
     # ------------------------------------------------------------------ per-kernel timing
     kern = time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst)
+    step_roof_us = kern.pop("step_roofline_us")
     try:  # reported beside the step, never part of it; a failure here is recorded, not fatal
         kern["cache_append"] = time_cache_append(dev, hbm_gbs)
     except Exception as e:  # noqa: BLE001
         kern["cache_append"] = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        kern["decompress_gate"] = time_gate(dev, hbm_gbs, tf_burst)
+    except Exception as e:  # noqa: BLE001
+        kern["decompress_gate"] = {"error": f"{type(e).__name__}: {e}"}
+    configs = None
+    if not args.no_configs:
+        configs = time_configs(dev, hbm_gbs, tf_burst)
     clk.stop()
     clocks = clk.summary()
 
@@ -346,12 +354,22 @@ def run_native(args):
         "roofline": roof,
         "kernels": {k: {kk: vv for kk, vv in v.items()} for k, v in kern.items()},
         "kernel_share_of_step": {k: v / sum(per_step.values()) for k, v in per_step.items()},
+        "step_roofline": {"us": step_roof_us, "ms_per_step": ms_max / args.steps,
+                          "frac": step_roof_us / 1000.0 / (ms_max / args.steps),
+                          "sum_of": "21 x (indexer + top-k) + 78 x sparse MLA, each max(bytes/HBM, FLOP/tensor) "
+                                    "of measured peaks"},
         "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops": tf_burst, "kind": peak_kind},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if configs is not None:
+        line["configs"] = configs
+        ref = configs.get("single_F_B8_N131072_per_query_caches", {}).get("indexer")
+        if ref and "roofline" in ref:
+            line["indexer_hbm_128k"] = {"workload": "single_F_B8_N131072_per_query_caches", "gbs": ref["gbs"],
+                                        "frac_of_hbm": ref["gbs"] / hbm_gbs, "us": ref["us"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, ta = cpu_sample_step()
         tf, ta = cpu_sample_step(seed=8)
@@ -397,6 +415,153 @@ def _time_loop(fn, n, stream, replays=3):
     e1.record(cur)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) * 1000.0 / (n * replays)  # us
+
+
+def roofline_time_us(bytes_, flops, hbm_gbs, tf_peak):
+    """The kernel's roofline time: the slower of moving its algorithmic bytes
+    at the HBM peak and doing its FLOPs at the tensor peak."""
+    return max(bytes_ / (hbm_gbs * 1e9), flops / (tf_peak * 1e12)) * 1e6
+
+
+def roofline_of(bytes_, flops, us, hbm_gbs, tf_peak):
+    """Achieved rate against the bound that sets the kernel's roofline."""
+    t_hbm = bytes_ / (hbm_gbs * 1e9)
+    t_tc = flops / (tf_peak * 1e12)
+    if t_tc > t_hbm:
+        ach = flops / (us * 1e-6) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": tf_peak, "unit": "TFLOP/s",
+                "frac": ach / tf_peak, "algorithmic_flops": flops, "algorithmic_bytes": bytes_}
+    ach = bytes_ / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s", "frac": ach / hbm_gbs,
+            "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
+
+
+def indexer_work(B, N, H_I, d_I, key_bytes_per_token, shared):
+    """Algorithmic bytes and FLOPs of one indexer call: every key read once
+    (once per query with per-query caches), queries and weights, the score
+    row written."""
+    keys = N * key_bytes_per_token * (1 if shared else B)
+    return keys + B * H_I * d_I * 2 + B * H_I * 4 + B * N * 4, 2.0 * B * H_I * d_I * N
+
+
+def topk_work(B, N, k):
+    return B * N * 4 + B * k * 4
+
+
+def mla_work(rows, B, H, k, gate):
+    """Gathered rows once each, q, the output (and gate) once, the indices."""
+    return (rows * D_QK * 2 + B * H * D_QK * 2 + B * H * D_V * 2 * (2 if gate else 1) + B * k * 4,
+            2.0 * B * H * k * (D_QK + D_V))
+
+
+def time_configs(dev, hbm_gbs, tf_burst):
+    """The other workloads' kernels, each timed alone (graph of n launches,
+    CUDA events on its stream): the single F layer at model shape (8 queries,
+    per-query caches of 131072 tokens), the 1M-token context (4 queries,
+    bf16 and e4m3 keys) and the prefill chunk (2048 causal queries over
+    264192 tokens). Inputs are larger than L2 except where noted."""
+    import gc
+    import torch
+    from lightning_indexer_cross_b200 import _abi, ops
+    from lightning_indexer_cross_b200 import workloads as W
+    stream = torch.cuda.Stream(device=dev)
+    res = {}
+
+    def leg(wl, n_ind, n_mla):
+        lay = wl.layers[0]
+        B, N = wl.B, wl.N
+        scores = torch.empty((B, N), dtype=torch.float32, device=dev)
+        idx = torch.empty((B, wl.topk), dtype=torch.int32, device=dev)
+        out = torch.empty((B, wl.H, D_V), dtype=torch.bfloat16, device=dev)
+        ws_i = ops.new_workspace(_abi.ic_indexer_workspace_size(), dev)
+        ws_t = ops.new_workspace(_abi.ic_topk_workspace_size(B, N, wl.topk), dev)
+        ws_m = ops.new_workspace(_abi.ic_sparse_mla_workspace_size(B, wl.H, wl.topk), dev)
+
+        def ind(i):
+            ops.indexer_score(lay.q_idx, lay.w, lay.k_idx, lay.k_scale, wl.n_valid, scores=scores, workspace=ws_i)
+
+        def tk(i):
+            ops.topk(scores, wl.topk, wl.n_valid, idx=idx, workspace=ws_t)
+
+        def mla(i):
+            ops.sparse_mla_decode(lay.q, lay.kv, idx, lay.sink, lay.gate, sm_scale=wl.sm_scale, out=out,
+                                  want_lse=False, workspace=ws_m)
+
+        ind(0)
+        tk(0)
+        mla(0)
+        torch.cuda.synchronize()
+        rows = 0
+        kvb = lay.kv.shape[0]
+        for b in range(B):
+            sel = idx[b][idx[b] >= 0]
+            rows += int(sel.numel()) if kvb > 1 else 0
+        if kvb == 1:
+            rows = int(torch.unique(idx[idx >= 0]).numel())
+        t_i = _time_loop(ind, n_ind, stream)
+        t_t = _time_loop(tk, n_ind, stream)
+        t_m = _time_loop(mla, n_mla, stream)
+        if _abi.ic_last_device_status(ops._ptr(ws_i), ops._stream_ptr()) != _abi.IC_OK:
+            raise RuntimeError("device status not OK")
+        kb = (wl.d_I + 4) if wl.k_fp8 else wl.d_I * 2
+        ib, iflops = indexer_work(B, N, wl.H_I, wl.d_I, kb, wl.shared_keys)
+        if wl.n_valid is not None:  # causal: only the visible keys are scored
+            nv = wl.n_valid.double()
+            iflops = 2.0 * wl.H_I * wl.d_I * float(nv.sum())
+        mb, mflops = mla_work(rows, B, wl.H, wl.topk, lay.gate is not None)
+        return {
+            "indexer": {"us": t_i, "gbs": ib / (t_i * 1e-6) / 1e9,
+                        "roofline": roofline_of(ib, iflops, t_i, hbm_gbs, tf_burst)},
+            "topk": {"us": t_t, "elems_per_s": B * N / (t_t * 1e-6),
+                     "roofline": roofline_of(topk_work(B, N, wl.topk), 0.0, t_t, hbm_gbs, tf_burst)},
+            "sparse_mla": {"us": t_m, "gathered_rows": rows,
+                           "roofline": roofline_of(mb, mflops, t_m, hbm_gbs, tf_burst)},
+        }
+
+    cases = [
+        ("single_F_B8_N131072_per_query_caches", lambda: W.single_f(dev), 6, 6),
+        ("long_ctx_B4_N1048576_bf16", lambda: W.long_context(dev, fp8=False), 3, 6),
+        ("long_ctx_B4_N1048576_e4m3", lambda: W.long_context(dev, fp8=True), 3, 6),
+        ("prefill_C2048_P262144_causal", lambda: W.prefill(dev), 2, 2),
+    ]
+    for name, make, n_ind, n_mla in cases:
+        try:
+            wl = make()
+            torch.cuda.synchronize()
+            res[name] = leg(wl, n_ind, n_mla)
+        except Exception as e:  # noqa: BLE001  (recorded, not fatal: the headline step is measured above)
+            res[name] = {"error": f"{type(e).__name__}: {e}"}
+        wl = None
+        gc.collect()
+        torch.cuda.empty_cache()
+    return res
+
+
+def time_gate(dev, hbm_gbs, tf_burst):
+    """The decompressed-space gate after each layer's attention at the
+    stack's decode shape (32 queries, 128 heads, d_v 128): 16 weight sets
+    rotated (269 MB, more than L2), one launch per layer in a graph."""
+    import torch
+    from lightning_indexer_cross_b200 import _abi, ops
+    from lightning_indexer_cross_b200 import workloads as Wl
+    stream = torch.cuda.Stream(device=dev)
+    sets = [Wl.gate_case(B, H, seed=90 + i, device=dev) for i in range(16)]
+    ws = ops.new_workspace(_abi.ic_decompress_gate_workspace_size(), dev)
+    out = torch.empty((B, H, 128), dtype=torch.bfloat16, device=dev)
+
+    def g(i):
+        o, w, gl = sets[i % len(sets)]
+        ops.decompress_gate(o, w, gl, out=out, workspace=ws)
+
+    for i in range(3):
+        g(i)
+    torch.cuda.synchronize()
+    us = _time_loop(g, L, stream)
+    if _abi.ic_last_device_status(ops._ptr(ws), ops._stream_ptr()) != _abi.IC_OK:
+        raise RuntimeError("device status not OK after the gate launches")
+    bytes_ = H * 128 * D_V * 2 + B * H * D_V * 2 + B * H * 128 * 2 * 2
+    flops = 2.0 * B * H * 128 * D_V
+    return {"us": us, "launches": L, "roofline": roofline_of(bytes_, flops, us, hbm_gbs, tf_burst)}
 
 
 def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
@@ -445,25 +610,19 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
     t_mla = _time_loop(mla, wl.L, stream)
 
     # algorithmic work per launch
-    ind_bytes = N * D_I * 2 + B * H_I * D_I * 2 + B * H_I * 4 + B * N * 4
-    ind_flops = 2.0 * B * H_I * D_I * N
-    tk_bytes = B * N * 4 + B * TOPK * 4
+    ind_bytes, ind_flops = indexer_work(B, N, H_I, D_I, D_I * 2, True)
+    tk_bytes = topk_work(B, N, TOPK)
     mla_rows = rows_distinct / wl.L
-    mla_bytes = mla_rows * D_QK * 2 + B * H * D_QK * 2 + B * H * D_V * 2 * 2 + B * TOPK * 4
-    mla_flops = 2.0 * B * H * TOPK * (D_QK + D_V)
+    mla_bytes, mla_flops = mla_work(mla_rows, B, H, TOPK, True)
 
     def roofline(bytes_, flops, us):
-        t_hbm = bytes_ / (hbm_gbs * 1e9)
-        t_tc = flops / (tf_burst * 1e12)
-        if t_tc > t_hbm:
-            ach = flops / (us * 1e-6) / 1e12
-            return {"bound": "tensor", "achieved": ach, "peak": tf_burst, "unit": "TFLOP/s",
-                    "frac": ach / tf_burst, "algorithmic_flops": flops, "algorithmic_bytes": bytes_}
-        ach = bytes_ / (us * 1e-6) / 1e9
-        return {"bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s", "frac": ach / hbm_gbs,
-                "algorithmic_bytes": bytes_, "algorithmic_flops": flops}
+        return roofline_of(bytes_, flops, us, hbm_gbs, tf_burst)
 
+    step_roof_us = (N_FULL * (roofline_time_us(ind_bytes, ind_flops, hbm_gbs, tf_burst) +
+                              roofline_time_us(tk_bytes, 0.0, hbm_gbs, tf_burst)) +
+                    L * roofline_time_us(mla_bytes, mla_flops, hbm_gbs, tf_burst))
     return {
+        "step_roofline_us": step_roof_us,
         "indexer": {"us": t_ind, "launches": reps, "gbs": ind_bytes / (t_ind * 1e-6) / 1e9,
                     "roofline": roofline(ind_bytes, ind_flops, t_ind)},
         "topk": {"us": t_tk, "launches": reps, "elems_per_s": B * N / (t_tk * 1e-6),
@@ -591,6 +750,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip timing the other workloads' kernels")
     ap.add_argument("--warmup-ref", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3:
