@@ -174,9 +174,10 @@ TopkLayout topk_layout(int B, int64_t N) {
   // the k-th key's 1/16-octave bin rarely holds more than a few percent of a
   // row; bigger bins fall back to passes over the row itself
   L.cand_cap = static_cast<int>(std::min<int64_t>(N, std::max<int64_t>(4096, N / 16)));
-  L.cnt_off = 0;  // control words: zero between calls
+  L.cnt_off = 0;  // control words and row histograms: zero between calls
   L.hist_off = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
-  L.cand_off = align256(L.hist_off + size_t(B) * std::max<int64_t>(L.cpr, cpr) * 4096 * 4);
+  L.cand_off = align256(L.hist_off + size_t(B) * 4096 * 4);
+  L.zero_bytes = L.cand_off;
   L.ckey_off = align256(L.cand_off + size_t(B) * L.cand_cap * 4);
   L.total = align256(L.ckey_off + size_t(B) * L.cand_cap * 4);
   return L;

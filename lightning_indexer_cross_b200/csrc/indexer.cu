@@ -26,10 +26,14 @@
 //               the TMA loads of the groups' Q (swizzled, zero-padded heads).
 //               bf16 keys: warps 2..9, two per TMEM lane quadrant, each
 //               reducing one half of the columns; e4m3 keys: warps 2..5.
-//   warps 6..9  (e4m3 keys only) convert e4m3 tiles to bf16 in shared memory.
-//               tcgen05 kind::f16 needs both operands bf16, and the e4m3 ->
-//               bf16 widening is exact; the per-token scale is applied to the
-//               head sum, since ReLU(c x) = c ReLU(x) for c >= 0.
+//   warps 6..9  (e4m3 keys only) widen e4m3 tiles to f16 in shared memory
+//               (one conversion instruction per two codes; exact) and, once
+//               per query group, the staged bf16 queries to f16 in place:
+//               tcgen05 kind::f16 takes two f16 (or two bf16) operands. A bf16
+//               query value is exact in f16 from 2^-14 up to 65504 (below,
+//               f16 keeps fewer bits: an error under 2^-25; the e4m3 path
+//               needs |q| < 65504). The per-token scale is applied to the head
+//               sum, since ReLU(c x) = c ReLU(x) for c >= 0.
 #include <cuda_fp8.h>
 
 #include <type_traits>
@@ -74,7 +78,7 @@ struct IdxCfg {
   static constexpr int kOffW = kOffQ + kQBytes;
   static constexpr int kOffNv = kOffW + kQSlots * kMaxCols * 4;
   static constexpr int kOffBar = kOffNv + kQSlots * 16 * 8;
-  static constexpr int kNumBars = 2 * kStages + 2 * kRawStages + 4 + 2;
+  static constexpr int kNumBars = 2 * kStages + 2 * kRawStages + 4 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(!(FP8 && PAIR), "e4m3 keys take one group per tile");
@@ -104,6 +108,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   uint64_t* acc_empty = acc_full + 2;             // [2]
   uint64_t* q_ready = acc_empty + 2;              // [1]
   uint64_t* mma_done = q_ready + 1;               // [1] every MMA issued has completed
+  uint64_t* q_conv = mma_done + 1;                // [1] (e4m3 keys) the queries are in f16
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -133,6 +138,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     }
     mbar_init(q_ready, 1);
     mbar_init(mma_done, 1);
+    mbar_init(q_conv, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -187,7 +193,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, ncols, false, false);
+      // bf16 keys: bf16 x bf16; e4m3 keys: both operands widened to f16
+      const uint32_t idesc = FP8 ? idesc_f16_f32(128, ncols) : idesc_bf16_f32(128, ncols, false, false);
       const uint32_t q_addr = smem_u32(qs);
       int cur_grp = -1;
       uint32_t q_phase = 0;
@@ -197,7 +204,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         const int grp = static_cast<int>(wi / a.tiles) * P;
         const int ng = P == 1 ? 1 : (a.groups - grp < P ? a.groups - grp : P);
         if (grp != cur_grp) {
-          if (!mbar_wait(q_ready, q_phase, abort_flag, a.status, a.wait_ns)) break;
+          if (!mbar_wait(FP8 ? q_conv : q_ready, q_phase, abort_flag, a.status, a.wait_ns)) break;
           q_phase ^= 1;
           cur_grp = grp;
         }
@@ -237,6 +244,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     const int row = quad * 32 + lane;                // key row inside the tile
     int cur_grp = -1;
     int64_t si = 0;  // (item, group) sub-items, as counted by the MMA issuer
+    uint32_t q_loads = 0;  // query-slot loads issued (by thread et == 0)
     bool got = true;
     for (int64_t wi = lo; wi < hi && got; ++wi) {
       const int grp = static_cast<int>(wi / a.tiles) * P;
@@ -251,6 +259,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         // HP heads, G queries), written in the 128-byte-swizzled K-major
         // layout the MMA reads; heads past H_I and queries past B are zero
         // filled. The MMA issuer waits for the bytes on q_ready.
+        ++q_loads;
         if (et == 0) {
           mbar_arrive_expect_tx(q_ready, static_cast<uint32_t>(ng * C::kBlocks * HP * a.G * 128));
           for (int slot = 0; slot < ng; ++slot)
@@ -431,11 +440,43 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       }
       }
     }
+    // the last query-slot load this thread issued has landed before the CTA
+    // can exit (it is otherwise waited on only by the MMA issuer, which may
+    // have given up)
+    if (et == 0 && q_loads > 0) mbar_drain(q_ready, (q_loads - 1) & 1u);
   } else if constexpr (FP8) {
-    // ------------------------------------------------------------ e4m3 -> bf16
+    // ------------------------------------------------------------ e4m3 -> f16
     const int ct = threadIdx.x - (kEpiWarp0 + 4) * 32;  // 0..127
     int64_t it = 0;
+    int cur_grp = -1;
+    uint32_t q_phase = 0;
     for (int64_t wi = lo; wi < hi; ++wi, ++it) {
+      const int grp = static_cast<int>(wi / a.tiles) * P;
+      if (grp != cur_grp) {
+        // the group's queries, staged as bf16 by TMA, become f16 in place
+        // (element by element, so the swizzled positions stay); the slot is
+        // rewritten only after the previous group's MMAs have completed
+        if (!mbar_wait(q_ready, q_phase, abort_flag, a.status, a.wait_ns)) break;
+        q_phase ^= 1;
+        cur_grp = grp;
+        constexpr int kRowChunks = 8;  // 16-byte chunks per 128-byte row
+        const int nchunks = C::kBlocks * ncols * kRowChunks;
+        for (int i = ct; i < nchunks; i += 128) {
+          const int bk = i / (ncols * kRowChunks), rem = i % (ncols * kRowChunks);
+          uint4* pq = reinterpret_cast<uint4*>(qs + bk * (kMaxCols * 128) + rem * 16);
+          const uint4 v = *pq;
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const __half2 h = __floats2half2_rn(bf16_lane(w4[j], 0), bf16_lane(w4[j], 1));
+            o[j] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          *pq = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(q_conv);
+      }
       const int rs = static_cast<int>(it % C::kRawStages);
       const uint32_t rph = static_cast<uint32_t>((it / C::kRawStages) & 1);
       const int bs = static_cast<int>(it % C::kStages);
@@ -455,12 +496,10 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         for (int j = 0; j < 4; ++j) {
           const __half2_raw lo2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w4[j] & 0xFFFF), __NV_E4M3);
           const __half2_raw hi2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w4[j] >> 16), __NV_E4M3);
-          const float2 flo = __half22float2(*reinterpret_cast<const __half2*>(&lo2));
-          const float2 fhi = __half22float2(*reinterpret_cast<const __half2*>(&hi2));
-          o[2 * j] = pack_bf16x2(flo.x, flo.y);
-          o[2 * j + 1] = pack_bf16x2(fhi.x, fhi.y);
+          o[2 * j] = static_cast<uint32_t>(lo2.x) | (static_cast<uint32_t>(lo2.y) << 16);
+          o[2 * j + 1] = static_cast<uint32_t>(hi2.x) | (static_cast<uint32_t>(hi2.y) << 16);
         }
-        // 16 bf16 = two 16-byte chunks: element offsets c*16 and c*16+8
+        // 16 f16 = two 16-byte chunks: element offsets c*16 and c*16+8
         const int e0 = c * 16;
         const uint32_t base = smem_u32(dst + (e0 >> 6) * (kTileKeys * 128));
         const int ch = (e0 & 63) >> 3;

@@ -107,7 +107,7 @@ struct TopkArgs {
   const float* scores;      // [B, N]
   const int64_t* n_valid;   // [B] or null
   int32_t* idx;             // [B, k]
-  uint32_t* hist;           // [B][cpr][4096] per-CTA histograms of the top 12 key bits
+  uint32_t* hist;           // [B][4096] row histograms of the top 12 key bits (zero between calls)
   int32_t* cand;            // [B][cand_cap] candidate positions (the k-th key's bin)
   uint32_t* cand_key;       // [B][cand_cap] their order-preserving keys
   uint32_t* counters;       // [B][kCtrlWords] per-row control state
@@ -130,10 +130,12 @@ struct TopkLayout {
   int fused;       // one clustered launch (cpr <= 4, slices <= 32768 scores)
   int cand_cap;
   size_t hist_off, cand_off, ckey_off, cnt_off, total;
+  size_t zero_bytes;  // [0, zero_bytes): control words and row histograms, zero between calls
 };
 TopkLayout topk_layout(int B, int64_t N);
-// Validate and enqueue the top-k passes. The control words (cnt_off) must be
-// zero on entry; every call that completes leaves them zero again.
+// Validate and enqueue the top-k passes. The control words and row
+// histograms ([0, zero_bytes)) must be zero on entry; every call that
+// completes leaves them zero again.
 ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_valid, int k, int32_t* idx,
                       uint8_t* ws, size_t ws_bytes, int* status, cudaStream_t stream, bool pdl);
 

@@ -4,10 +4,11 @@
 // Radix select on the order-preserving 32-bit key of each fp32 score
 // (negative floats: all bits flipped; others: sign bit set). Two launches,
 // neither of which ever waits on another CTA:
-//   histogram  each CTA writes the 12-bit histogram of key[31:20] over its
-//              slice of the row to its own slot; the last CTA of the row
-//              (atomic ticket) sums the slots and picks the bin d1 holding
-//              the k-th key.
+//   histogram  each CTA builds the 12-bit histogram of key[31:20] over its
+//              slice of the row in shared memory and adds its nonzero bins
+//              into the row's histogram in global memory; the last CTA of the
+//              row (atomic ticket) reads it once, clears it for the next
+//              call and picks the bin d1 holding the k-th key.
 //   filter     keys in bins above d1 are final and are written straight to
 //              the output (compacted per CTA with one warp scan per 128
 //              keys, one atomic reservation per CTA); keys in bin d1 are
@@ -192,7 +193,7 @@ IC_DEV void list_push(int32_t* list, uint32_t* count, uint32_t cap, int64_t i, b
 
 // ------------------------------------------------------------------ pass 1
 __global__ void __launch_bounds__(kThreads) topk_hist_kernel(const TopkArgs a) {
-  __shared__ uint32_t sh_hist[kBins1];
+  __shared__ __align__(16) uint32_t sh_hist[kBins1];
   __shared__ uint32_t warp_tot[kWarps];
   __shared__ int sh_d;
   __shared__ uint32_t sh_kr;
@@ -209,13 +210,13 @@ __global__ void __launch_bounds__(kThreads) topk_hist_kernel(const TopkArgs a) {
   if (lo < hi)
     for_slice(a, b, lo, hi, [&](int64_t, uint32_t key, bool valid) { hist_add(sh_hist, key >> 20, valid); });
   __syncthreads();
-  // this CTA's histogram to its own slot (every bin; no atomics)
-  uint4* slots = reinterpret_cast<uint4*>(a.hist + static_cast<int64_t>(b) * a.cpr * kBins1);
-  constexpr int kVec = kBins1 / 4;  // uint4 per histogram
-  for (int j = threadIdx.x; j < kVec; j += kThreads)
-    slots[static_cast<int64_t>(c) * kVec + j] = reinterpret_cast<const uint4*>(sh_hist)[j];
-  // the last CTA of the row sums the slots and picks the bin of the k-th key
-  // once for everyone
+  // this CTA's nonzero bins into the row's histogram (a few hundred atomics)
+  uint32_t* rh = a.hist + static_cast<int64_t>(b) * kBins1;
+  for (int j = threadIdx.x; j < kBins1; j += kThreads) {
+    const uint32_t v = sh_hist[j];
+    if (v) atomicAdd(&rh[j], v);
+  }
+  // the last CTA of the row picks the bin of the k-th key once for everyone
   uint32_t* ctrl = row_ctrl(a, b);
   __threadfence();
   __syncthreads();
@@ -223,29 +224,10 @@ __global__ void __launch_bounds__(kThreads) topk_hist_kernel(const TopkArgs a) {
   __syncthreads();
   if (!sh_last) return;
   __threadfence();
-  for (int j = threadIdx.x; j < kVec; j += kThreads) {
-    uint4 acc = make_uint4(0, 0, 0, 0);
-    int s0 = 0;
-    for (; s0 + 4 <= a.cpr; s0 += 4) {  // four slots' loads in flight
-      uint4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __ldcg(&slots[static_cast<int64_t>(s0 + u) * kVec + j]);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc.x += v[u].x;
-        acc.y += v[u].y;
-        acc.z += v[u].z;
-        acc.w += v[u].w;
-      }
-    }
-    for (; s0 < a.cpr; ++s0) {
-      const uint4 v = __ldcg(&slots[static_cast<int64_t>(s0) * kVec + j]);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    reinterpret_cast<uint4*>(sh_hist)[j] = acc;
+  // read the whole row's histogram, and leave it zero for the next call
+  for (int j = threadIdx.x; j < kBins1 / 4; j += kThreads) {
+    reinterpret_cast<uint4*>(sh_hist)[j] = __ldcg(reinterpret_cast<const uint4*>(rh) + j);
+    reinterpret_cast<uint4*>(rh)[j] = make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
   select_digit(sh_hist, kBins1, static_cast<uint32_t>(a.k), &sh_d, &sh_kr, warp_tot);

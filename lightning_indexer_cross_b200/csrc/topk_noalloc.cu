@@ -77,11 +77,10 @@ extern "C" ic_status_t ic_topk_noalloc(const float* scores, int B, int64_t N, co
   if (scratch_address(&base) != cudaSuccess) return IC_ERR_CUDA;
   uint8_t* scratch = static_cast<uint8_t*>(base);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the status word and the control words start at zero on every call
-  // (a previous call that hit a device error may have left them set)
-  if (cudaMemsetAsync(scratch, 0, kStatusBytes, s) != cudaSuccess) return IC_ERR_CUDA;
-  if (cudaMemsetAsync(scratch + kStatusBytes + L.cnt_off, 0, size_t(B) * ic::kCtrlWords * 4, s) != cudaSuccess)
-    return IC_ERR_CUDA;
+  // the status word, the control words and the row histograms start at zero
+  // on every call (a previous call that hit a device error may have left
+  // them set)
+  if (cudaMemsetAsync(scratch, 0, kStatusBytes + L.zero_bytes, s) != cudaSuccess) return IC_ERR_CUDA;
   return ic::topk_impl(scores, B, N, n_valid, k, idx, scratch + kStatusBytes, kScratchBytes - kStatusBytes,
                        reinterpret_cast<int*>(scratch), s, false);
 }
