@@ -467,7 +467,7 @@ def time_configs(dev, hbm_gbs, tf_burst):
     stream = torch.cuda.Stream(device=dev)
     res = {}
 
-    def leg(wl, n_ind, n_mla):
+    def leg(wl, n_ind, n_mla, rows_per_pass=None):
         lay = wl.layers[0]
         B, N = wl.B, wl.N
         scores = torch.empty((B, N), dtype=torch.float32, device=dev)
@@ -501,6 +501,20 @@ def time_configs(dev, hbm_gbs, tf_burst):
         t_i = _time_loop(ind, n_ind, stream)
         t_t = _time_loop(tk, n_ind, stream)
         t_m = _time_loop(mla, n_mla, stream)
+        fused = {}
+        if rows_per_pass is not None:
+            ws_f = ops.new_workspace(_abi.ic_indexer_topk_workspace_size(B, N, wl.topk, rows_per_pass), dev)
+
+            def fz(i):
+                ops.indexer_topk(lay.q_idx, lay.w, lay.k_idx, wl.topk, lay.k_scale, wl.n_valid,
+                                 rows_per_pass=rows_per_pass, idx=idx, workspace=ws_f)
+
+            fz(0)
+            torch.cuda.synchronize()
+            t_f = _time_loop(fz, n_ind, stream)
+            fused = {"indexer_topk": {"us": t_f, "rows_per_pass": rows_per_pass,
+                                      "score_scratch_bytes": int(ws_f.numel())}}
+            del ws_f
         if _abi.ic_last_device_status(ops._ptr(ws_i), ops._stream_ptr()) != _abi.IC_OK:
             raise RuntimeError("device status not OK")
         kb = (wl.d_I + 4) if wl.k_fp8 else wl.d_I * 2
@@ -516,19 +530,20 @@ def time_configs(dev, hbm_gbs, tf_burst):
                      "roofline": roofline_of(topk_work(B, N, wl.topk), 0.0, t_t, hbm_gbs, tf_burst)},
             "sparse_mla": {"us": t_m, "gathered_rows": rows,
                            "roofline": roofline_of(mb, mflops, t_m, hbm_gbs, tf_burst)},
+            **fused,
         }
 
     cases = [
-        ("single_F_B8_N131072_per_query_caches", lambda: W.single_f(dev), 6, 6),
-        ("long_ctx_B4_N1048576_bf16", lambda: W.long_context(dev, fp8=False), 3, 6),
-        ("long_ctx_B4_N1048576_e4m3", lambda: W.long_context(dev, fp8=True), 3, 6),
-        ("prefill_C2048_P262144_causal", lambda: W.prefill(dev), 2, 2),
+        ("single_F_B8_N131072_per_query_caches", lambda: W.single_f(dev), 6, 6, None),
+        ("long_ctx_B4_N1048576_bf16", lambda: W.long_context(dev, fp8=False), 3, 6, None),
+        ("long_ctx_B4_N1048576_e4m3", lambda: W.long_context(dev, fp8=True), 3, 6, None),
+        ("prefill_C2048_P262144_causal", lambda: W.prefill(dev), 2, 2, 128),
     ]
-    for name, make, n_ind, n_mla in cases:
+    for name, make, n_ind, n_mla, rpp in cases:
         try:
             wl = make()
             torch.cuda.synchronize()
-            res[name] = leg(wl, n_ind, n_mla)
+            res[name] = leg(wl, n_ind, n_mla, rpp)
         except Exception as e:  # noqa: BLE001  (recorded, not fatal: the headline step is measured above)
             res[name] = {"error": f"{type(e).__name__}: {e}"}
         wl = None
@@ -600,10 +615,18 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
         ops.sparse_mla_decode(lay.q, lay.kv, idx_by_layer[gi], lay.sink, lay.gate, out=out, want_lse=False,
                               workspace=ws_m)
 
-    for fn in (ind, tk, mla):
+    ws_f = ops.new_workspace(_abi.ic_indexer_topk_workspace_size(B, N, TOPK, 0), dev)
+    idx_f = torch.empty((B, TOPK), dtype=torch.int32, device=dev)
+
+    def fused(i):
+        lay = wl.layers[f_layers[i % len(f_layers)]]
+        ops.indexer_topk(lay.q_idx, lay.w, lay.k_idx, TOPK, idx=idx_f, workspace=ws_f)
+
+    for fn in (ind, tk, mla, fused):
         for i in range(3):
             fn(i)
     torch.cuda.synchronize()
+    t_fused = _time_loop(fused, reps, stream)
     t_ind = _time_loop(ind, reps, stream)
     # top-k reads scores written just before (as in the stack); time it alone
     t_tk = _time_loop(tk, reps, stream)
@@ -623,6 +646,9 @@ def time_kernels(wl, st, args, dev, rows_distinct, hbm_gbs, tf_burst):
                     L * roofline_time_us(mla_bytes, mla_flops, hbm_gbs, tf_burst))
     return {
         "step_roofline_us": step_roof_us,
+        "indexer_topk": {"us": t_fused, "launches": reps,
+                         "what": "ic_indexer_topk per F layer (indexer and top-k in one call)",
+                         "roofline": roofline(ind_bytes + tk_bytes, ind_flops, t_fused)},
         "indexer": {"us": t_ind, "launches": reps, "gbs": ind_bytes / (t_ind * 1e-6) / 1e9,
                     "roofline": roofline(ind_bytes, ind_flops, t_ind)},
         "topk": {"us": t_tk, "launches": reps, "elems_per_s": B * N / (t_tk * 1e-6),

@@ -105,6 +105,25 @@ ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_vali
 size_t ic_topk_workspace_size(int B, int64_t N, int k);
 
 /* ---------------------------------------------------------------------------
+ * ic_indexer_topk -- the indexer and the top-k of an F layer in one call
+ * (Hy4 IndexCache explainer, Jargon "Indexer" and "Top-k selection": the
+ * indexer's scores exist only to pick the k best tokens). Writes idx [B, k]
+ * exactly as ic_indexer_score followed by ic_topk would; the scores never
+ * leave the workspace, whose score scratch holds rows_per_pass rows at a
+ * time: the rows are scored and selected in passes of that many rows
+ * (rounded up to a multiple of 8; 0 = all B rows in one pass), so a long
+ * prefill chunk needs rows_per_pass * N * 4 bytes of scores, not B * N * 4.
+ * Arguments as for ic_indexer_score and ic_topk; the workspace must hold
+ * ic_indexer_topk_workspace_size(B, N, k, rows_per_pass) bytes and follows
+ * the workspace rules above (zeroed once before first use).
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_indexer_topk(const void* q, const float* w, const void* k, const float* k_scale,
+                            ic_dtype_t k_dtype, int B, int H_I, int d_I, int64_t N, int64_t k_batch_stride,
+                            int64_t scale_batch_stride, const int64_t* n_valid, int topk, int rows_per_pass,
+                            int32_t* idx, void* workspace, size_t ws_bytes, ic_stream_t stream);
+size_t ic_indexer_topk_workspace_size(int B, int64_t N, int k, int rows_per_pass);
+
+/* ---------------------------------------------------------------------------
  * ic_topk_noalloc -- ic_topk for callers that cannot allocate device memory.
  * The pages have no counterpart: this is an interface choice of the library.
  *
@@ -158,8 +177,8 @@ size_t ic_sparse_mla_workspace_size(int B, int H, int k);
 /* ---------------------------------------------------------------------------
  * ic_layer_stack -- the IndexCache decode step over L layers.
  *
- * Layer l with schedule[l] == 'F' runs ic_indexer_score and ic_topk and
- * overwrites index_buf; with 'S' it leaves index_buf as the last preceding
+ * Layer l with schedule[l] == 'F' runs ic_indexer_topk (the indexer and the
+ * top-k) and overwrites index_buf; with 'S' it leaves index_buf as the last preceding
  * F layer wrote it (Hy4-preview porting issue, "Indexer" bullet: shared
  * layers reuse the last preceding full layer's top-k). Every layer then runs
  * ic_sparse_mla_decode reading index_buf in place. schedule[0] must be 'F'.
@@ -193,6 +212,8 @@ typedef struct {
   int64_t scale_batch_stride;  /* elements between queries' key scales (0 = shared) */
   int64_t kv_batch_stride;     /* elements between queries' latent caches (0 = shared) */
   const int64_t* n_valid;      /* device [B] causal limits, or NULL */
+  int rows_per_pass;           /* F layers score and select this many rows at a time
+                                  (ic_indexer_topk); 0 = all B rows at once */
 } ic_stack_shape_t;
 
 typedef struct {

@@ -31,6 +31,8 @@ EXPORTED = [
     "ic_topk",
     "ic_topk_workspace_size",
     "ic_topk_noalloc",
+    "ic_indexer_topk",
+    "ic_indexer_topk_workspace_size",
     "ic_sparse_mla_decode",
     "ic_sparse_mla_workspace_size",
     "ic_layer_stack",
@@ -74,7 +76,7 @@ class ic_stack_shape_t(ctypes.Structure):
     _fields_ = [
         ("B", _i), ("N", _i64), ("H_I", _i), ("d_I", _i), ("k_dtype", _i), ("topk", _i), ("H", _i),
         ("sm_scale", _f), ("out_dtype", _i), ("k_batch_stride", _i64), ("scale_batch_stride", _i64),
-        ("kv_batch_stride", _i64), ("n_valid", _p),
+        ("kv_batch_stride", _i64), ("n_valid", _p), ("rows_per_pass", _i),
     ]
 
 
@@ -97,6 +99,9 @@ _indexer = _sig("ic_indexer_score", _i, [_p, _p, _p, _p, _i, _i, _i, _i, _i64, _
 _indexer_ws = _sig("ic_indexer_workspace_size", _sz, [])
 _topk = _sig("ic_topk", _i, [_p, _i, _i64, _p, _i, _p, _p, _sz, _p])
 _topk_ws = _sig("ic_topk_workspace_size", _sz, [_i, _i64, _i])
+_indexer_topk = _sig("ic_indexer_topk", _i,
+                     [_p, _p, _p, _p, _i, _i, _i, _i, _i64, _i64, _i64, _p, _i, _i, _p, _p, _sz, _p])
+_indexer_topk_ws = _sig("ic_indexer_topk_workspace_size", _sz, [_i, _i64, _i, _i])
 _topk_noalloc = _sig("ic_topk_noalloc", _i, [_p, _i, _i64, _p, _i, _p, _p])
 _mla = _sig("ic_sparse_mla_decode", _i,
             [_p, _p, _i64, _i64, _p, _i, _p, _p, _f, _i, _i, _i, _p, _p, _p, _sz, _p])
@@ -142,6 +147,16 @@ def ic_indexer_workspace_size() -> int:
 
 def ic_topk(scores, B, N, n_valid, k, idx, workspace, ws_bytes, stream) -> None:
     _check(_topk(scores, B, N, n_valid, k, idx, workspace, ws_bytes, stream), "ic_topk")
+
+
+def ic_indexer_topk(q, w, k, k_scale, k_dtype, B, H_I, d_I, N, k_batch_stride, scale_batch_stride, n_valid, topk,
+                    rows_per_pass, idx, workspace, ws_bytes, stream) -> None:
+    _check(_indexer_topk(q, w, k, k_scale, k_dtype, B, H_I, d_I, N, k_batch_stride, scale_batch_stride, n_valid,
+                         topk, rows_per_pass, idx, workspace, ws_bytes, stream), "ic_indexer_topk")
+
+
+def ic_indexer_topk_workspace_size(B, N, k, rows_per_pass) -> int:
+    return int(_indexer_topk_ws(B, N, k, rows_per_pass))
 
 
 def ic_topk_noalloc(scores, B, N, n_valid, k, idx, stream) -> None:

@@ -221,6 +221,70 @@ using ic::TopkLayout;
 using ic::topk_layout;
 using ic::topk_impl;
 
+// ------------------------------------------------------------------ indexer -> top-k
+// Rows per pass of the fused indexer -> top-k: all B rows when rows_per_pass
+// is 0, else rows_per_pass rounded up to a multiple of 8 (whole pairs of
+// 4-query groups; keeps every row offset of q, w and idx 16-byte aligned).
+int fused_rows(int B, int rows_per_pass) {
+  if (rows_per_pass <= 0 || rows_per_pass >= B) return B;
+  const int r = (rows_per_pass + 7) / 8 * 8;
+  return r < B ? r : B;
+}
+
+struct FusedLayout {
+  int R;
+  size_t scores_off, topk_off, total;  // offsets from the start of the region
+  TopkLayout tk;
+};
+
+FusedLayout fused_layout(int B, int64_t N, int rows_per_pass) {
+  FusedLayout L{};
+  L.R = fused_rows(B, rows_per_pass);
+  L.tk = topk_layout(L.R, N);
+  L.scores_off = 0;
+  L.topk_off = align256(size_t(L.R) * N * 4);
+  L.total = align256(L.topk_off + L.tk.total);
+  return L;
+}
+
+// Scores of R rows at a time into the region's scratch, then their top-k;
+// the next pass reuses the scratch. The first kernel launches with
+// programmatic serialisation only if `pdl` (it follows one of the
+// library's kernels in the stream).
+ic_status_t indexer_topk_impl(const void* q, const float* w, const void* k, const float* k_scale, ic_dtype_t k_dtype,
+                              int B, int H_I, int d_I, int64_t N, int64_t k_batch_stride, int64_t scale_batch_stride,
+                              const int64_t* n_valid, int topk, int rows_per_pass, int32_t* idx, uint8_t* region,
+                              size_t region_bytes, int* status, cudaStream_t stream, bool pdl, int* launches) {
+  if (!q || !w || !k || !idx || !region) return IC_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H_I < 1 || topk < 1) return IC_ERR_INVALID_ARG;
+  const FusedLayout L = fused_layout(B, N, rows_per_pass);
+  if (region_bytes < L.total || !aligned16(region)) return IC_ERR_INVALID_ARG;
+  const bool fp8 = k_dtype == IC_FP8_E4M3;
+  const int64_t esz = fp8 ? 1 : 2;
+  const bool per_query = k_batch_stride != 0 && B > 1;
+  const bool per_query_scale = scale_batch_stride != 0 && B > 1;
+  float* scores = reinterpret_cast<float*>(region + L.scores_off);
+  for (int r0 = 0; r0 < B; r0 += L.R) {
+    const int R = B - r0 < L.R ? B - r0 : L.R;
+    const uint8_t* qb = static_cast<const uint8_t*>(q) + size_t(r0) * H_I * d_I * 2;
+    const uint8_t* kb = static_cast<const uint8_t*>(k) + (per_query ? size_t(r0) * k_batch_stride * esz : 0);
+    const float* ksb = k_scale ? k_scale + (per_query_scale ? size_t(r0) * scale_batch_stride : 0) : nullptr;
+    const int64_t* nvb = n_valid ? n_valid + r0 : nullptr;
+    g_launches = 0;
+    ic_status_t st = indexer_impl(qb, w + size_t(r0) * H_I, kb, ksb, k_dtype, R, H_I, d_I, N,
+                                  per_query ? k_batch_stride : 0, per_query_scale ? scale_batch_stride : 0, nvb,
+                                  scores, status, stream, pdl || r0 > 0);
+    if (st != IC_OK) return st;
+    *launches += g_launches;
+    g_launches = 0;
+    st = topk_impl(scores, R, N, nvb, topk, idx + size_t(r0) * topk, region + L.topk_off, L.tk.total, status,
+                   stream, true);
+    if (st != IC_OK) return st;
+    *launches += g_launches;
+  }
+  return IC_OK;
+}
+
 // ------------------------------------------------------------------ sparse MLA
 // Selected rows per work unit: the largest of 256, 128 that still gives at
 // least 4/5 of a work unit per SM, else 64.
@@ -327,18 +391,17 @@ ic_status_t mla_impl(const void* q, const void* kv, int64_t kv_batch_stride, int
 
 // ------------------------------------------------------------------ stack
 struct StackLayout {
-  size_t scores_off, topk_off, mla_off, total;
-  TopkLayout tk;
+  size_t fused_off, mla_off, total;
+  FusedLayout fz;
   MlaLayout ml;
 };
 
 StackLayout stack_layout(const ic_stack_shape_t& s) {
   StackLayout L{};
-  L.tk = topk_layout(s.B, s.N);
+  L.fz = fused_layout(s.B, s.N, s.rows_per_pass);
   L.ml = mla_layout(s.B, s.H, s.topk);
-  L.scores_off = kStatusBytes;
-  L.topk_off = align256(L.scores_off + size_t(s.B) * s.N * 4);
-  L.mla_off = align256(L.topk_off + L.tk.total);
+  L.fused_off = kStatusBytes;
+  L.mla_off = align256(L.fused_off + L.fz.total);
   L.total = align256(L.mla_off + L.ml.total);
   return L;
 }
@@ -392,6 +455,28 @@ ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_vali
                    reinterpret_cast<int*>(ws), reinterpret_cast<cudaStream_t>(stream), false);
 }
 
+size_t ic_indexer_topk_workspace_size(int B, int64_t N, int k, int rows_per_pass) {
+  (void)k;
+  if (B < 1 || N < 1) return kStatusBytes;
+  return kStatusBytes + fused_layout(B, N, rows_per_pass).total;
+}
+
+ic_status_t ic_indexer_topk(const void* q, const float* w, const void* k, const float* k_scale, ic_dtype_t k_dtype,
+                            int B, int H_I, int d_I, int64_t N, int64_t k_batch_stride, int64_t scale_batch_stride,
+                            const int64_t* n_valid, int topk, int rows_per_pass, int32_t* idx, void* workspace,
+                            size_t ws_bytes, ic_stream_t stream) {
+  g_launches = 0;
+  if (!workspace || ws_bytes < kStatusBytes || !aligned16(workspace)) return IC_ERR_INVALID_ARG;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int n = 0;
+  const ic_status_t r = indexer_topk_impl(q, w, k, k_scale, k_dtype, B, H_I, d_I, N, k_batch_stride,
+                                          scale_batch_stride, n_valid, topk, rows_per_pass, idx, ws + kStatusBytes,
+                                          ws_bytes - kStatusBytes, reinterpret_cast<int*>(ws),
+                                          reinterpret_cast<cudaStream_t>(stream), false, &n);
+  g_launches = n;
+  return r;
+}
+
 size_t ic_sparse_mla_workspace_size(int B, int H, int k) {
   if (B < 1 || H < 1 || k < 1) return kStatusBytes;
   return kStatusBytes + mla_layout(B, H, k).total;
@@ -437,7 +522,6 @@ ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule
   if (ws_bytes < SL.total) return IC_ERR_INVALID_ARG;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int* status = reinterpret_cast<int*>(ws);
-  float* scores = reinterpret_cast<float*>(ws + SL.scores_off);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int total = 0;
   // Consecutive kernels of the stack overlap their launch and prologue with
@@ -452,17 +536,12 @@ ic_status_t ic_layer_stack(const ic_layer_t* layers, int L, const char* schedule
       after_kernel = false;
     }
     if (schedule[l] == 'F') {
-      g_launches = 0;
-      ic_status_t r = indexer_impl(y.q_idx, y.w, y.k_idx, y.k_scale, s.k_dtype, s.B, s.H_I, s.d_I, s.N,
-                                   s.k_batch_stride, s.scale_batch_stride, s.n_valid, scores, status, st,
-                                   after_kernel);
+      int n = 0;
+      ic_status_t r = indexer_topk_impl(y.q_idx, y.w, y.k_idx, y.k_scale, s.k_dtype, s.B, s.H_I, s.d_I, s.N,
+                                        s.k_batch_stride, s.scale_batch_stride, s.n_valid, s.topk, s.rows_per_pass,
+                                        index_buf, ws + SL.fused_off, SL.fz.total, status, st, after_kernel, &n);
       if (r != IC_OK) return r;
-      total += g_launches;
-      g_launches = 0;
-      r = topk_impl(scores, s.B, s.N, s.n_valid, s.topk, index_buf, ws + SL.topk_off, SL.tk.total, status, st,
-                    true);
-      if (r != IC_OK) return r;
-      total += g_launches;
+      total += n;
       after_kernel = true;
     }
     g_launches = 0;

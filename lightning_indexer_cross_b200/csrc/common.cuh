@@ -416,6 +416,14 @@ IC_DEV float2 ffma2(float2 a, float2 b, float2 c) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
   return d;
 }
+// Four e4m3 codes (one 32-bit word, lowest byte first) to four f16 values
+// (two f16x2 words, lowest first), exactly: one conversion per two codes.
+IC_DEV void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
 IC_DEV float bf16_lane(uint32_t w, int e) { return __uint_as_float(e ? (w & 0xffff0000u) : (w << 16)); }
 IC_DEV uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

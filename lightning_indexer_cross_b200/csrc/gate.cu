@@ -118,6 +118,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
     const int d = quad * 32 + lane;
+    // The gate logits of this thread's value dim for every query of the
+    // tile, requested before the accumulator wait so that their latency
+    // overlaps the MMAs (one round trip instead of one per query).
+    __nv_bfloat16 gl[kTileQ];
+#pragma unroll
+    for (int j = 0; j < kTileQ; ++j) {
+      gl[j] = __float2bfloat16_rn(0.f);
+      if (a.gate && j < nq) gl[j] = __ldg(a.gate + (static_cast<int64_t>(q0 + j) * a.H + h) * kDv + d);
+    }
     bool got = mbar_wait(acc_full, 0u, abort_flag, a.status, a.wait_ns);
     __syncwarp();  // tcgen05.ld below is warp-collective
     got = got && !*abort_flag;
@@ -125,20 +134,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (got) {
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-      for (int c0 = 0; c0 < n_mma; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32_issue(taddr + c0, r);  // columns past n_mma are allocated and ignored
-        tmem_ld_wait(r);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (c0 + j < nq) {
-            const int64_t o = (static_cast<int64_t>(q0 + c0 + j) * a.H + h) * kDv + d;
-            float v = __uint_as_float(r[j]);
-            if (a.gate) v *= 1.f / (1.f + __expf(-__bfloat162float(a.gate[o])));
-            if (a.out_f32)
-              static_cast<float*>(a.out)[o] = v;
-            else
-              static_cast<__nv_bfloat16*>(a.out)[o] = __float2bfloat16_rn(v);
+      for (int c0 = 0; c0 < kTileQ; c0 += 32) {
+        if (c0 < n_mma) {
+          uint32_t r[32];
+          tmem_ld32_issue(taddr + c0, r);  // columns past n_mma are allocated and ignored
+          tmem_ld_wait(r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (c0 + j < nq) {
+              const int64_t o = (static_cast<int64_t>(q0 + c0 + j) * a.H + h) * kDv + d;
+              float v = __uint_as_float(r[j]);
+              if (a.gate) v *= 1.f / (1.f + __expf(-__bfloat162float(gl[c0 + j])));
+              if (a.out_f32)
+                static_cast<float*>(a.out)[o] = v;
+              else
+                static_cast<__nv_bfloat16*>(a.out)[o] = __float2bfloat16_rn(v);
+            }
           }
         }
       }

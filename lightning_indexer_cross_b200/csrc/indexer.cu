@@ -24,9 +24,9 @@
 //   warps 2..    epilogue: TMEM -> registers -> score row; also stage the
 //               query groups' head weights, and one of their threads issues
 //               the TMA loads of the groups' Q (swizzled, zero-padded heads).
-//               bf16 keys: warps 2..9, two per TMEM lane quadrant, each
-//               reducing one half of the columns; e4m3 keys: warps 2..5.
-//   warps 6..9  (e4m3 keys only) widen e4m3 tiles to f16 in shared memory
+//               warps 2..9, two per TMEM lane quadrant, each reducing one
+//               half of the columns.
+//   warps 10..13 (e4m3 keys only) widen e4m3 tiles to f16 in shared memory
 //               (one conversion instruction per two codes; exact) and, once
 //               per query group, the staged bf16 queries to f16 in place:
 //               tcgen05 kind::f16 takes two f16 (or two bf16) operands. A bf16
@@ -62,15 +62,18 @@ struct IdxCfg {
   static constexpr int kQSlots = PAIR ? 2 : 1;
   static constexpr int kQSlotBytes = kMaxCols * D_I * 2;
   static constexpr int kQBytes = kQSlots * kQSlotBytes;
-  // bf16 keys: 8 epilogue warps, two per TMEM lane quadrant, each reducing
-  // one half of the columns (two warps per SM sub-partition hide each other's
-  // TMEM-load and FMA latencies; measured: four per quadrant at the 96
-  // registers of 18 warps spill and run slower). e4m3 keys: 4 epilogue warps
-  // (one per quadrant, whole rows) plus 4 converter warps.
-  static constexpr int kEpiWarps = FP8 ? 4 : 8;
-  static constexpr int kHalves = FP8 ? 1 : 2;
+  // 8 epilogue warps, two per TMEM lane quadrant, each reducing one half of
+  // the columns (two warps per SM sub-partition hide each other's TMEM-load
+  // and FMA latencies; measured: four per quadrant at the 96 registers of 18
+  // warps spill and run slower); e4m3 keys add 4 converter warps (measured at
+  // the 1M-token per-query shape: 260 us, against 292 us with 4 epilogue
+  // warps reducing whole rows, whose two 64-column loads in flight spilled).
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kHalves = 2;
   static constexpr int kEpiThreads = kEpiWarps * 32;
-  static constexpr int kThreads = (kEpiWarp0 + kEpiWarps + (FP8 ? 4 : 0)) * 32;
+  static constexpr int kConvWarps = FP8 ? 4 : 0;  // e4m3 -> f16 converter warps
+  static constexpr int kConvThreads = kConvWarps * 32;
+  static constexpr int kThreads = (kEpiWarp0 + kEpiWarps + kConvWarps) * 32;
   // smem layout offsets (from a 1024-aligned base)
   static constexpr int kOffStages = 0;
   static constexpr int kOffRaw = kOffStages + kStages * kTileBytes;
@@ -125,12 +128,12 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(&full[i], FP8 ? 128 : 1);
+      mbar_init(&full[i], FP8 ? C::kConvThreads : 1);
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < C::kRawStages; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_empty[i], 128);
+      mbar_init(&raw_empty[i], C::kConvThreads);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -138,7 +141,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     }
     mbar_init(q_ready, 1);
     mbar_init(mma_done, 1);
-    mbar_init(q_conv, 128);
+    mbar_init(q_conv, FP8 ? C::kConvThreads : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -286,6 +289,14 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       for (int sub = 0; sub < ng; ++sub, ++si) {
       const int acc = static_cast<int>(si & 1);
       const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
+      const int64_t s = static_cast<int64_t>(t) * kTileKeys + row;
+      // e4m3 keys: this key's scale, requested before the accumulator wait
+      // so that its latency is hidden behind it
+      float scale = 1.f;
+      if constexpr (FP8) {
+        const int64_t zb = a.per_query ? grp + sub : 0;
+        if (s < a.N) scale = __ldg(a.k_scale + zb * a.scale_batch_stride + s);
+      }
       got = mbar_wait(&acc_full[acc], aph, abort_flag, a.status, a.wait_ns);
       __syncwarp();  // tcgen05.ld below is warp-collective
       if (!got) break;
@@ -294,7 +305,6 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       const int b0 = (grp + sub) * a.G;
       const float* wsl = ws + sub * kMaxCols;
       const int64_t* nvsl = nvs + sub * 16;
-      const int64_t s = static_cast<int64_t>(t) * kTileKeys + row;
       // One half of the columns = a contiguous run of whole queries.
       auto tile_half = [&](auto half_c) {
         constexpr int H = decltype(half_c)::value;
@@ -410,11 +420,6 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&acc_empty[acc]);
         if (s < a.N) {
-          float scale = 1.f;
-          if constexpr (FP8) {
-            const int64_t zb = a.per_query ? grp + sub : 0;
-            scale = a.k_scale[zb * a.scale_batch_stride + s];
-          }
 #pragma unroll
           for (int g = 0; g < kQ; ++g) {
             const int gg = kQ0 + g;
@@ -446,7 +451,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     if (et == 0 && q_loads > 0) mbar_drain(q_ready, (q_loads - 1) & 1u);
   } else if constexpr (FP8) {
     // ------------------------------------------------------------ e4m3 -> f16
-    const int ct = threadIdx.x - (kEpiWarp0 + 4) * 32;  // 0..127
+    const int ct = threadIdx.x - (kEpiWarp0 + C::kEpiWarps) * 32;  // 0 .. kConvThreads - 1
     int64_t it = 0;
     int cur_grp = -1;
     uint32_t q_phase = 0;
@@ -461,7 +466,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         cur_grp = grp;
         constexpr int kRowChunks = 8;  // 16-byte chunks per 128-byte row
         const int nchunks = C::kBlocks * ncols * kRowChunks;
-        for (int i = ct; i < nchunks; i += 128) {
+        for (int i = ct; i < nchunks; i += C::kConvThreads) {
           const int bk = i / (ncols * kRowChunks), rem = i % (ncols * kRowChunks);
           uint4* pq = reinterpret_cast<uint4*>(qs + bk * (kMaxCols * 128) + rem * 16);
           const uint4 v = *pq;
@@ -487,24 +492,25 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       uint8_t* dst = stages + bs * C::kTileBytes;
       constexpr int kChunks16 = D_I / 16;  // 16-element e4m3 chunks per row
 #pragma unroll 2
-      for (int i = ct; i < kTileKeys * kChunks16; i += 128) {
+      for (int i = ct; i < kTileKeys * kChunks16; i += C::kConvThreads) {
         const int r = i / kChunks16, c = i % kChunks16;
         const uint4 in = *reinterpret_cast<const uint4*>(src + r * D_I + c * 16);
         const uint32_t w4[4] = {in.x, in.y, in.z, in.w};
         uint32_t o[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __half2_raw lo2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w4[j] & 0xFFFF), __NV_E4M3);
-          const __half2_raw hi2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w4[j] >> 16), __NV_E4M3);
-          o[2 * j] = static_cast<uint32_t>(lo2.x) | (static_cast<uint32_t>(lo2.y) << 16);
-          o[2 * j + 1] = static_cast<uint32_t>(hi2.x) | (static_cast<uint32_t>(hi2.y) << 16);
-        }
-        // 16 f16 = two 16-byte chunks: element offsets c*16 and c*16+8
+        for (int j = 0; j < 4; ++j) e4m3x4_to_f16x4(w4[j], o[2 * j], o[2 * j + 1]);
+        // 16 f16 = two 16-byte chunks: element offsets c*16 and c*16+8. The
+        // eight threads of a row write chunks 2(c%4) and 2(c%4)+1 of block
+        // c/4; the odd block's threads write their second chunk first, so
+        // each store instruction covers eight distinct chunk positions of a
+        // row (no bank conflicts).
         const int e0 = c * 16;
         const uint32_t base = smem_u32(dst + (e0 >> 6) * (kTileKeys * 128));
         const int ch = (e0 & 63) >> 3;
-        st_shared_v4(base + sw128_offset(r, ch), make_uint4(o[0], o[1], o[2], o[3]));
-        st_shared_v4(base + sw128_offset(r, ch + 1), make_uint4(o[4], o[5], o[6], o[7]));
+        const bool second_first = D_I == 128 && ((c >> 2) & 1);
+        const uint4 v0 = make_uint4(o[0], o[1], o[2], o[3]), v1 = make_uint4(o[4], o[5], o[6], o[7]);
+        st_shared_v4(base + sw128_offset(r, second_first ? ch + 1 : ch), second_first ? v1 : v0);
+        st_shared_v4(base + sw128_offset(r, second_first ? ch : ch + 1), second_first ? v0 : v1);
       }
       fence_proxy_async_smem();
       mbar_arrive(&raw_empty[rs]);

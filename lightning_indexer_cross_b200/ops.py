@@ -83,6 +83,34 @@ def indexer_score(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, k_scale: Op
     return scores
 
 
+def indexer_topk(q: torch.Tensor, w: torch.Tensor, k: torch.Tensor, topk: int,
+                 k_scale: Optional[torch.Tensor] = None, n_valid: Optional[torch.Tensor] = None,
+                 rows_per_pass: int = 0, idx: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The indexer and the top-k in one call: idx [B, topk] int32, the scores kept in a workspace scratch of
+    rows_per_pass rows (0 = all rows)."""
+    _need_cuda(q, w, k, k_scale, n_valid, idx)
+    _need_dense(q, w, n_valid, idx)
+    _need_dense_rows(k, k_scale)
+    B, H_I, d_I = q.shape
+    Bk, N, dk = k.shape
+    assert dk == d_I and Bk in (1, B) and q.dtype == torch.bfloat16 and w.dtype == torch.float32
+    fp8 = k.dtype == torch.uint8
+    assert k.dtype in (torch.bfloat16, torch.uint8)
+    assert k_scale is None or (fp8 and k_scale.dtype == torch.float32 and k_scale.shape == (Bk, N))
+    if idx is None:
+        idx = torch.empty((B, topk), dtype=torch.int32, device=q.device)
+    assert idx.shape == (B, topk) and idx.dtype == torch.int32
+    if workspace is None:
+        workspace = new_workspace(_abi.ic_indexer_topk_workspace_size(B, N, topk, rows_per_pass), q.device)
+    kbs = k.stride(0) if Bk > 1 else 0
+    sbs = k_scale.stride(0) if (k_scale is not None and k_scale.shape[0] > 1) else 0
+    _abi.ic_indexer_topk(_ptr(q), _ptr(w), _ptr(k), _ptr(k_scale), _abi.IC_FP8_E4M3 if fp8 else _abi.IC_BF16,
+                         B, H_I, d_I, N, kbs, sbs, _ptr(n_valid), topk, int(rows_per_pass), _ptr(idx),
+                         _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    return idx
+
+
 def topk(scores: torch.Tensor, k: int, n_valid: Optional[torch.Tensor] = None,
          idx: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     _need_cuda(scores, n_valid, idx)
@@ -265,7 +293,7 @@ class LayerStack:
                  k_fp8: bool = False, shared_keys: bool = True, shared_kv: bool = True,
                  n_valid: Optional[torch.Tensor] = None, sm_scale: Optional[float] = None,
                  out_dtype: torch.dtype = torch.bfloat16, trace: bool = False, device="cuda",
-                 want_lse: bool = False):
+                 want_lse: bool = False, rows_per_pass: int = 0):
         self.L = len(schedule)
         self.schedule = schedule.encode()
         self.layers = layers
@@ -287,6 +315,7 @@ class LayerStack:
         sh.scale_batch_stride = 0 if (shared_keys or B == 1 or first_f.k_scale is None) else first_f.k_scale.stride(0)
         sh.kv_batch_stride = 0 if (shared_kv or B == 1) else first_kv.stride(0)
         sh.n_valid = None if n_valid is None else n_valid.data_ptr()
+        sh.rows_per_pass = int(rows_per_pass)
         self.n_valid = n_valid
         self.shape = sh
         table = (_abi.ic_layer_t * self.L)()
@@ -327,8 +356,9 @@ class LayerStack:
         return _abi.ic_last_device_status(_ptr(self.ws), _stream_ptr(stream))
 
 
-def stack_from_workload(wl, trace: bool = False, out_dtype=torch.bfloat16, want_lse: bool = False) -> LayerStack:
+def stack_from_workload(wl, trace: bool = False, out_dtype=torch.bfloat16, want_lse: bool = False,
+                        rows_per_pass: int = 0) -> LayerStack:
     return LayerStack(wl.layers, wl.schedule, wl.B, wl.N, wl.H_I, wl.d_I, wl.topk, wl.H, k_fp8=wl.k_fp8,
                       shared_keys=wl.shared_keys, shared_kv=wl.shared_kv, n_valid=wl.n_valid,
                       sm_scale=wl.sm_scale, out_dtype=out_dtype, trace=trace,
-                      device=wl.layers[0].q.device, want_lse=want_lse)
+                      device=wl.layers[0].q.device, want_lse=want_lse, rows_per_pass=rows_per_pass)

@@ -109,6 +109,37 @@ def test_topk_deterministic_set(cuda_dev):
     assert torch.equal(a, b)
 
 
+# ------------------------------------------------------------------ indexer -> top-k in one call
+FUSED_CASES = [
+    # B, N, H_I, d_I, shared, fp8, causal, topk, rows per pass
+    (32, 20000, 64, 128, True, False, False, 2048, 0),
+    (32, 20000, 64, 128, True, False, False, 2048, 8),
+    (20, 9000, 64, 128, True, False, True, 512, 16),     # ragged last pass
+    (9, 30001, 64, 128, False, False, False, 1024, 4),    # per-query caches, passes of 8
+    (6, 12000, 64, 128, False, True, True, 700, 0),       # e4m3 keys
+    (6, 12000, 64, 128, False, True, False, 700, 3),
+    (3, 500, 16, 64, True, False, False, 2048, 0),        # fewer tokens than k
+]
+
+
+@pytest.mark.parametrize("B,N,H_I,d_I,shared,fp8,causal,k,rpp", FUSED_CASES)
+def test_indexer_topk_equals_the_two_calls_and_the_oracle(cuda_dev, B, N, H_I, d_I, shared, fp8, causal, k, rpp):
+    """ic_indexer_topk gives exactly the index sets of ic_indexer_score +
+    ic_topk (the scores are the same fp32 values, however the rows are
+    grouped into passes), and they match the oracle."""
+    ops = _ops()
+    q, w, kk, ks, nv = W.indexer_case(B, N, H_I, d_I, shared=shared, fp8=fp8, causal=causal, seed=B + N + k,
+                                      device=cuda_dev)
+    got = ops.indexer_topk(q, w, kk, k, ks, nv, rows_per_pass=rpp)
+    ref = ops.topk(ops.indexer_score(q, w, kk, ks, nv), k, nv)
+    torch.cuda.synchronize()
+    for b in range(B):
+        assert set(got[b].tolist()) == set(ref[b].tolist()), f"row {b}"
+    sc = oracle.indexer_scores(q, w, kk, ks, nv, keys_are_e4m3=fp8)
+    ok, msg = index_sets_match(got, oracle.topk_indices(sc, k, nv), sc, k, nv)
+    assert ok, msg
+
+
 # ------------------------------------------------------------------ sparse MLA
 MLA_CASES = [
     # B, N, H, k, shared, gate, n_invalid, out dtype
