@@ -146,9 +146,10 @@ namespace ic {
 uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 // ------------------------------------------------------------------ top-k
-TopkLayout topk_layout(int B, int64_t N) {
+TopkLayout topk_layout(int B, int64_t N, int k) {
   TopkLayout L{};
-  // one wave: two 512-thread CTAs per SM in total, at least 4096 scores per CTA
+  // the row's CTAs: about two 512-thread CTAs per SM in total, at least 4096
+  // scores per CTA
   const int64_t target = std::max<int64_t>(1, 2 * num_sms() / std::max(B, 1));
   int64_t cpr = std::min<int64_t>(ceil_div<int64_t>(N, 4096), target);
   cpr = std::max<int64_t>(cpr, 1);
@@ -157,26 +158,36 @@ TopkLayout topk_layout(int B, int64_t N) {
   cpr = ceil_div<int64_t>(N, slice);
   L.cpr = static_cast<int>(cpr);
   L.slice = slice;
+  L.mode = kTopkTwoPass;
   // one clustered launch per row (a cluster of c <= 4 CTAs, one per SM, each
   // holding up to 32768 scores) when the rows keep at least half of the SMs
   // busy; c grows while the grid still fits one wave
-  L.fused = 0;
   if ((N & 3) == 0 && N <= 4 * 32768) {
     int c = 1;
     while (c < 4 && ceil_div<int64_t>(N, c) > 32768) c *= 2;
     while (c < 4 && int64_t(B) * c * 2 <= num_sms() && ceil_div<int64_t>(N, c * 2) >= 4096) c *= 2;
     if (int64_t(B) * c * 2 >= num_sms()) {
-      L.fused = 1;
+      L.mode = kTopkCluster;
       L.cpr = c;
       L.slice = ceil_div<int64_t>(ceil_div<int64_t>(N, c), 4) * 4;
     }
   }
-  // the k-th key's 1/16-octave bin rarely holds more than a few percent of a
-  // row; bigger bins fall back to passes over the row itself
-  L.cand_cap = static_cast<int>(std::min<int64_t>(N, std::max<int64_t>(4096, N / 16)));
-  L.cnt_off = 0;  // control words and row histograms: zero between calls
+  // many rows, few CTAs per row (a prefill chunk): each CTA would pass over
+  // a large slice twice; one pass above a sampled threshold instead
+  if (L.mode == kTopkTwoPass && L.cpr <= 4) L.mode = kTopkThreshold;
+  L.fused = L.mode == kTopkCluster ? 1 : 0;
+  L.cnt_off = 0;  // control words (and row histograms): zero between calls
   L.hist_off = align256(L.cnt_off + size_t(B) * ic::kCtrlWords * 4);
-  L.cand_off = align256(L.hist_off + size_t(B) * 4096 * 4);
+  if (L.mode == kTopkThreshold) {
+    // candidates above the threshold: twice the expected 2k per row
+    L.cand_cap = static_cast<int>(std::min<int64_t>(N, std::max<int64_t>(8192, 4 * int64_t(std::max(k, 1)))));
+    L.cand_off = L.hist_off;  // no row histograms
+  } else {
+    // the k-th key's 1/16-octave bin rarely holds more than a few percent of
+    // a row; bigger bins fall back to passes over the row itself
+    L.cand_cap = static_cast<int>(std::min<int64_t>(N, std::max<int64_t>(4096, N / 16)));
+    L.cand_off = align256(L.hist_off + size_t(B) * 4096 * 4);
+  }
   L.zero_bytes = L.cand_off;
   L.ckey_off = align256(L.cand_off + size_t(B) * L.cand_cap * 4);
   L.total = align256(L.ckey_off + size_t(B) * L.cand_cap * 4);
@@ -188,7 +199,7 @@ ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_va
   if (!scores || !idx || !ws) return IC_ERR_INVALID_ARG;
   if (B < 1 || N < 1 || N >= (int64_t(1) << 31) || k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
   if (!aligned16(scores) || !aligned16(idx)) return IC_ERR_INVALID_ARG;
-  TopkLayout L = topk_layout(B, N);
+  TopkLayout L = topk_layout(B, N, k);
   if (ws_bytes < L.total) return IC_ERR_INVALID_ARG;
   ic::TopkArgs a{};
   a.scores = scores;
@@ -207,7 +218,8 @@ ic_status_t topk_impl(const float* scores, int B, int64_t N, const int64_t* n_va
   a.slice = L.slice;
   a.fused = L.fused;
   int launches = 0;
-  cudaError_t e = ic::launch_topk(a, stream, pdl, &launches);
+  cudaError_t e = L.mode == kTopkThreshold ? ic::launch_topk_threshold(a, stream, pdl, &launches)
+                                            : ic::launch_topk(a, stream, pdl, &launches);
   if (e != cudaSuccess) return IC_ERR_CUDA;
   g_launches += launches;
   return IC_OK;
@@ -237,10 +249,10 @@ struct FusedLayout {
   TopkLayout tk;
 };
 
-FusedLayout fused_layout(int B, int64_t N, int rows_per_pass) {
+FusedLayout fused_layout(int B, int64_t N, int topk, int rows_per_pass) {
   FusedLayout L{};
   L.R = fused_rows(B, rows_per_pass);
-  L.tk = topk_layout(L.R, N);
+  L.tk = topk_layout(L.R, N, topk);
   L.scores_off = 0;
   L.topk_off = align256(size_t(L.R) * N * 4);
   L.total = align256(L.topk_off + L.tk.total);
@@ -257,7 +269,7 @@ ic_status_t indexer_topk_impl(const void* q, const float* w, const void* k, cons
                               size_t region_bytes, int* status, cudaStream_t stream, bool pdl, int* launches) {
   if (!q || !w || !k || !idx || !region) return IC_ERR_INVALID_ARG;
   if (B < 1 || N < 1 || H_I < 1 || topk < 1) return IC_ERR_INVALID_ARG;
-  const FusedLayout L = fused_layout(B, N, rows_per_pass);
+  const FusedLayout L = fused_layout(B, N, topk, rows_per_pass);
   if (region_bytes < L.total || !aligned16(region)) return IC_ERR_INVALID_ARG;
   const bool fp8 = k_dtype == IC_FP8_E4M3;
   const int64_t esz = fp8 ? 1 : 2;
@@ -398,7 +410,7 @@ struct StackLayout {
 
 StackLayout stack_layout(const ic_stack_shape_t& s) {
   StackLayout L{};
-  L.fz = fused_layout(s.B, s.N, s.rows_per_pass);
+  L.fz = fused_layout(s.B, s.N, s.topk, s.rows_per_pass);
   L.ml = mla_layout(s.B, s.H, s.topk);
   L.fused_off = kStatusBytes;
   L.mla_off = align256(L.fused_off + L.fz.total);
@@ -441,9 +453,8 @@ ic_status_t ic_indexer_score(const void* q, const float* w, const void* k, const
 }
 
 size_t ic_topk_workspace_size(int B, int64_t N, int k) {
-  (void)k;
   if (B < 1 || N < 1) return kStatusBytes;
-  return kStatusBytes + topk_layout(B, N).total;
+  return kStatusBytes + topk_layout(B, N, k).total;
 }
 
 ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_valid, int k, int32_t* idx,
@@ -456,9 +467,8 @@ ic_status_t ic_topk(const float* scores, int B, int64_t N, const int64_t* n_vali
 }
 
 size_t ic_indexer_topk_workspace_size(int B, int64_t N, int k, int rows_per_pass) {
-  (void)k;
   if (B < 1 || N < 1) return kStatusBytes;
-  return kStatusBytes + fused_layout(B, N, rows_per_pass).total;
+  return kStatusBytes + fused_layout(B, N, k, rows_per_pass).total;
 }
 
 ic_status_t ic_indexer_topk(const void* q, const float* w, const void* k, const float* k_scale, ic_dtype_t k_dtype,

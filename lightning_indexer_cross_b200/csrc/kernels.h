@@ -121,18 +121,24 @@ struct TopkArgs {
   int fused;                // one clustered launch per row (cpr CTAs = one cluster) instead of two
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream, bool pdl, int* launches);
+// The one-pass form: a sampled threshold, then one filter pass whose last
+// CTA per row selects among the candidates (uses counters, cand, cand_key,
+// cand_cap, cpr, slice; counters zero between calls).
+cudaError_t launch_topk_threshold(const TopkArgs& a, cudaStream_t stream, bool pdl, int* launches);
 
 // Scratch layout of the top-k passes for B rows of N scores (byte offsets
 // from the start of the scratch region, which follows the status word).
+enum TopkMode : int { kTopkCluster = 0, kTopkTwoPass = 1, kTopkThreshold = 2 };
 struct TopkLayout {
   int cpr;         // CTAs per row
   int64_t slice;   // scores per CTA
+  int mode;        // which kernels run (TopkMode)
   int fused;       // one clustered launch (cpr <= 4, slices <= 32768 scores)
   int cand_cap;
   size_t hist_off, cand_off, ckey_off, cnt_off, total;
   size_t zero_bytes;  // [0, zero_bytes): control words and row histograms, zero between calls
 };
-TopkLayout topk_layout(int B, int64_t N);
+TopkLayout topk_layout(int B, int64_t N, int k);
 // Validate and enqueue the top-k passes. The control words and row
 // histograms ([0, zero_bytes)) must be zero on entry; every call that
 // completes leaves them zero again.

@@ -71,7 +71,7 @@ extern "C" ic_status_t ic_topk_noalloc(const float* scores, int B, int64_t N, co
   if (!scores || !idx) return IC_ERR_INVALID_ARG;
   if (B < 1 || N < 1 || N >= (int64_t(1) << 31) || k < 1 || k > 16384) return IC_ERR_INVALID_ARG;
   if (B > IC_TOPK_NOALLOC_MAX_ROWS) return IC_ERR_UNSUPPORTED;
-  const ic::TopkLayout L = ic::topk_layout(B, N);
+  const ic::TopkLayout L = ic::topk_layout(B, N, k);
   if (kStatusBytes + L.total > kScratchBytes) return IC_ERR_UNSUPPORTED;
   void* base = nullptr;
   if (scratch_address(&base) != cudaSuccess) return IC_ERR_CUDA;

@@ -73,9 +73,10 @@ def test_topk_rejects_bad_arguments(abi):
     assert call(k=0) == abi.IC_ERR_INVALID_ARG
     assert call(k=20000) == abi.IC_ERR_INVALID_ARG
     assert call(s=None) == abi.IC_ERR_INVALID_ARG
-    assert call(wsb=300) == abi.IC_ERR_INVALID_ARG  # too small for the histograms
+    assert call(wsb=300) == abi.IC_ERR_INVALID_ARG  # too small for the candidate buffers
     need = abi.ic_topk_workspace_size(2, 1000, 64)
-    assert need >= 2 * 4096 * 4  # per-row 12-bit histograms at least
+    assert need >= 2 * 1000 * 8  # a candidate buffer (position, key) per row, here the whole row
+    assert call(wsb=need - 256 - 1) == abi.IC_ERR_INVALID_ARG
 
 
 def test_sparse_mla_rejects_bad_arguments(abi):

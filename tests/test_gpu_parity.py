@@ -73,6 +73,11 @@ TOPK_CASES = [
     (40, 20000, 2048, False, 0.0, True),      # two-CTA clusters, causal rows
     (24, 131072, 2048, True, 0.3, False),     # four-CTA clusters, heavy ties, -inf
     (20, 131072, 1, False, 0.0, False),
+    # many rows, few CTAs per row: one pass above a sampled threshold
+    (80, 200000, 2048, False, 0.0, False),    # sampled threshold, candidates in shared memory
+    (100, 12001, 1000, False, 0.0, True),     # whole row read for the threshold; causal short rows
+    (90, 150001, 300, True, 0.3, False),      # heavy ties: the threshold bin overflows the buffer
+    (160, 150000, 4096, False, 0.0, False),   # k = 4096: candidates selected from global memory
 ]
 
 
@@ -92,6 +97,36 @@ def test_topk_is_exact(cuda_dev, B, N, k, ties, ninf, causal):
     for b in range(B):
         assert set(gi[b][gi[b] >= 0].tolist()) == set(ref[b][ref[b] >= 0].tolist()), f"row {b}"
         assert (gi[b] == -1).sum() == (ref[b] == -1).sum()
+
+
+@pytest.mark.parametrize("N", [150000, 300000])
+def test_topk_exact_when_the_sampled_threshold_misses(cuda_dev, N):
+    """With many rows the top-k takes its threshold from a sample of each
+    row: 256 blocks of 32 consecutive scores, block j picked inside stretch j
+    of the row by a multiplicative hash of j. Row 0 holds its 400 largest
+    scores at sampled positions and nothing else stands out, so the
+    threshold lands among them and fewer than k keys reach it: the selection
+    falls back to the whole row and must still be exact. Row 1 plants them
+    away from the sample (the ordinary path); the other rows are random."""
+    B, k = 80, 2048
+    s = W.scores_case(B, N, seed=N, device=cuda_dev)
+    blocks = N // 32
+    starts = []
+    for j in range(256):
+        b0, b1 = j * blocks // 256, (j + 1) * blocks // 256
+        h = ((j + 1) * 2654435761) & 0xFFFFFFFF
+        starts.append((b0 + (h >> 8) % (b1 - b0)) * 32)
+    sampled = torch.cat([torch.arange(32, device=cuda_dev) + st for st in starts])
+    pick = sampled[torch.randperm(sampled.numel(), device=cuda_dev)[:400]]
+    s[0, pick] = 100.0 + torch.rand(400, device=cuda_dev)
+    away = (sampled[:400] + 16 * 32 + 7) % N
+    s[1, away] = 100.0 + torch.rand(400, device=cuda_dev)
+    idx = _ops().topk(s, k)
+    torch.cuda.synchronize()
+    ref = oracle.topk_indices(s, k)
+    for b in range(B):
+        assert set(idx[b].tolist()) == set(ref[b].tolist()), f"row {b}"
+    assert set(pick.tolist()) <= set(idx[0].tolist())
 
 
 def test_topk_all_equal_scores_take_lowest_indices(cuda_dev):
