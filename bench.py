@@ -385,14 +385,155 @@ def run_native(args):
     return 0
 
 
+# ----------------------------------------------------------------------------- ncu summaries
+# Helpers for the committed profile notes (profiles/*.md): a per-kernel
+# summary of an ncu launch list, and the DRAM traffic per launch of a kernel
+# family recorded with the SHA-256 of its sources, which load_traffic reads
+# back only while the sources are unchanged.
+_NCU_UNIT = {"nsecond": 1e-3, "ns": 1e-3, "usecond": 1.0, "us": 1.0, "msecond": 1e3, "ms": 1e3, "second": 1e6}
+
+
+def _ncu_rows(path):
+    import csv
+    rows = list(csv.reader(open(path)))
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    return rows[hi], rows[hi + 1:]
+
+
+def _ncu_name(k):
+    return k.split("(")[0].replace("void ", "").replace("(anonymous namespace)::", "")
+
+
+def ncu_launches(path):
+    """Per kernel of a gpu__time_duration.sum launch list: launches, total
+    time, mean and share."""
+    import collections
+    h, body = _ncu_rows(path)
+    ki, mi, vi, ui = (h.index(x) for x in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit"))
+    agg = collections.defaultdict(lambda: [0, 0.0])
+    for r in body:
+        if len(r) <= vi or r[mi] != "gpu__time_duration.sum":
+            continue
+        name = _ncu_name(r[ki])
+        agg[name][0] += 1
+        agg[name][1] += float(r[vi].replace(",", "")) * _NCU_UNIT.get(r[ui], 1e-3)
+    tot = sum(t for _, t in agg.values())
+    print(f"{'kernel':58s} {'launches':>8s} {'total_us':>11s} {'mean_us':>9s} {'share':>6s}")
+    for k, (n, t) in sorted(agg.items(), key=lambda x: -x[1][1]):
+        print(f"{k[:58]:58s} {n:8d} {t:11.1f} {t / n:9.2f} {t / tot:6.3f}")
+
+
+def sources_sha256(paths):
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()
+
+
+def ncu_traffic(path, name, regex, sources):
+    """DRAM bytes (read + write) of one launch of each kernel matching regex,
+    summed, as the traffic block load_traffic reads."""
+    import collections
+    import re
+    h, body = _ncu_rows(path)
+    ki, ii, mi, vi = (h.index(x) for x in ("Kernel Name", "ID", "Metric Name", "Metric Value"))
+    per = collections.defaultdict(dict)
+    kern = {}
+    for r in body:
+        if len(r) <= vi or not re.search(regex, r[ki]):
+            continue
+        per[r[ii]][r[mi]] = float(r[vi].replace(",", ""))
+        kern[r[ii]] = _ncu_name(r[ki])
+    first = {}
+    for lid in sorted(per, key=int):
+        first.setdefault(kern[lid], per[lid])
+    total = sum(m.get("dram__bytes_read.sum", 0.0) + m.get("dram__bytes_write.sum", 0.0) for m in first.values())
+    print(f"traffic-kernel: {name}")
+    print(f"traffic-sources: {' '.join(sources)}")
+    print(f"traffic-sha256: {sources_sha256(sources)}")
+    print(f"traffic-dram-bytes-per-launch: {int(total)}")
+    for k, m in first.items():
+        print(f"traffic-part: {k} read {int(m.get('dram__bytes_read.sum', 0))} write "
+              f"{int(m.get('dram__bytes_write.sum', 0))}")
+
+
 def load_traffic(kernel):
     """DRAM bytes per launch from the committed ncu summary under profiles/,
     if one was taken on the current kernel sources; else None."""
-    from lightning_indexer_cross_b200.ncu_summary import read_traffic
-    try:
-        return read_traffic(kernel, os.path.join(ROOT, "profiles"))
-    except Exception:
+    import re
+    pdir = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(pdir):
         return None
+    for fn in sorted(os.listdir(pdir)):
+        if not fn.endswith(".md"):
+            continue
+        kv = dict(re.findall(r"^traffic-([a-z0-9-]+):\s*(.+)$", open(os.path.join(pdir, fn)).read(), flags=re.M))
+        if kv.get("kernel") != kernel or "dram-bytes-per-launch" not in kv:
+            continue
+        try:
+            if sources_sha256(kv["sources"].split()) != kv["sha256"].strip():
+                continue
+        except OSError:
+            continue
+        return int(kv["dram-bytes-per-launch"])
+    return None
+
+
+# ----------------------------------------------------------------------------- one kernel family, for profiling
+DRIVER_SHAPES = {
+    "stack": dict(B=32, N=131072, shared=True),     # one layer of the 78-layer stack
+    "single": dict(B=8, N=131072, shared=False),    # the single F layer, per-query caches
+    "long": dict(B=4, N=262144, shared=False),      # the long-context shape at a quarter of its length
+    "prefill": dict(B=256, N=264192, shared=True),  # 256 rows of the prefill chunk
+}
+
+
+def kernel_driver(kernel, shape, fp8, warmup, iters):
+    """Run one kernel family on a fixed shape: `warmup` untimed launches,
+    then `iters` timed ones (for ncu -k <kernel> -s <warm-up launches>)."""
+    import torch
+    from lightning_indexer_cross_b200 import _abi, ops
+    from lightning_indexer_cross_b200 import workloads as W
+    sh = DRIVER_SHAPES[shape]
+    dev = torch.device("cuda:0")
+    Bq, Nk, shared = sh["B"], sh["N"], sh["shared"]
+    K = TOPK
+    if kernel == "gate":
+        o, wv, gl = W.gate_case(Bq, H, seed=90, device=dev)
+        ws = ops.new_workspace(_abi.ic_decompress_gate_workspace_size(), dev)
+        fn = lambda: ops.decompress_gate(o, wv, gl, workspace=ws)
+    else:
+        q, w, k, ks, _ = W.indexer_case(Bq, Nk, H_I, D_I, shared=shared, fp8=fp8, seed=5, device=dev)
+        scores = ops.indexer_score(q, w, k, ks)
+        idx = ops.topk(scores, K)
+        torch.cuda.synchronize()
+        if kernel == "indexer":
+            ws = ops.new_workspace(256, dev)
+            fn = lambda: ops.indexer_score(q, w, k, ks, scores=scores, workspace=ws)
+        elif kernel == "topk":
+            ws = ops.new_workspace(_abi.ic_topk_workspace_size(Bq, Nk, K), dev)
+            fn = lambda: ops.topk(scores, K, idx=idx, workspace=ws)
+        else:
+            g = torch.Generator(device=dev).manual_seed(6)
+            qa = torch.randn((Bq, H, W.D_QK), generator=g, device=dev).to(torch.bfloat16)
+            kv = torch.randn((1 if shared else Bq, Nk, W.D_QK), generator=g, device=dev).to(torch.bfloat16)
+            sink = torch.randn((H,), generator=g, device=dev) * 0.5
+            gate = torch.randn((Bq, H, W.D_LATENT), generator=g, device=dev).to(torch.bfloat16)
+            out = torch.empty((Bq, H, W.D_LATENT), dtype=torch.bfloat16, device=dev)
+            ws = ops.new_workspace(_abi.ic_sparse_mla_workspace_size(Bq, H, K), dev)
+            fn = lambda: ops.sparse_mla_decode(qa, kv, idx, sink, gate, out=out, want_lse=False, workspace=ws)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    print(f"{kernel} {shape}{' fp8' if fp8 else ''}: {e0.elapsed_time(e1) * 1000 / max(iters, 1):.2f} us/call")
+    return 0
 
 
 def _time_loop(fn, n, stream, replays=3):
@@ -778,7 +919,22 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip timing the other workloads' kernels")
     ap.add_argument("--warmup-ref", type=int, default=1)
+    ap.add_argument("--kernel-driver", choices=["indexer", "topk", "mla", "gate"],
+                    help="run one kernel family on --shape instead (for ncu): --warmup untimed, --steps timed")
+    ap.add_argument("--shape", choices=list(DRIVER_SHAPES), default="stack")
+    ap.add_argument("--fp8", action="store_true", help="e4m3 keys for --kernel-driver")
+    ap.add_argument("--ncu-launches", metavar="CSV", help="summarise an ncu launch list and exit")
+    ap.add_argument("--ncu-traffic", nargs="+", metavar="ARG",
+                    help="CSV NAME REGEX SOURCE...: the DRAM traffic block of a kernel family, then exit")
     args = ap.parse_args()
+    if args.ncu_launches:
+        ncu_launches(args.ncu_launches)
+        return 0
+    if args.ncu_traffic:
+        ncu_traffic(args.ncu_traffic[0], args.ncu_traffic[1], args.ncu_traffic[2], args.ncu_traffic[3:])
+        return 0
+    if args.kernel_driver:
+        return kernel_driver(args.kernel_driver, args.shape, args.fp8, args.warmup, args.steps)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
