@@ -129,6 +129,10 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   const int64_t groups = ceil_div<int64_t>(B, a.G);
   a.groups = static_cast<int>(groups);
   a.pair = (!fp8 && !per_query && groups >= 2) ? 2 : 1;
+  // one group's heads fill at most half of the accumulator: two key tiles per
+  // item, so that both halves of the epilogue reduce
+  a.dual = (a.pair == 1 && a.G * HP <= 128) ? 1 : 0;
+  if (a.dual) a.tiles = static_cast<int>(ceil_div<int64_t>(a.tiles, 2));
   a.total_items = ceil_div<int64_t>(groups, a.pair) * a.tiles;
   a.per_query = per_query ? 1 : 0;
   a.wait_ns = ic::wait_limit_ns();

@@ -88,12 +88,18 @@ struct IdxCfg {
   static_assert(kSmemBytes <= 232448, "fits one CTA per SM");
 };
 
-template <int D_I, int HP, bool FP8, bool PAIR>
+// DUAL: the group's heads fill at most half of the accumulator columns
+// (n <= 128, one group per tile), so a work item takes two consecutive key
+// tiles: the first accumulates into columns [0, n), the second into
+// [128, 128 + n), and each half of the epilogue warps reduces one tile.
+template <int D_I, int HP, bool FP8, bool PAIR, bool DUAL>
 __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                       const IndexerArgs a) {
   using C = IdxCfg<D_I, FP8, PAIR>;
+  static_assert(!(DUAL && PAIR), "two tiles per item take one query group");
   constexpr int P = C::kQSlots;  // query groups per work item
+  constexpr int TPI = DUAL ? 2 : 1;  // key tiles per work item
   constexpr int GMAX = kMaxCols / HP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -120,7 +126,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   pdl_trigger();
 
   // This CTA's contiguous share of the work list: item (pair, tile) covers
-  // query groups P pair .. P pair + P - 1 (fewer at the end) on one key tile.
+  // query groups P pair .. P pair + P - 1 (fewer at the end) on one key tile
+  // (DUAL: item (group, j) covers one group on key tiles 2j and 2j + 1).
   const int64_t total = a.total_items;
   const int64_t lo = total * blockIdx.x / gridDim.x;
   const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
@@ -162,33 +169,37 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int64_t it = 0;
-      for (int64_t wi = lo; wi < hi; ++wi, ++it) {
+      int64_t jt = 0;  // key tiles loaded (the stage sequence)
+      bool ok = true;
+      for (int64_t wi = lo; wi < hi && ok; ++wi) {
         const int grp = static_cast<int>(wi / a.tiles) * P;  // first group of the item
-        const int t = static_cast<int>(wi % a.tiles);
+        const int t0 = static_cast<int>(wi % a.tiles) * TPI;
         const int z = a.per_query ? grp : 0;
-        if constexpr (!FP8) {
-          const int st = static_cast<int>(it % C::kStages);
-          const uint32_t ph = static_cast<uint32_t>((it / C::kStages) & 1);
-          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
-          mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+        // (a second tile past the end reads as zeros; its scores are not stored)
+        for (int h = 0; h < TPI; ++h, ++jt) {
+          if constexpr (!FP8) {
+            const int st = static_cast<int>(jt % C::kStages);
+            const uint32_t ph = static_cast<uint32_t>((jt / C::kStages) & 1);
+            if (!mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+            mbar_arrive_expect_tx(&full[st], C::kTileBytes);
 #pragma unroll
-          for (int bk = 0; bk < C::kBlocks; ++bk)
-            tma_load_3d(stages + st * C::kTileBytes + bk * (kTileKeys * 128), &kmap, &full[st], bk * 64,
-                        t * kTileKeys, z);
-        } else {
-          const int st = static_cast<int>(it % C::kRawStages);
-          const uint32_t ph = static_cast<uint32_t>((it / C::kRawStages) & 1);
-          if (!mbar_wait(&raw_empty[st], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
-          mbar_arrive_expect_tx(&raw_full[st], C::kRawBytes);
-          tma_load_3d(raw + st * C::kRawBytes, &kmap, &raw_full[st], 0, t * kTileKeys, z);
+            for (int bk = 0; bk < C::kBlocks; ++bk)
+              tma_load_3d(stages + st * C::kTileBytes + bk * (kTileKeys * 128), &kmap, &full[st], bk * 64,
+                          (t0 + h) * kTileKeys, z);
+          } else {
+            const int st = static_cast<int>(jt % C::kRawStages);
+            const uint32_t ph = static_cast<uint32_t>((jt / C::kRawStages) & 1);
+            if (!mbar_wait(&raw_empty[st], ph ^ 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+            mbar_arrive_expect_tx(&raw_full[st], C::kRawBytes);
+            tma_load_3d(raw + st * C::kRawBytes, &kmap, &raw_full[st], 0, (t0 + h) * kTileKeys, z);
+          }
         }
       }
       if (*abort_flag) {
         // wind down: let every load this thread issued land before exiting
         const int S = FP8 ? C::kRawStages : C::kStages;
         uint64_t* fb = FP8 ? raw_full : full;
-        const int64_t issued = it;  // loads actually issued before the abort
+        const int64_t issued = jt;  // loads actually issued before the abort
         for (int64_t j = (issued > S ? issued - S : 0); j < issued; ++j)
           mbar_drain(&fb[j % S], static_cast<uint32_t>((j / S) & 1));
       }
@@ -202,6 +213,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       int cur_grp = -1;
       uint32_t q_phase = 0;
       int64_t it = 0, si = 0;  // items; (item, group) sub-items -> accumulator si & 1
+      int64_t jt = 0;          // key tiles consumed (the stage sequence)
       bool ok = true;
       for (int64_t wi = lo; wi < hi && ok; ++wi, ++it) {
         const int grp = static_cast<int>(wi / a.tiles) * P;
@@ -211,8 +223,36 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
           q_phase ^= 1;
           cur_grp = grp;
         }
-        const int st = static_cast<int>(it % C::kStages);
-        const uint32_t ph = static_cast<uint32_t>((it / C::kStages) & 1);
+        if constexpr (DUAL) {
+          // one accumulator, two key tiles: columns [0, n) and [128, 128 + n)
+          const int acc = static_cast<int>(si & 1);
+          const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
+          if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status, a.wait_ns)) break;
+          tc_fence_after();
+          for (int h = 0; h < 2 && ok; ++h, ++jt) {
+            const int st = static_cast<int>(jt % C::kStages);
+            const uint32_t ph = static_cast<uint32_t>((jt / C::kStages) & 1);
+            if (!mbar_wait(&full[st], ph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(stages + st * C::kTileBytes);
+            const uint32_t d_tmem = tmem_base + acc * 256 + h * 128;
+#pragma unroll
+            for (int kk = 0; kk < D_I / 16; ++kk) {
+              const uint32_t koff = (kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32;
+              const uint32_t qoff = (kk >> 2) * (kMaxCols * 128) + (kk & 3) * 32;
+              mma_bf16_ss(d_tmem, sw128_desc(a_addr + koff, 16, 1024), sw128_desc(q_addr + qoff, 16, 1024), idesc,
+                          kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&empty[st]);
+          }
+          if (!ok) break;
+          mma_commit(&acc_full[acc]);
+          ++si;
+          continue;
+        }
+        const int st = static_cast<int>(jt % C::kStages);
+        const uint32_t ph = static_cast<uint32_t>((jt / C::kStages) & 1);
+        ++jt;
         if (!mbar_wait(&full[st], ph, abort_flag, a.status, a.wait_ns)) break;
         const uint32_t a_addr = smem_u32(stages + st * C::kTileBytes);
         for (int sub = 0; sub < ng; ++sub, ++si) {
@@ -275,7 +315,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
           const int b0 = (grp + slot) * a.G;
           float* wslot = ws + slot * kMaxCols;
           for (int i = et; i < kMaxCols; i += kNumEpiThreads) {
-            const int g = i / HP, h = i % HP, b = b0 + g;
+            const int ii = DUAL ? (i & 127) : i;  // (DUAL: both halves hold the group's heads)
+            const int g = ii / HP, h = ii % HP, b = b0 + g;
             wslot[i] = (g < a.G && h < a.H_I && b < a.B) ? a.w[static_cast<int64_t>(b) * a.H_I + h] : 0.f;
           }
           if (et < GMAX) {
@@ -289,7 +330,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       for (int sub = 0; sub < ng; ++sub, ++si) {
       const int acc = static_cast<int>(si & 1);
       const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
-      const int64_t s = static_cast<int64_t>(t) * kTileKeys + row;
+      // (DUAL: half h reduces key tile 2 t + h)
+      const int64_t s = static_cast<int64_t>(DUAL ? 2 * t + half : t) * kTileKeys + row;
       // e4m3 keys: this key's scale, requested before the accumulator wait
       // so that its latency is hidden behind it
       float scale = 1.f;
@@ -308,6 +350,8 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       // One half of the columns = a contiguous run of whole queries.
       auto tile_half = [&](auto half_c) {
         constexpr int H = decltype(half_c)::value;
+        // last column of this half's accumulator that the MMAs wrote
+        const int lim = DUAL ? H * 128 + ncols : ncols;
         constexpr int kChunks = kMaxCols / 32 / C::kHalves;  // 32-column chunks of this half
         constexpr int kC0 = H * kChunks;
         constexpr int kQ = GMAX / C::kHalves;                 // queries of this half
@@ -365,7 +409,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         };
         if constexpr (kPerWait == 1) {
           const int c0 = kC0 * 32;
-          if (c0 + kChunks * 32 <= ncols) {
+          if (c0 + kChunks * 32 <= lim) {
             // every column of the half is present: 64-column TMEM loads, the
             // next one in flight while the current one is reduced
             uint32_t ra[64], rb[64];
@@ -387,7 +431,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
 #pragma unroll
             for (int pass = 0; pass < kLoads; ++pass) {
               const int cA = c0 + 64 * pass;
-              if (cA < ncols) {
+              if (cA < lim) {
                 uint32_t ra[64];
                 tmem_ld64_issue(taddr + cA, ra);
                 tmem_ld_wait64(ra);
@@ -401,7 +445,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
 #pragma unroll
           for (int pass = 0; pass < kLoads; pass += 2) {
             const int cA = (kC0 + 2 * pass) * 32, cB = cA + 64;
-            const bool haveA = cA < ncols, haveB = cB < ncols && pass + 1 < kLoads;
+            const bool haveA = cA < lim, haveB = cB < lim && pass + 1 < kLoads;
             uint32_t ra[64], rb[64];
             if (haveA) tmem_ld64_issue(taddr + cA, ra);
             if (haveB) tmem_ld64_issue(taddr + cB, rb);
@@ -422,7 +466,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         if (s < a.N) {
 #pragma unroll
           for (int g = 0; g < kQ; ++g) {
-            const int gg = kQ0 + g;
+            const int gg = DUAL ? g : kQ0 + g;  // (DUAL: both halves hold the same queries)
             if (gg < a.G && b0 + gg < a.B) {
               float tot = 0.f;
               if constexpr (kPacked) {
@@ -452,10 +496,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   } else if constexpr (FP8) {
     // ------------------------------------------------------------ e4m3 -> f16
     const int ct = threadIdx.x - (kEpiWarp0 + C::kEpiWarps) * 32;  // 0 .. kConvThreads - 1
-    int64_t it = 0;
+    int64_t jt = 0;  // key tiles converted (the stage sequence)
     int cur_grp = -1;
     uint32_t q_phase = 0;
-    for (int64_t wi = lo; wi < hi; ++wi, ++it) {
+    bool ok = true;
+    for (int64_t wi = lo; wi < hi && ok; ++wi) {
       const int grp = static_cast<int>(wi / a.tiles) * P;
       if (grp != cur_grp) {
         // the group's queries, staged as bf16 by TMA, become f16 in place
@@ -482,12 +527,13 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(q_conv);
       }
-      const int rs = static_cast<int>(it % C::kRawStages);
-      const uint32_t rph = static_cast<uint32_t>((it / C::kRawStages) & 1);
-      const int bs = static_cast<int>(it % C::kStages);
-      const uint32_t bph = static_cast<uint32_t>((it / C::kStages) & 1);
-      if (!mbar_wait(&raw_full[rs], rph, abort_flag, a.status, a.wait_ns)) break;
-      if (!mbar_wait(&empty[bs], bph ^ 1, abort_flag, a.status, a.wait_ns)) break;
+      for (int h = 0; h < TPI; ++h, ++jt) {
+      const int rs = static_cast<int>(jt % C::kRawStages);
+      const uint32_t rph = static_cast<uint32_t>((jt / C::kRawStages) & 1);
+      const int bs = static_cast<int>(jt % C::kStages);
+      const uint32_t bph = static_cast<uint32_t>((jt / C::kStages) & 1);
+      if (!mbar_wait(&raw_full[rs], rph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+      if (!mbar_wait(&empty[bs], bph ^ 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
       const uint8_t* src = raw + rs * C::kRawBytes;
       uint8_t* dst = stages + bs * C::kTileBytes;
       constexpr int kChunks16 = D_I / 16;  // 16-element e4m3 chunks per row
@@ -515,6 +561,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(&raw_empty[rs]);
       mbar_arrive(&full[bs]);
+      }
     }
   }
 
@@ -527,11 +574,11 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   }
 }
 
-template <int D_I, int HP, bool FP8, bool PAIR>
+template <int D_I, int HP, bool FP8, bool PAIR, bool DUAL>
 cudaError_t launch_indexer_inst(const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int grid,
                                 cudaStream_t stream, bool pdl) {
   using C = IdxCfg<D_I, FP8, PAIR>;
-  auto kern = indexer_tc_kernel<D_I, HP, FP8, PAIR>;
+  auto kern = indexer_tc_kernel<D_I, HP, FP8, PAIR, DUAL>;
   static bool done[64] = {false};  // one flag set per template instance
   cudaError_t e = set_smem_once(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
@@ -539,14 +586,14 @@ cudaError_t launch_indexer_inst(const CUtensorMap& map, const CUtensorMap& qmap,
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int D_I, bool FP8, bool PAIR>
+template <int D_I, bool FP8, bool PAIR, bool DUAL>
 cudaError_t dispatch_hp(int HP, const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int grid,
                         cudaStream_t s, bool pdl) {
   switch (HP) {
-    case 16: return launch_indexer_inst<D_I, 16, FP8, PAIR>(map, qmap, a, grid, s, pdl);
-    case 32: return launch_indexer_inst<D_I, 32, FP8, PAIR>(map, qmap, a, grid, s, pdl);
-    case 64: return launch_indexer_inst<D_I, 64, FP8, PAIR>(map, qmap, a, grid, s, pdl);
-    case 128: return launch_indexer_inst<D_I, 128, FP8, PAIR>(map, qmap, a, grid, s, pdl);
+    case 16: return launch_indexer_inst<D_I, 16, FP8, PAIR, DUAL>(map, qmap, a, grid, s, pdl);
+    case 32: return launch_indexer_inst<D_I, 32, FP8, PAIR, DUAL>(map, qmap, a, grid, s, pdl);
+    case 64: return launch_indexer_inst<D_I, 64, FP8, PAIR, DUAL>(map, qmap, a, grid, s, pdl);
+    case 128: return launch_indexer_inst<D_I, 128, FP8, PAIR, DUAL>(map, qmap, a, grid, s, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -560,18 +607,23 @@ int indexer_smem_bytes(int d_I, bool fp8) {
 
 cudaError_t launch_indexer(const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int HP, int d_I,
                            bool fp8, int grid, cudaStream_t stream, bool pdl) {
+  const bool dual = a.dual != 0;
   if (fp8) {
-    if (d_I == 64) return dispatch_hp<64, true, false>(HP, map, qmap, a, grid, stream, pdl);
-    if (d_I == 128) return dispatch_hp<128, true, false>(HP, map, qmap, a, grid, stream, pdl);
+    if (d_I == 64) return dual ? dispatch_hp<64, true, false, true>(HP, map, qmap, a, grid, stream, pdl)
+                               : dispatch_hp<64, true, false, false>(HP, map, qmap, a, grid, stream, pdl);
+    if (d_I == 128) return dual ? dispatch_hp<128, true, false, true>(HP, map, qmap, a, grid, stream, pdl)
+                                : dispatch_hp<128, true, false, false>(HP, map, qmap, a, grid, stream, pdl);
     return cudaErrorInvalidValue;
   }
   if (a.pair == 2) {
-    if (d_I == 64) return dispatch_hp<64, false, true>(HP, map, qmap, a, grid, stream, pdl);
-    if (d_I == 128) return dispatch_hp<128, false, true>(HP, map, qmap, a, grid, stream, pdl);
+    if (d_I == 64) return dispatch_hp<64, false, true, false>(HP, map, qmap, a, grid, stream, pdl);
+    if (d_I == 128) return dispatch_hp<128, false, true, false>(HP, map, qmap, a, grid, stream, pdl);
     return cudaErrorInvalidValue;
   }
-  if (d_I == 64) return dispatch_hp<64, false, false>(HP, map, qmap, a, grid, stream, pdl);
-  if (d_I == 128) return dispatch_hp<128, false, false>(HP, map, qmap, a, grid, stream, pdl);
+  if (d_I == 64) return dual ? dispatch_hp<64, false, false, true>(HP, map, qmap, a, grid, stream, pdl)
+                             : dispatch_hp<64, false, false, false>(HP, map, qmap, a, grid, stream, pdl);
+  if (d_I == 128) return dual ? dispatch_hp<128, false, false, true>(HP, map, qmap, a, grid, stream, pdl)
+                              : dispatch_hp<128, false, false, false>(HP, map, qmap, a, grid, stream, pdl);
   return cudaErrorInvalidValue;
 }
 

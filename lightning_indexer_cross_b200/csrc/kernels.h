@@ -90,6 +90,8 @@ struct IndexerArgs {
   int pair;           // groups per work item: 2 (one cache shared by all queries, >= 2 groups) or 1
   int64_t total_items;  // ceil(groups / pair) * tiles
   int per_query;      // 1: key cache z-coordinate = group (G == 1)
+  int dual;           // 1: an item is one group on two key tiles (G * HP <= 128, pair == 1);
+                      //    tiles then counts tile pairs
   uint64_t wait_ns;   // bound of every wait (0: give up unless already complete)
 };
 
