@@ -32,9 +32,12 @@ INDEXER_CASES = [
     (6, 1100, 64, 128, True, True, True),
     (2, 640, 20, 64, False, True, False),
     (1, 1, 64, 128, False, False, False),
-    # one shared cache, two query groups per key tile (64, 16 and 128 heads)
+    # one shared cache, two query groups per key tile (64, 16, 32 and 128
+    # heads; a last item of one group)
     (8, 3000, 64, 128, True, False, False),
     (17, 1000, 16, 64, True, False, True),
+    (12, 2100, 64, 128, True, False, False),
+    (40, 1500, 32, 128, True, False, True),
     (4, 2000, 128, 128, True, False, False),
 ]
 
