@@ -370,6 +370,10 @@ def run_native(args):
         if ref and "roofline" in ref:
             line["indexer_hbm_128k"] = {"workload": "single_F_B8_N131072_per_query_caches", "gbs": ref["gbs"],
                                         "frac_of_hbm": ref["gbs"] / hbm_gbs, "us": ref["us"]}
+    if rank == 0 and world == 1 and not args.no_configs:
+        del st, graph, wl
+        torch.cuda.empty_cache()
+        line["reuse_overlap"] = reuse_diagnostic(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, ta = cpu_sample_step()
         tf, ta = cpu_sample_step(seed=8)
@@ -593,6 +597,42 @@ def mla_work(rows, B, H, k, gate):
     """Gathered rows once each, q, the output (and gate) once, the indices."""
     return (rows * D_QK * 2 + B * H * D_QK * 2 + B * H * D_V * 2 * (2 if gate else 1) + B * k * 4,
             2.0 * B * H * k * (D_QK + D_V))
+
+
+def reuse_diagnostic(dev):
+    """Recall of the reused index on every S layer of the stack (outside the
+    timed region): the overlap of the last F layer's top-k with the top-k the
+    S layer would compute from indexer inputs of its own, over k. Two key
+    recipes: independent keys per layer (the stack's; recall ~ k/N by
+    construction) and one key cache for all layers (the queries' layer-to-
+    layer correlation rho = 0.8 is then what the reuse keeps)."""
+    import torch
+    from lightning_indexer_cross_b200 import ops
+    from lightning_indexer_cross_b200 import workloads as W
+    out = {"what": "overlap of the reused index with the S layer's own top-k, / k (mean over queries)"}
+    for keys in ("per_layer", "shared"):
+        wl = W.stack(dev, seed=replica_seed(0), L=L, n_full=N_FULL, B=B, N=N, H_I=H_I, d_I=D_I, topk=TOPK, H=H,
+                     gate=False, s_indexers=True, layer_keys=keys)
+        for lay in wl.layers:  # only the indexer inputs are used
+            lay.kv = lay.q = None
+        torch.cuda.empty_cache()
+        got = ops.reuse_overlap(wl.layers, wl.schedule, wl.topk)
+        torch.cuda.synchronize()
+        gov, last = [], -1
+        for l, c in enumerate(wl.schedule):
+            last = l if c == "F" else last
+            gov.append(last)
+        rec = {l: float(v.double().mean().item()) / wl.topk for l, v in got.items()}
+        by_d = {}
+        for l, r in rec.items():
+            by_d.setdefault(l - gov[l], []).append(r)
+        vals = list(rec.values())
+        out[keys + "_keys"] = {"s_layers": len(vals), "recall_mean": sum(vals) / len(vals), "recall_min": min(vals),
+                               "recall_max": max(vals),
+                               "recall_by_distance": {str(d): sum(v) / len(v) for d, v in sorted(by_d.items())}}
+        del wl, got
+        torch.cuda.empty_cache()
+    return out
 
 
 def time_configs(dev, hbm_gbs, tf_burst):

@@ -357,6 +357,27 @@ ic_status_t ic_cp_combine(const float* part_out, int64_t out_stride, const float
                           float* lse, ic_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * ic_index_overlap -- per-row overlap of two index sets: the reuse diagnostic
+ * of the layer stack (Hy4 IndexCache explainer: reuse is free only where
+ * nearby layers want the same tokens -- the bet that sparse selections are
+ * largely shared between nearby layers; Bai et al. record: cross-layer reuse
+ * is not exact equality to each layer's own selection). With a = the index
+ * an S layer reuses and b = the top-k it would compute itself, count / k is
+ * the recall of the reused index.
+ *
+ *   a, b   [B, k] int32, device; entries outside [0, N) (the -1 padding)
+ *          are ignored. A row of b is expected to hold distinct indices
+ *          (as every top-k output does): a repeated entry is counted again.
+ *   count  [B] int32, device: count[r] = number of valid b[r, :] entries
+ *          that occur in a[r, :].
+ *   N      1 <= N <= 1,851,392 (one bit per position in shared memory);
+ *          larger N: IC_ERR_UNSUPPORTED.
+ * One kernel launch on `stream`, no workspace.
+ * ------------------------------------------------------------------------- */
+ic_status_t ic_index_overlap(const int32_t* a, const int32_t* b, int B, int k, int64_t N, int32_t* count,
+                             ic_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * ic_last_device_status -- synchronises `stream`, then reads and clears the
  * device status word at the start of `workspace` (any of the workspaces
  * above). Returns IC_OK, IC_ERR_TIMEOUT or IC_ERR_BAD_INDEX (or IC_ERR_CUDA

@@ -49,6 +49,7 @@ EXPORTED = [
     "ic_cp_workspace_size",
     "ic_cp_merge_topk",
     "ic_cp_combine",
+    "ic_index_overlap",
 ]
 
 
@@ -122,6 +123,7 @@ _cp_cand = _sig("ic_cp_candidates", _i, [_p, _p, _i, _i64, _i, _i64, _p, _p, _p,
 _cp_ws = _sig("ic_cp_workspace_size", _sz, [])
 _cp_merge = _sig("ic_cp_merge_topk", _i, [_p, _p, _i64, _i, _i, _i, _i, _i64, _i64, _p, _p, _p])
 _cp_combine = _sig("ic_cp_combine", _i, [_p, _i64, _p, _i64, _i, _i, _i, _p, _p, _i, _p, _p, _p])
+_overlap = _sig("ic_index_overlap", _i, [_p, _p, _i, _i, _i64, _p, _p])
 _set_wait = _sig("ic_set_wait_limit_ns", None, [ctypes.c_uint64])
 _get_wait = _sig("ic_wait_limit_ns", ctypes.c_uint64, [])
 
@@ -237,6 +239,10 @@ def ic_cp_combine(part_out, out_stride, part_lse, lse_stride, G, B, H, sink, gat
                   stream) -> None:
     _check(_cp_combine(part_out, out_stride, part_lse, lse_stride, G, B, H, sink, gate, out_dtype, out, lse, stream),
            "ic_cp_combine")
+
+
+def ic_index_overlap(a, b, B, k, N, count, stream) -> None:
+    _check(_overlap(a, b, B, k, N, count, stream), "ic_index_overlap")
 
 
 IC_CP_MAX_CANDIDATES = 16384

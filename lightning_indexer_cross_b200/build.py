@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libindexcache.so")
-SOURCES = ["api.cu", "indexer.cu", "topk.cu", "sparse_mla.cu", "topk_noalloc.cu", "append.cu", "gate.cu", "context_parallel.cu", "topk_threshold.cu"]
+SOURCES = ["api.cu", "indexer.cu", "topk.cu", "sparse_mla.cu", "topk_noalloc.cu", "append.cu", "gate.cu", "context_parallel.cu", "topk_threshold.cu", "overlap.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "-diag-suppress", "177", "-I", INCLUDE]

@@ -775,4 +775,17 @@ ic_status_t ic_last_device_status(void* workspace, ic_stream_t stream) {
   return v == 0 ? IC_OK : IC_ERR_CUDA;
 }
 
+ic_status_t ic_index_overlap(const int32_t* a, const int32_t* b, int B, int k, int64_t N, int32_t* count,
+                             ic_stream_t stream) {
+  g_launches = 0;
+  if (!a || !b || !count || B < 1 || k < 1 || N < 1) return IC_ERR_INVALID_ARG;
+  if (ic::index_overlap_smem_bytes(N) > 232448 - 1024) return IC_ERR_UNSUPPORTED;
+  int n = 0;
+  if (ic::launch_index_overlap(a, b, B, k, N, count, reinterpret_cast<cudaStream_t>(stream), false, &n) !=
+      cudaSuccess)
+    return IC_ERR_CUDA;
+  g_launches = n;
+  return IC_OK;
+}
+
 }  // extern "C"

@@ -179,6 +179,11 @@ int mla_smem_bytes(int ts);
 cudaError_t launch_sparse_mla(const CUtensorMap& qmap, const CUtensorMap& omap, const MlaArgs& a,
                               cudaStream_t stream, bool pdl, int* launches);
 
+// ---------------------------------------------------------------- index overlap
+size_t index_overlap_smem_bytes(int64_t N);
+cudaError_t launch_index_overlap(const int32_t* a, const int32_t* b, int B, int k, int64_t N, int32_t* count,
+                                 cudaStream_t stream, bool pdl, int* launches);
+
 // ---------------------------------------------------------------- cache append
 struct AppendArgs {
   const __nv_bfloat16* k_raw;    // [T, d_I] indexer keys before the norm

@@ -285,6 +285,46 @@ def cp_combine(part_out: torch.Tensor, part_lse: torch.Tensor, sink: torch.Tenso
     return out, lse
 
 
+def index_overlap(a: torch.Tensor, b: torch.Tensor, N: int, count: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """Per row, the number of valid entries of b ([B, k] int32) that occur in a: [B] int32."""
+    _need_cuda(a, b, count)
+    _need_dense(a, b, count)
+    assert a.dim() == 2 and a.shape == b.shape and a.dtype == torch.int32 and b.dtype == torch.int32
+    B, k = a.shape
+    if count is None:
+        count = torch.empty((B,), dtype=torch.int32, device=a.device)
+    assert count.shape == (B,) and count.dtype == torch.int32
+    _abi.ic_index_overlap(_ptr(a), _ptr(b), B, k, int(N), _ptr(count), _stream_ptr(stream))
+    return count
+
+
+def reuse_overlap(layers: Sequence, schedule: str, topk: int, n_valid: Optional[torch.Tensor] = None,
+                  rows_per_pass: int = 0, stream=None) -> dict:
+    """The reuse diagnostic of a layer stack: for every S layer that carries
+    indexer inputs, the overlap (per query, [B] int32) of the index it reuses
+    -- the last preceding F layer's top-k -- with the top-k of its own
+    indexer; recall = overlap / topk. Layers without indexer inputs (the
+    stack's S layers normally) are skipped."""
+    own, last, ws = {}, None, None
+    for l, c in enumerate(schedule):
+        lay = layers[l]
+        if lay.q_idx is None:
+            if c == "F":
+                raise ValueError(f"F layer {l} has no indexer inputs")
+            continue
+        B, N = lay.q_idx.shape[0], lay.k_idx.shape[1]
+        if ws is None:
+            ws = new_workspace(_abi.ic_indexer_topk_workspace_size(B, N, topk, rows_per_pass), lay.q_idx.device)
+        idx = indexer_topk(lay.q_idx, lay.w, lay.k_idx, topk, lay.k_scale, n_valid, rows_per_pass, workspace=ws,
+                           stream=stream)
+        if c == "F":
+            last = idx
+        elif last is not None:
+            own[l] = index_overlap(last, idx, N, stream=stream)
+    return own
+
+
 class LayerStack:
     """Holds the per-layer pointer table, the shape struct, the index buffer
     and the workspace of one decode stack, so that a step is one C call."""

@@ -237,15 +237,25 @@ def single_f(device="cpu", seed: int = 1, N: int = 131072, B: int = 8, H_I: int 
 
 def stack(device="cpu", seed: int = 2, L: int = 78, n_full: int = 21, B: int = 32,
           N: int = 131072, H_I: int = 64, d_I: int = 128, topk: int = 2048, H: int = 128,
-          rho: float = 0.8, schedule: Optional[str] = None, gate: bool = True) -> Workload:
+          rho: float = 0.8, schedule: Optional[str] = None, gate: bool = True,
+          s_indexers: bool = False, layer_keys: str = "per_layer") -> Workload:
     """The 78-layer F/S decode stack: one key cache and one KV cache per layer,
     shared by all B queries; keys independent per layer; indexer and attention
-    queries correlated across layers, q_l = rho q_{l-1} + sqrt(1-rho^2) eps_l."""
+    queries correlated across layers, q_l = rho q_{l-1} + sqrt(1-rho^2) eps_l.
+
+    For the reuse diagnostic only: s_indexers also gives every S layer the
+    indexer inputs it would have (its query from the same correlated chain,
+    weights and keys from a second generator, so the stack's own inputs are
+    unchanged); layer_keys="shared" makes every layer's indexer keys those of
+    layer 0 (the draws of the others are still made and then dropped)."""
+    assert layer_keys in ("per_layer", "shared")
     sched = schedule if schedule is not None else hy4_schedule(L, n_full, seed)
     assert len(sched) == L
     g = _gen(seed, device)
+    g2 = _gen(seed + 7919, device) if s_indexers else None
     c = math.sqrt(1.0 - rho * rho)
     qi_prev = q_prev = None
+    keys0 = None
     layers = []
     for l in range(L):
         eps_i = _randn((B, H_I, d_I), g, device, 1.0 / math.sqrt(d_I))
@@ -261,6 +271,13 @@ def stack(device="cpu", seed: int = 2, L: int = 78, n_full: int = 21, B: int = 3
             lay.q_idx = qi_f.to(torch.bfloat16)
             lay.w = _rand((B, H_I), g, device, 1.0 / H_I)
             lay.k_idx = _randn((1, N, d_I), g, device, 1.0 / math.sqrt(d_I)).to(torch.bfloat16)
+        elif s_indexers:
+            lay.q_idx = qi_f.to(torch.bfloat16)
+            lay.w = _rand((B, H_I), g2, device, 1.0 / H_I)
+            lay.k_idx = _randn((1, N, d_I), g2, device, 1.0 / math.sqrt(d_I)).to(torch.bfloat16)
+        if layer_keys == "shared" and lay.k_idx is not None:
+            keys0 = lay.k_idx if keys0 is None else keys0
+            lay.k_idx = keys0
         layers.append(lay)
     return Workload(f"stack{L}_B{B}_N{N}", B, N, H_I, d_I, topk, H, sched, layers,
                     shared_keys=True, shared_kv=True, seed=seed)

@@ -19,6 +19,8 @@ from .indexcache_oracle import (  # noqa: F401
     layer_stack,
     validate_schedule,
     governing_full_layer,
+    index_overlap,
+    reuse_overlap,
 )
 from .cache_append_oracle import (  # noqa: F401
     layernorm_bias,

@@ -260,3 +260,40 @@ def layer_stack(layers: Sequence, schedule: str, topk: int, n_valid=None,
         lses.append(lse)
     return {"idx": idx_per_layer, "out": outs, "lse": lses, "n_scores": n_scores,
             "governing": gov}
+
+
+# ----------------------------------------------------------------------------
+# Reuse diagnostic
+# ----------------------------------------------------------------------------
+def index_overlap(a, b, N: int) -> np.ndarray:
+    """Per row, how many valid entries of b (in [0, N); -1 padding and
+    anything else ignored) occur among the valid entries of a. Reuse is free
+    only where nearby layers want the same tokens (Hy4 IndexCache explainer,
+    the bet that sparse selections are largely shared between nearby layers);
+    with a = the reused index and b = a layer's own top-k this counts what
+    the reuse keeps (Bai et al. record: cross-layer reuse is not exact
+    equality to each layer's own selection)."""
+    a = np.asarray(_f64(a), dtype=np.int64)
+    b = np.asarray(_f64(b), dtype=np.int64)
+    out = np.zeros(a.shape[0], dtype=np.int64)
+    for r in range(a.shape[0]):
+        have = {int(x) for x in a[r] if 0 <= x < N}
+        out[r] = sum(1 for x in b[r] if 0 <= x < N and int(x) in have)
+    return out
+
+
+def reuse_overlap(layers: Sequence, schedule: str, topk: int, n_valid=None, k_fp8: bool = False) -> Dict[int, np.ndarray]:
+    """For each S layer that carries indexer inputs: index_overlap of the
+    index it reuses (the last preceding F layer's top-k) with the top-k of
+    its own indexer scores, per query."""
+    gov = governing_full_layer(schedule)
+    own = {}
+    for l, c in enumerate(schedule):
+        lay = layers[l]
+        if lay.q_idx is None:
+            continue
+        sc = indexer_scores(lay.q_idx, lay.w, lay.k_idx, lay.k_scale, n_valid, keys_are_e4m3=k_fp8)
+        own[l] = topk_indices(sc, topk, n_valid)
+    N = layers[0].k_idx.shape[1]
+    return {l: index_overlap(own[gov[l]], own[l], N) for l, c in enumerate(schedule) if c == "S" and l in own}
+

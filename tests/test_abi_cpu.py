@@ -94,6 +94,19 @@ def test_sparse_mla_rejects_bad_arguments(abi):
     assert call(wsb=64) == abi.IC_ERR_INVALID_ARG
 
 
+def test_index_overlap_rejects_bad_arguments(abi):
+    # every case fails on the host before any launch (the pointers are host memory)
+    p, keep = _fake()
+    call = lambda **kw: abi._overlap(*[kw.get(n, d) for n, d in [
+        ("a", p), ("b", p), ("B", 2), ("k", 16), ("N", 100), ("count", p), ("st", None)]])
+    assert call(a=None) == abi.IC_ERR_INVALID_ARG
+    assert call(count=None) == abi.IC_ERR_INVALID_ARG
+    assert call(B=0) == abi.IC_ERR_INVALID_ARG
+    assert call(k=0) == abi.IC_ERR_INVALID_ARG
+    assert call(N=0) == abi.IC_ERR_INVALID_ARG
+    assert call(N=1851392 + 1) == abi.IC_ERR_UNSUPPORTED  # one bit per position in shared memory
+
+
 def test_cache_append_rejects_bad_arguments(abi):
     # every case below must fail validation: the pointers are host memory
     p, keep = _fake()
