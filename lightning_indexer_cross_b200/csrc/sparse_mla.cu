@@ -683,14 +683,14 @@ IC_DEV void combine_staged_row(const MlaArgs& a, const uint8_t* prow, const floa
   const int S = a.splits;
   float M = sink2;
   for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, mr[s2].x);
-  float den = sink2 == -INFINITY ? 0.f : exp2f(sink2 - M);  // (no term for a sink of -inf)
+  float den = sink2 == -INFINITY ? 0.f : ex2_approx(sink2 - M);  // (no term for a sink of -inf)
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
   // one split's contribution (a split with no valid row has weight 0)
   auto add_split = [&](int s2) {
     const float2 v = mr[s2];
-    const float wgt = v.x == -INFINITY ? 0.f : exp2f(v.x - M) * v.y;
+    const float wgt = v.x == -INFINITY ? 0.f : ex2_approx(v.x - M) * v.y;
     den += wgt;
     const uint8_t* ps = prow + static_cast<size_t>(s2) * kDv * ES;
 #pragma unroll
@@ -723,7 +723,8 @@ IC_DEV void combine_staged_row(const MlaArgs& a, const uint8_t* prow, const floa
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       o[e] = acc[8 * c + e] * inv;
-      if (a.gate) o[e] *= 1.f / (1.f + __expf(-bf16_lane(gwd[e >> 1], e & 1)));
+      // sigmoid with the hardware 2^x and reciprocal (relative error ~2^-21)
+      if (a.gate) o[e] *= __fdividef(1.f, 1.f + ex2_approx(-kLog2e * bf16_lane(gwd[e >> 1], e & 1)));
     }
     if (a.out_f32) {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + gw * kDv + 8 * q + 256 * c);
