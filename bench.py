@@ -945,7 +945,11 @@ def time_e2e(wl, st, args, dev, world):
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     return {"value": world * B * n / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n,
-            "overlap": "per-layer input copies on two copy streams, two input buffer sets alternating"}
+            "overlap": "per-layer input copies on two copy streams, two input buffer sets alternating",
+            "note": "the per-layer queries, weights and gates are uploaded every step because the path starts at "
+                    "them; a model computes them on the device from one hidden state per token (which the pages "
+                    "do not size), so its step would move far fewer host bytes and run at about the device-"
+                    "resident value"}
 
 
 def main():
