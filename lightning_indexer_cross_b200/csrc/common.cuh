@@ -22,12 +22,6 @@ IC_DEV void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
-// Relaxed GPU-scope load (sees other CTAs' stores without caching in L1).
-IC_DEV uint32_t ld_relaxed_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 
 IC_DEV uint64_t globaltimer_ns() {
   uint64_t t;
@@ -191,16 +185,6 @@ IC_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
-// Four rows (y0..y3, any order) x one box of columns starting at x of a 2-D
-// tensor map whose box is one row high; the rows land consecutively at dst
-// (128-byte-swizzled by shared-memory address when the map swizzles).
-IC_DEV void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y0, int y1, int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-      : "memory");
-}
 // Global -> shared contiguous copy (TMA bulk, no tensor map): both addresses
 // 16-byte aligned, bytes a multiple of 16; completes `bytes` transactions on
 // bar.
@@ -239,7 +223,6 @@ IC_DEV void cp_async16_l2_256(uint32_t dst, const void* src, uint32_t src_bytes)
   asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                : "memory");
 }
-IC_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 // One arrival on `bar` once every cp.async this thread has issued so far has
 // landed; the arrival is not pre-counted, so it is one of the barrier's
 // expected arrivals.
@@ -247,10 +230,6 @@ IC_DEV void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 IC_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-template <int N>
-IC_DEV void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // ---------------------------------------------------------------- tcgen05
 IC_DEV void tmem_alloc(uint32_t* holder, uint32_t ncols) {
@@ -281,25 +260,6 @@ IC_DEV void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane, waited on before
-// returning (the wait lives in the same asm block so no use can be hoisted
-// above it).
-IC_DEV void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 // Split form for software pipelining: issue a load of 32 columns into r[]
 // without waiting, then later wait for every outstanding load. The wait names
@@ -349,10 +309,6 @@ IC_DEV void tmem_ld_wait64(uint32_t (&r)[64]) {
                : "memory");
 }
 
-// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned) into L2.
-IC_DEV void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor of tcgen05 for a 128-byte-swizzled
