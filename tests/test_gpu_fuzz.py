@@ -89,3 +89,45 @@ def test_sparse_mla_random_shapes(cuda_dev, seed):
     what = (B, N, H, k, shared, gate, n_invalid, odt, scale)
     assert err <= ATTN_TOL[odt], f"{what}: attention row error {err:.3e}"
     np.testing.assert_allclose(lse.double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-3, err_msg=str(what))
+
+
+def _stack_draw(seed):
+    r = np.random.default_rng(seed)
+    L = int(r.integers(1, 9))
+    sched = "F" + "".join("F" if r.random() < 0.35 else "S" for _ in range(L - 1))
+    B = int(r.integers(1, 9))
+    N = int(r.integers(300, 8000))
+    k = int(r.choice([16, 100, 256, 512]))
+    H = int(r.choice([8, 64, 128]))
+    odt = torch.float32 if r.random() < 0.5 else torch.bfloat16
+    return sched, B, N, k, H, odt
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_layer_stack_random_schedules(cuda_dev, seed):
+    """Random F/S schedules over one shared cache per layer: every S layer's
+    index buffer byte-identical to its governing F layer's, every F layer's
+    set the oracle's, every layer's attention the oracle's on that set."""
+    from tests.test_gpu_parity import _check_stack
+    sched, B, N, k, H, odt = _stack_draw(5000 + seed)
+    wl = W.stack(cuda_dev, seed=6000 + seed, L=len(sched), B=B, N=N, H_I=64, d_I=128, topk=k, H=H,
+                 schedule=sched)
+    st = _ops().stack_from_workload(wl, trace=True, out_dtype=odt)
+    st.step()
+    torch.cuda.synchronize()
+    assert st.device_status() == 0
+    _check_stack(wl, st)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_decompress_gate_random_shapes(cuda_dev, seed):
+    r = np.random.default_rng(7000 + seed)
+    B, H = int(r.integers(1, 140)), int(r.choice([1, 8, 64, 128]))
+    gate = bool(r.random() < 0.7)
+    odt = torch.float32 if r.random() < 0.5 else torch.bfloat16
+    o, wv, gl = W.gate_case(B, H, gate=gate, seed=8000 + seed, device=cuda_dev)
+    out = _ops().decompress_gate(o, wv, gl, out_dtype=odt)
+    torch.cuda.synchronize()
+    from tests.test_gpu_gate import TOL, _row_err
+    err = _row_err(out, oracle.decompressed_gate(o, wv, gl))
+    assert err <= TOL[odt], f"(B,H,gate,odt)={(B, H, gate, odt)}: {err:.3e}"
