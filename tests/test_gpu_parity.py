@@ -216,6 +216,26 @@ def test_sparse_mla_all_padding_gives_zero_and_sink_lse(cuda_dev):
     torch.testing.assert_close(lse, sink.unsqueeze(0).expand(2, -1).contiguous(), rtol=1e-5, atol=1e-5)
 
 
+@pytest.mark.parametrize("odt", [torch.bfloat16, torch.float32])
+def test_sparse_mla_without_a_sink(cuda_dev, odt):
+    """sink = -inf on every head (the header's "no sink term", used by the
+    context-parallel split's local attention): plain softmax attention over
+    the selected rows, lse = log-sum-exp of the logits; a row with no valid
+    selected token gives out = 0 and lse = -inf."""
+    B, N, H, k = 3, 4000, 128, 700
+    q, kv, idx, _, g = W.attention_case(B, N, H, k, shared=True, gate=True, n_invalid=50, seed=77, device=cuda_dev)
+    idx[2].fill_(-1)
+    sink = torch.full((H,), float("-inf"), device=cuda_dev)
+    out, lse = _ops().sparse_mla_decode(q, kv, idx, sink, g, out_dtype=odt)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle.sparse_mla(q[:2], kv, idx[:2], sink, g[:2])
+    err = attn_row_error(out[:2], ref)
+    assert err <= ATTN_TOL[odt], f"attention row error {err:.3e}"
+    np.testing.assert_allclose(lse[:2].double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-3)
+    assert torch.all(out[2] == 0)
+    assert torch.all(torch.isneginf(lse[2]))
+
+
 def test_sparse_mla_very_negative_logits_after_an_empty_first_chunk(cuda_dev):
     """Every selected row equal to v, q = -c v with logits of about -200 and a
     sink of -1000: the softmax is uniform over the valid rows, so the output is
