@@ -31,8 +31,8 @@ namespace {
 constexpr int kT = 512;
 constexpr int kSample = 8192;       // sampled keys per row (the whole row up to 2 x this)
 constexpr float kAlpha = 2.f;       // candidates expected per row, in units of k
-constexpr int kLocalCap = 2048;     // candidates one filter CTA stages in shared memory
-constexpr int kSmemCand = 8192;     // candidates the last CTA selects in shared memory
+constexpr int kLocalCap = 4096;     // candidates one filter CTA stages in shared memory
+constexpr int kSmemCand = 6144;     // candidates the last CTA selects in shared memory (2k expected, 1.5 x margin)
 constexpr int kUnroll = 4;          // float4 loads in flight per thread in the scan
 
 // per-row control words (kCtrlWords 32-bit words, one 128-byte line per row)
@@ -112,14 +112,21 @@ __global__ void __launch_bounds__(kT) topk_sample_kernel(const TopkArgs a) {
     a.counters[static_cast<int64_t>(b) * kCtrlWords + kThresh] = (d1 << 20) | (static_cast<uint32_t>(sh.d) << 10);
 }
 
+// The staging lists are written out before the row's last CTA selects, so
+// its candidate array reuses their space (50 KB a CTA).
 struct FilterShared {
-  int32_t pos[kLocalCap];
-  uint32_t key[kLocalCap];
+  union {
+    struct {
+      int32_t pos[kLocalCap];
+      uint32_t key[kLocalCap];
+    };
+    uint64_t cand[kSmemCand];
+  };
   uint32_t n_local, base;
   int last;
   SelectShared sel;
-  uint64_t cand[kSmemCand];
 };
+static_assert(kSmemCand * 8 >= kLocalCap * 8, "the candidate array covers the staging lists");
 
 __global__ void __launch_bounds__(kT) topk_filter_kernel(const TopkArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -170,6 +177,40 @@ __global__ void __launch_bounds__(kT) topk_filter_kernel(const TopkArgs a) {
       }
     }
   };
+  // The same for the candidates among a lane's four consecutive keys
+  // (mask m): the warp's inclusive scan of the counts gives every lane its
+  // first slot after one reservation by the last lane.
+  auto push4 = [&](int64_t i, uint32_t m, uint32_t k0, uint32_t k1, uint32_t k2, uint32_t k3) {
+    const uint32_t cnt = static_cast<uint32_t>(__popc(m));
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    uint32_t base = 0;
+    if (lane == 31) base = atomicAdd(&sh.n_local, incl);
+    base = __shfl_sync(0xffffffffu, base, 31);
+    uint32_t p = base + incl - cnt;
+    const uint32_t kk[4] = {k0, k1, k2, k3};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if ((m >> e) & 1u) {
+        if (p < static_cast<uint32_t>(kLocalCap)) {
+          sh.pos[p] = static_cast<int32_t>(i + e);
+          sh.key[p] = kk[e];
+        } else {
+          // past the staging capacity: straight to the row's buffer
+          const uint32_t gp = atomicAdd(&ctrl[kCount], 1u);
+          if (gp < static_cast<uint32_t>(a.cand_cap)) {
+            cbuf[gp] = static_cast<int32_t>(i + e);
+            ckbuf[gp] = kk[e];
+          }
+        }
+        ++p;
+      }
+    }
+  };
   const int64_t lo = static_cast<int64_t>(c) * a.slice;
   const int64_t hi = lo + a.slice < nv ? lo + a.slice : nv;
   const float* row = a.scores + static_cast<int64_t>(b) * a.N;
@@ -198,12 +239,12 @@ __global__ void __launch_bounds__(kT) topk_filter_kernel(const TopkArgs a) {
                          k3 = order_key(v[u].w);
           const bool h0 = i < hi && k0 >= T, h1 = i + 1 < hi && k1 >= T, h2 = i + 2 < hi && k2 >= T,
                      h3 = i + 3 < hi && k3 >= T;
-          // most groups of 128 keys hold no candidate: one vote skips them
-          if (__ballot_sync(0xffffffffu, h0 | h1 | h2 | h3) == 0u) continue;
-          push(i, k0, h0);
-          push(i + 1, k1, h1);
-          push(i + 2, k2, h2);
-          push(i + 3, k3, h3);
+          // a group of 128 keys with no candidate is skipped on one vote;
+          // otherwise one warp scan of the lanes' counts and one shared
+          // reservation place the group's candidates
+          const uint32_t m = (h0 ? 1u : 0u) | (h1 ? 2u : 0u) | (h2 ? 4u : 0u) | (h3 ? 8u : 0u);
+          if (__ballot_sync(0xffffffffu, m != 0u) == 0u) continue;
+          push4(i, m, k0, k1, k2, k3);
         }
       }
     } else {
