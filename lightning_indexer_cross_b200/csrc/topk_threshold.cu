@@ -142,6 +142,9 @@ __global__ void __launch_bounds__(kT) topk_filter_kernel(const TopkArgs a) {
   }
   uint32_t* ctrl = a.counters + static_cast<int64_t>(b) * kCtrlWords;
   const uint32_t T = __ldcg(&ctrl[kThresh]);
+  // the fp32 value whose order key is T (every finite value when T lies at
+  // or below the key of -inf)
+  const float tf = T <= 0x007FFFFFu ? -INFINITY : __uint_as_float((T & 0x80000000u) ? (T & 0x7FFFFFFFu) : ~T);
   int32_t* cbuf = a.cand + static_cast<int64_t>(b) * a.cand_cap;
   uint32_t* ckbuf = a.cand_key + static_cast<int64_t>(b) * a.cand_cap;
   if (t == 0) sh.n_local = 0;
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(kT) topk_filter_kernel(const TopkArgs a) {
   // The same for the candidates among a lane's four consecutive keys
   // (mask m): the warp's inclusive scan of the counts gives every lane its
   // first slot after one reservation by the last lane.
-  auto push4 = [&](int64_t i, uint32_t m, uint32_t k0, uint32_t k1, uint32_t k2, uint32_t k3) {
+  auto push4 = [&](int64_t i, uint32_t m, const float4& x) {
     const uint32_t cnt = static_cast<uint32_t>(__popc(m));
     uint32_t incl = cnt;
 #pragma unroll
@@ -192,19 +195,20 @@ __global__ void __launch_bounds__(kT) topk_filter_kernel(const TopkArgs a) {
     if (lane == 31) base = atomicAdd(&sh.n_local, incl);
     base = __shfl_sync(0xffffffffu, base, 31);
     uint32_t p = base + incl - cnt;
-    const uint32_t kk[4] = {k0, k1, k2, k3};
+    const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if ((m >> e) & 1u) {
+        const uint32_t key = order_key(xs[e]);
         if (p < static_cast<uint32_t>(kLocalCap)) {
           sh.pos[p] = static_cast<int32_t>(i + e);
-          sh.key[p] = kk[e];
+          sh.key[p] = key;
         } else {
           // past the staging capacity: straight to the row's buffer
           const uint32_t gp = atomicAdd(&ctrl[kCount], 1u);
           if (gp < static_cast<uint32_t>(a.cand_cap)) {
             cbuf[gp] = static_cast<int32_t>(i + e);
-            ckbuf[gp] = kk[e];
+            ckbuf[gp] = key;
           }
         }
         ++p;
@@ -235,16 +239,17 @@ __global__ void __launch_bounds__(kT) topk_filter_kernel(const TopkArgs a) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
           const int64_t i = base + u * 128 + lane * 4;
-          const uint32_t k0 = order_key(v[u].x), k1 = order_key(v[u].y), k2 = order_key(v[u].z),
-                         k3 = order_key(v[u].w);
-          const bool h0 = i < hi && k0 >= T, h1 = i + 1 < hi && k1 >= T, h2 = i + 2 < hi && k2 >= T,
-                     h3 = i + 3 < hi && k3 >= T;
+          // x >= tf picks every key >= T (plus -0.0 when tf is +0.0: an extra
+          // candidate, harmless to the exact selection); keys are formed
+          // only for the candidates
+          const bool h0 = i < hi && v[u].x >= tf, h1 = i + 1 < hi && v[u].y >= tf, h2 = i + 2 < hi && v[u].z >= tf,
+                     h3 = i + 3 < hi && v[u].w >= tf;
           // a group of 128 keys with no candidate is skipped on one vote;
           // otherwise one warp scan of the lanes' counts and one shared
           // reservation place the group's candidates
           const uint32_t m = (h0 ? 1u : 0u) | (h1 ? 2u : 0u) | (h2 ? 4u : 0u) | (h3 ? 8u : 0u);
           if (__ballot_sync(0xffffffffu, m != 0u) == 0u) continue;
-          push4(i, m, k0, k1, k2, k3);
+          push4(i, m, v[u]);
         }
       }
     } else {
