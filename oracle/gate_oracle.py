@@ -23,7 +23,9 @@ from .indexcache_oracle import _f64
 
 
 def _sigmoid(x):
-    return 1.0 / (1.0 + np.exp(-x))
+    # exp(-x) overflows to inf for x < -709; 1 / (1 + inf) = 0 is then the exact limit
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-x))
 
 
 def decompress(o_latent, wv_b) -> np.ndarray:

@@ -132,7 +132,9 @@ def topk_indices(scores, k: int, n_valid=None) -> np.ndarray:
 # Sparse MLA attention with sink and gate
 # ----------------------------------------------------------------------------
 def _sigmoid(x):
-    return 1.0 / (1.0 + np.exp(-x))
+    # exp(-x) overflows to inf for x < -709; 1 / (1 + inf) = 0 is then the exact limit
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-x))
 
 
 def sparse_mla(q, kv, idx, sink, gate=None, sm_scale: Optional[float] = None, d_v: int = 512):
