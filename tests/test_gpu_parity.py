@@ -311,6 +311,34 @@ def test_sparse_mla_three_units_per_cta(cuda_dev, odt):
         np.testing.assert_allclose(lse[b:b + 1].double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-3)
 
 
+@pytest.mark.parametrize("H,odt", [(128, torch.bfloat16), (128, torch.float32), (64, torch.float32)])
+def test_sparse_mla_second_wave_and_workspace_reuse(cuda_dev, H, odt):
+    """20 queries x 8 splits = 160 work units on (at most) 148 persistent
+    CTAs: a short second wave (12 CTAs take a second unit, with the other
+    TMEM half). Every query against the oracle, with -1 rows and a ragged
+    last split, and twice on one workspace: the second call gives the same
+    bytes."""
+    from lightning_indexer_cross_b200 import _abi
+    ops = _ops()
+    B, N, k = 20, 6000, 2000
+    q, kv, idx, sink, g = W.attention_case(B, N, H, k, shared=True, gate=True, n_invalid=9, seed=43,
+                                           device=cuda_dev)
+    ws = ops.new_workspace(_abi.ic_sparse_mla_workspace_size(B, H, k), cuda_dev)
+    ref, ref_lse = oracle.sparse_mla(q, kv, idx, sink, g)
+    for call in range(2):
+        out, lse = ops.sparse_mla_decode(q, kv, idx, sink, g, out_dtype=odt, workspace=ws)
+        torch.cuda.synchronize()
+        assert _abi.ic_last_device_status(ops._ptr(ws), ops._stream_ptr()) == _abi.IC_OK
+        for b in range(B):
+            err = attn_row_error(out[b:b + 1], ref[b:b + 1])
+            assert err <= ATTN_TOL[odt], f"call {call}, query {b}: attention row error {err:.3e}"
+        np.testing.assert_allclose(lse.double().cpu().numpy(), ref_lse, rtol=1e-3, atol=1e-3)
+        if call == 0:
+            first = out.clone()
+        else:
+            torch.testing.assert_close(out, first, rtol=0, atol=0)
+
+
 def test_sparse_mla_bad_index_is_reported_and_skipped(cuda_dev):
     from lightning_indexer_cross_b200 import _abi
     ops = _ops()
