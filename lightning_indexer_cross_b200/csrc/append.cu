@@ -116,11 +116,35 @@ __global__ void __launch_bounds__(kThreads) cache_append_kernel(const AppendArgs
   __shared__ double cs_s[kPairs], sn_s[kPairs];
   if (threadIdx.x < kPairs) rope_angle(a.q_pos[b], threadIdx.x, a.log2_base, &cs_s[threadIdx.x], &sn_s[threadIdx.x]);
   __syncthreads();
-  uint32_t* qb = reinterpret_cast<uint32_t*>(a.q + static_cast<int64_t>(b) * a.H * kRowD);
-  for (int p = threadIdx.x; p < a.H * kPairs; p += kThreads) {
-    const int h = p / kPairs, i = p % kPairs;
-    uint32_t* w = qb + (static_cast<int64_t>(h) * kRowD + kLatent) / 2 + i;
-    *w = rotate_pair(*w, cs_s[i], sn_s[i]);
+  // A head's rotary dims are 128 contiguous bytes: 8 words of 16 bytes, word
+  // j holding pairs 4j .. 4j+3 (words 64 .. 71 of the head's 72). Thread x
+  // takes words x, x + kThreads, ... of the query, kWordsPer at a time with
+  // every load issued before the first store.
+  constexpr int kWordsPer = 8;
+  constexpr int kHeadWords = kRowD * 2 / 16;     // 72
+  constexpr int kRotWord0 = kLatent * 2 / 16;    // 64
+  uint4* qb = reinterpret_cast<uint4*>(a.q + static_cast<int64_t>(b) * a.H * kRowD);
+  const int words = a.H * 8;
+  for (int base = 0; base < words; base += kThreads * kWordsPer) {
+    uint4 v[kWordsPer];
+#pragma unroll
+    for (int j = 0; j < kWordsPer; ++j) {
+      const int x = base + j * kThreads + threadIdx.x;
+      if (x < words) v[j] = qb[(x >> 3) * kHeadWords + kRotWord0 + (x & 7)];
+    }
+#pragma unroll
+    for (int j = 0; j < kWordsPer; ++j) {
+      const int x = base + j * kThreads + threadIdx.x;
+      if (x < words) {
+        const int i0 = 4 * (x & 7);
+        uint4 o;
+        o.x = rotate_pair(v[j].x, cs_s[i0], sn_s[i0]);
+        o.y = rotate_pair(v[j].y, cs_s[i0 + 1], sn_s[i0 + 1]);
+        o.z = rotate_pair(v[j].z, cs_s[i0 + 2], sn_s[i0 + 2]);
+        o.w = rotate_pair(v[j].w, cs_s[i0 + 3], sn_s[i0 + 3]);
+        qb[(x >> 3) * kHeadWords + kRotWord0 + (x & 7)] = o;
+      }
+    }
   }
 }
 
