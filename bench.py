@@ -507,6 +507,13 @@ def kernel_driver(kernel, shape, fp8, warmup, iters):
         o, wv, gl = W.gate_case(Bq, H, seed=90, device=dev)
         ws = ops.new_workspace(_abi.ic_decompress_gate_workspace_size(), dev)
         fn = lambda: ops.decompress_gate(o, wv, gl, workspace=ws)
+    elif kernel == "append":
+        # Bq new tokens into an Nk-row shared cache, Bq queries' rotary dims
+        c = W.append_case(Bq, Nk, D_I, per_token=False, fp8=fp8, B=Bq, H=H, seed=70, device=dev)
+        ws = ops.new_workspace(_abi.ic_cache_append_workspace_size(), dev)
+        fn = lambda: ops.cache_append(c["k_raw"], c["gamma"], c["beta"], c["kv_raw"], c["pos"], c["key_cache"],
+                                      c["kv_cache"], key_scale=c.get("key_scale"), q=c["q"], q_pos=c["q_pos"],
+                                      workspace=ws)
     else:
         q, w, k, ks, _ = W.indexer_case(Bq, Nk, H_I, D_I, shared=shared, fp8=fp8, seed=5, device=dev)
         scores = ops.indexer_score(q, w, k, ks)
@@ -963,7 +970,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip timing the other workloads' kernels")
     ap.add_argument("--warmup-ref", type=int, default=1)
-    ap.add_argument("--kernel-driver", choices=["indexer", "topk", "mla", "gate"],
+    ap.add_argument("--kernel-driver", choices=["indexer", "topk", "mla", "gate", "append"],
                     help="run one kernel family on --shape instead (for ncu): --warmup untimed, --steps timed")
     ap.add_argument("--shape", choices=list(DRIVER_SHAPES), default="stack")
     ap.add_argument("--fp8", action="store_true", help="e4m3 keys for --kernel-driver")
