@@ -98,7 +98,9 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(&map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(k), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                   // e4m3 keys with d_I = 128 go to the MMA as they land (128-byte
+                   // rows, 128-byte swizzle); with d_I = 64 they are widened first
+                   (fp8 && d_I == 64) ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
   const int HP = indexer_hp(H_I);
@@ -115,6 +117,7 @@ ic_status_t indexer_impl(const void* q, const float* w, const void* k, const flo
   if (r != CUDA_SUCCESS) return IC_ERR_INVALID_ARG;
 
   ic::IndexerArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
   a.w = w;
   a.k_scale = k_scale;
   a.scale_batch_stride = per_query ? scale_batch_stride : 0;

@@ -26,14 +26,24 @@
 //               the TMA loads of the groups' Q (swizzled, zero-padded heads).
 //               warps 2..9, two per TMEM lane quadrant, each reducing one
 //               half of the columns.
-//   warps 10..13 (e4m3 keys only) widen e4m3 tiles to f16 in shared memory
-//               (one conversion instruction per two codes; exact) and, once
-//               per query group, the staged bf16 queries to f16 in place:
-//               tcgen05 kind::f16 takes two f16 (or two bf16) operands. A bf16
-//               query value is exact in f16 from 2^-14 up to 65504 (below,
-//               f16 keeps fewer bits: an error under 2^-25; the e4m3 path
-//               needs |q| < 65504). The per-token scale is applied to the head
-//               sum, since ReLU(c x) = c ReLU(x) for c >= 0.
+//   warps 10..13 (e4m3 keys only). With d_I = 128 the key tiles go to the
+//               MMA as they are (tcgen05 kind::f8f6f4, e4m3 x e4m3, fp32
+//               accumulation), and these warps, once per query group, split
+//               each query column (one head of one query) into two e4m3
+//               parts, q s = hi + lo, with s a power of two that puts the
+//               column's largest |q| in [128, 256): hi = e4m3(q s) keeps its
+//               leading 4 bits, lo = e4m3(q s - hi) the next 4, so the sum
+//               equals the bf16 value exactly for every element with
+//               |q s| >= 2^-2 (smaller ones keep a 2^-10 grid); each key tile
+//               then takes two MMA passes, hi and lo, into one accumulator, and
+//               the head weight w is read as w / s. With d_I = 64 they widen
+//               the e4m3 tiles to f16 in shared memory (one conversion
+//               instruction per two codes; exact) and the staged bf16
+//               queries to f16 in place for kind::f16 (two f16 operands; a
+//               bf16 query value is exact in f16 from 2^-14 up to 65504, an
+//               error under 2^-25 below; the path needs |q| < 65504). The
+//               per-token scale is applied to the head sum, since
+//               ReLU(c x) = c ReLU(x) for c >= 0.
 #include <cuda_fp8.h>
 
 #include <type_traits>
@@ -49,6 +59,32 @@ constexpr int kTileKeys = 128;
 constexpr int kMaxCols = 256;  // MMA N limit for M = 128
 constexpr int kEpiWarp0 = 2;
 
+// Named barrier over n threads that also ORs a predicate across them: every
+// participating thread gets the same answer.
+IC_DEV bool named_bar_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1 : 0), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// tcgen05.mma with e4m3 A and B from shared memory (kind::f8f6f4: K = 32 per
+// instruction; the instruction descriptor's A and B formats 0 are e4m3).
+IC_DEV void mma_e4m3_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // PAIR: two query groups (two Q slots, one TMEM accumulator each) share every
 // key tile a CTA loads -- one cache shared by all queries; half the key-tile
 // traffic, two key stages instead of four.
@@ -57,10 +93,18 @@ struct IdxCfg {
   static constexpr int kBlocks = D_I / 64;                        // 64-element (128 B) swizzle blocks
   static constexpr int kTileBytes = kTileKeys * D_I * 2;          // bf16 tile
   static constexpr int kRawBytes = FP8 ? kTileKeys * D_I : 0;     // e4m3 tile
-  static constexpr int kStages = FP8 ? 2 : (PAIR ? (D_I == 128 ? 2 : 4) : (D_I == 128 ? 4 : 6));  // bf16 stages
-  static constexpr int kRawStages = FP8 ? 4 : 0;
+  // e4m3 keys with d_I = 128: 128-byte rows, 128-byte swizzle, read by the
+  // MMA directly (kind::f8f6f4); no bf16 / f16 key stages
+  static constexpr bool kF8Mma = FP8 && D_I == 128;
+  static constexpr int kStages =
+      kF8Mma ? 0 : (FP8 ? 2 : (PAIR ? (D_I == 128 ? 2 : 4) : (D_I == 128 ? 4 : 6)));  // bf16 stages
+  static constexpr int kRawStages = kF8Mma ? 6 : (FP8 ? 4 : 0);
   static constexpr int kQSlots = PAIR ? 2 : 1;
+  // a slot: the group's stacked query columns, bf16 (or f16) in kBlocks
+  // 64-dim blocks; kF8Mma: the e4m3 high parts, then the low parts, 128 B
+  // per column each (the same 64 KB)
   static constexpr int kQSlotBytes = kMaxCols * D_I * 2;
+  static constexpr int kQPartBytes = kMaxCols * 128;
   static constexpr int kQBytes = kQSlots * kQSlotBytes;
   // 8 epilogue warps, two per TMEM lane quadrant, each reducing one half of
   // the columns (two warps per SM sub-partition hide each other's TMEM-load
@@ -80,11 +124,13 @@ struct IdxCfg {
   static constexpr int kOffQ = kOffRaw + kRawStages * kRawBytes;
   static constexpr int kOffW = kOffQ + kQBytes;
   static constexpr int kOffNv = kOffW + kQSlots * kMaxCols * 4;
-  static constexpr int kOffBar = kOffNv + kQSlots * 16 * 8;
+  static constexpr int kOffQs = kOffNv + kQSlots * 16 * 8;        // kF8Mma: 1 / s of each query column
+  static constexpr int kOffBar = kOffQs + (kF8Mma ? kMaxCols * 4 : 0);
   static constexpr int kNumBars = 2 * kStages + 2 * kRawStages + 4 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(!(FP8 && PAIR), "e4m3 keys take one group per tile");
+  static_assert(kOffQ % 1024 == 0 && kRawBytes % 1024 == 0, "swizzled operands 1024-byte aligned");
   static_assert(kSmemBytes <= 232448, "fits one CTA per SM");
 };
 
@@ -108,6 +154,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   uint8_t* qs = smem + C::kOffQ;
   float* ws = reinterpret_cast<float*>(smem + C::kOffW);
   int64_t* nvs = reinterpret_cast<int64_t*>(smem + C::kOffNv);
+  float* qinv = reinterpret_cast<float*>(smem + C::kOffQs);  // kF8Mma
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;                          // [kStages] bf16 tile ready
   uint64_t* empty = full + C::kStages;            // [kStages] bf16 tile consumed
@@ -140,7 +187,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     }
     for (int i = 0; i < C::kRawStages; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_empty[i], C::kConvThreads);
+      mbar_init(&raw_empty[i], C::kF8Mma ? 1 : C::kConvThreads);  // kF8Mma: freed by the MMA commit
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -207,7 +254,9 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // bf16 keys: bf16 x bf16; e4m3 keys: both operands widened to f16
+      // bf16 keys: bf16 x bf16; e4m3 keys: e4m3 x e4m3 (kF8Mma) or both
+      // operands widened to f16 -- format 0 of kind::f8f6f4 and of kind::f16
+      // alike, so one descriptor serves both
       const uint32_t idesc = FP8 ? idesc_f16_f32(128, ncols) : idesc_bf16_f32(128, ncols, false, false);
       const uint32_t q_addr = smem_u32(qs);
       int cur_grp = -1;
@@ -215,6 +264,47 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
       int64_t it = 0, si = 0;  // items; (item, group) sub-items -> accumulator si & 1
       int64_t jt = 0;          // key tiles consumed (the stage sequence)
       bool ok = true;
+      // key tile j: wait until it is in shared memory; its operand address
+      auto tile_in = [&](int64_t j, uint32_t& a_addr) -> bool {
+        if constexpr (C::kF8Mma) {
+          const int rs = static_cast<int>(j % C::kRawStages);
+          if (!mbar_wait(&raw_full[rs], static_cast<uint32_t>((j / C::kRawStages) & 1), abort_flag, a.status,
+                         a.wait_ns))
+            return false;
+          a_addr = smem_u32(raw + rs * C::kRawBytes);
+        } else {
+          const int st = static_cast<int>(j % C::kStages);
+          if (!mbar_wait(&full[st], static_cast<uint32_t>((j / C::kStages) & 1), abort_flag, a.status, a.wait_ns))
+            return false;
+          a_addr = smem_u32(stages + st * C::kTileBytes);
+        }
+        tc_fence_after();
+        return true;
+      };
+      // D[128 keys x ncols] (+)= tile . Q^T over d_I
+      auto tile_mma = [&](uint32_t d_tmem, uint32_t a_addr, uint32_t qb) {
+        if constexpr (C::kF8Mma) {
+#pragma unroll
+          for (int part = 0; part < 2; ++part)  // high, then low parts of the queries
+#pragma unroll
+            for (int kk = 0; kk < D_I / 32; ++kk)
+              mma_e4m3_ss(d_tmem, sw128_desc(a_addr + kk * 32, 16, 1024),
+                          sw128_desc(qb + part * C::kQPartBytes + kk * 32, 16, 1024), idesc, (part | kk) != 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D_I / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32;
+            const uint32_t qoff = (kk >> 2) * (kMaxCols * 128) + (kk & 3) * 32;
+            mma_bf16_ss(d_tmem, sw128_desc(a_addr + koff, 16, 1024), sw128_desc(qb + qoff, 16, 1024), idesc,
+                        kk > 0 ? 1u : 0u);
+          }
+        }
+      };
+      // the stage of key tile j is free once the MMAs issued so far complete
+      auto tile_out = [&](int64_t j) {
+        if constexpr (C::kF8Mma) mma_commit(&raw_empty[j % C::kRawStages]);
+        else mma_commit(&empty[j % C::kStages]);
+      };
       for (int64_t wi = lo; wi < hi && ok; ++wi, ++it) {
         const int grp = static_cast<int>(wi / a.tiles) * P;
         const int ng = P == 1 ? 1 : (a.groups - grp < P ? a.groups - grp : P);
@@ -230,49 +320,29 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
           if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status, a.wait_ns)) break;
           tc_fence_after();
           for (int h = 0; h < 2 && ok; ++h, ++jt) {
-            const int st = static_cast<int>(jt % C::kStages);
-            const uint32_t ph = static_cast<uint32_t>((jt / C::kStages) & 1);
-            if (!mbar_wait(&full[st], ph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t a_addr = smem_u32(stages + st * C::kTileBytes);
-            const uint32_t d_tmem = tmem_base + acc * 256 + h * 128;
-#pragma unroll
-            for (int kk = 0; kk < D_I / 16; ++kk) {
-              const uint32_t koff = (kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32;
-              const uint32_t qoff = (kk >> 2) * (kMaxCols * 128) + (kk & 3) * 32;
-              mma_bf16_ss(d_tmem, sw128_desc(a_addr + koff, 16, 1024), sw128_desc(q_addr + qoff, 16, 1024), idesc,
-                          kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&empty[st]);
+            uint32_t a_addr;
+            if (!tile_in(jt, a_addr)) { ok = false; break; }
+            tile_mma(tmem_base + acc * 256 + h * 128, a_addr, q_addr);
+            tile_out(jt);
           }
           if (!ok) break;
           mma_commit(&acc_full[acc]);
           ++si;
           continue;
         }
-        const int st = static_cast<int>(jt % C::kStages);
-        const uint32_t ph = static_cast<uint32_t>((jt / C::kStages) & 1);
-        ++jt;
-        if (!mbar_wait(&full[st], ph, abort_flag, a.status, a.wait_ns)) break;
-        const uint32_t a_addr = smem_u32(stages + st * C::kTileBytes);
+        uint32_t a_addr;
+        const int64_t j = jt++;
+        if (!tile_in(j, a_addr)) break;
         for (int sub = 0; sub < ng; ++sub, ++si) {
           const int acc = static_cast<int>(si & 1);
           const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
           if (!mbar_wait(&acc_empty[acc], aph ^ 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + acc * 256;
-          const uint32_t qb = q_addr + sub * C::kQSlotBytes;
-#pragma unroll
-          for (int kk = 0; kk < D_I / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32;
-            const uint32_t qoff = (kk >> 2) * (kMaxCols * 128) + (kk & 3) * 32;
-            mma_bf16_ss(d_tmem, sw128_desc(a_addr + koff, 16, 1024), sw128_desc(qb + qoff, 16, 1024), idesc,
-                        kk > 0 ? 1u : 0u);
-          }
+          tile_mma(tmem_base + acc * 256, a_addr, q_addr + sub * C::kQSlotBytes);
           mma_commit(&acc_full[acc]);
         }
         if (!ok) break;
-        mma_commit(&empty[st]);
+        tile_out(j);
       }
       // make sure nothing issued is still running before TMEM is released
       mma_commit(mma_done);
@@ -288,6 +358,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     int cur_grp = -1;
     int64_t si = 0;  // (item, group) sub-items, as counted by the MMA issuer
     uint32_t q_loads = 0;  // query-slot loads issued (by thread et == 0)
+    uint32_t conv_phase = 0;  // kF8Mma: the converters' query splits completed
     bool got = true;
     for (int64_t wi = lo; wi < hi && got; ++wi) {
       const int grp = static_cast<int>(wi / a.tiles) * P;
@@ -304,12 +375,16 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         // filled. The MMA issuer waits for the bytes on q_ready.
         ++q_loads;
         if (et == 0) {
-          mbar_arrive_expect_tx(q_ready, static_cast<uint32_t>(ng * C::kBlocks * HP * a.G * 128));
-          for (int slot = 0; slot < ng; ++slot)
+          if constexpr (C::kF8Mma) {
+            mbar_arrive(q_ready);  // the slot is free: the converters read the queries themselves
+          } else {
+            mbar_arrive_expect_tx(q_ready, static_cast<uint32_t>(ng * C::kBlocks * HP * a.G * 128));
+            for (int slot = 0; slot < ng; ++slot)
 #pragma unroll
-            for (int bk = 0; bk < C::kBlocks; ++bk)
-              tma_load_3d(qs + slot * C::kQSlotBytes + bk * (kMaxCols * 128), &qmap, q_ready, bk * 64, 0,
-                          (grp + slot) * a.G);
+              for (int bk = 0; bk < C::kBlocks; ++bk)
+                tma_load_3d(qs + slot * C::kQSlotBytes + bk * (kMaxCols * 128), &qmap, q_ready, bk * 64, 0,
+                            (grp + slot) * a.G);
+          }
         }
         for (int slot = 0; slot < ng; ++slot) {
           const int b0 = (grp + slot) * a.G;
@@ -325,6 +400,20 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
           }
         }
         named_bar_sync(1, kNumEpiThreads);
+        if constexpr (C::kF8Mma) {
+          // the weights of the columns split as q s = hi + lo become w / s
+          const bool fail = !mbar_wait(q_conv, conv_phase, abort_flag, a.status, a.wait_ns);
+          conv_phase ^= 1;
+          if (named_bar_or(1, kNumEpiThreads, fail)) {  // every epilogue thread leaves together
+            got = false;
+            break;
+          }
+          for (int i = et; i < kMaxCols; i += kNumEpiThreads) {
+            const int col = DUAL ? (i & 127) : i;  // (columns past ncols: weight 0, qinv unwritten)
+            if (col < ncols) ws[i] *= qinv[col];
+          }
+          named_bar_sync(1, kNumEpiThreads);
+        }
         cur_grp = grp;
       }
       for (int sub = 0; sub < ng; ++sub, ++si) {
@@ -496,71 +585,134 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
   } else if constexpr (FP8) {
     // ------------------------------------------------------------ e4m3 -> f16
     const int ct = threadIdx.x - (kEpiWarp0 + C::kEpiWarps) * 32;  // 0 .. kConvThreads - 1
-    int64_t jt = 0;  // key tiles converted (the stage sequence)
-    int cur_grp = -1;
-    uint32_t q_phase = 0;
-    bool ok = true;
-    for (int64_t wi = lo; wi < hi && ok; ++wi) {
-      const int grp = static_cast<int>(wi / a.tiles) * P;
-      if (grp != cur_grp) {
-        // the group's queries, staged as bf16 by TMA, become f16 in place
-        // (element by element, so the swizzled positions stay); the slot is
-        // rewritten only after the previous group's MMAs have completed
+    if constexpr (C::kF8Mma) {
+      // Once per query group, each query column (head h of query b) split as
+      // q s = hi + lo into the slot's two e4m3 operands (128-byte rows,
+      // 128-byte swizzle), 1 / s to qinv; the slot is rewritten only after
+      // the previous group's MMAs have completed (the epilogue frees it).
+      int cur_grp = -1;
+      uint32_t q_phase = 0;
+      const uint32_t qhi = smem_u32(qs), qlo = qhi + C::kQPartBytes;
+      for (int64_t wi = lo; wi < hi; ++wi) {
+        const int grp = static_cast<int>(wi / a.tiles) * P;
+        if (grp == cur_grp) continue;
         if (!mbar_wait(q_ready, q_phase, abort_flag, a.status, a.wait_ns)) break;
         q_phase ^= 1;
         cur_grp = grp;
-        constexpr int kRowChunks = 8;  // 16-byte chunks per 128-byte row
-        const int nchunks = C::kBlocks * ncols * kRowChunks;
-        for (int i = ct; i < nchunks; i += C::kConvThreads) {
-          const int bk = i / (ncols * kRowChunks), rem = i % (ncols * kRowChunks);
-          uint4* pq = reinterpret_cast<uint4*>(qs + bk * (kMaxCols * 128) + rem * 16);
-          const uint4 v = *pq;
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o[4];
+        const int b0 = grp * a.G;
+        for (int r = ct; r < ncols; r += C::kConvThreads) {
+          const int g = r / HP, h = r % HP, b = b0 + g;
+          const bool valid = g < a.G && h < a.H_I && b < a.B;
+          const uint4* src = reinterpret_cast<const uint4*>(a.q + (static_cast<int64_t>(b) * a.H_I + h) * D_I);
+          // two passes over the column's 256 bytes (few registers: these
+          // warps share the register budget of the epilogue)
+          float mx = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < D_I / 8; ++c) {
+            const uint4 x = valid ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const __half2 h = __floats2half2_rn(bf16_lane(w4[j], 0), bf16_lane(w4[j], 1));
-            o[j] = *reinterpret_cast<const uint32_t*>(&h);
+            for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(bf16_lane(w4[e >> 1], e & 1)));
           }
-          *pq = make_uint4(o[0], o[1], o[2], o[3]);
+          // s = 2^(7 - E) for 2^E <= mx < 2^(E + 1): mx s in [128, 256)
+          int E = static_cast<int>((__float_as_uint(mx) >> 23) & 0xFFu) - 127;
+          E = E < -119 ? -119 : E;
+          const float sc = __uint_as_float(static_cast<uint32_t>(127 + 7 - E) << 23);
+          qinv[r] = mx > 0.f ? __uint_as_float(static_cast<uint32_t>(127 - 7 + E) << 23) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D_I / 16; ++c) {  // 16 elements: one 16-byte chunk of codes
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) hw[j] = lw[j] = 0u;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {  // elements 16 c + 8 half .. + 7
+              const uint4 x = valid ? __ldg(src + 2 * c + half) : make_uint4(0, 0, 0, 0);
+              const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {  // element 8 half + e of the chunk: byte (8 half + e) % 4 of word
+                const float v = bf16_lane(w4[e >> 1], e & 1) * sc;
+                const __nv_fp8_storage_t hc = __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+                const float hv = __half2float(__half(__nv_cvt_fp8_to_halfraw(hc, __NV_E4M3)));
+                const __nv_fp8_storage_t lc = __nv_cvt_float_to_fp8(v - hv, __NV_SATFINITE, __NV_E4M3);
+                const int k = 8 * half + e;  // 0 .. 15, lowest byte first
+                hw[k >> 2] |= static_cast<uint32_t>(hc) << (8 * (k & 3));
+                lw[k >> 2] |= static_cast<uint32_t>(lc) << (8 * (k & 3));
+              }
+            }
+            st_shared_v4(qhi + sw128_offset(r, c), make_uint4(hw[0], hw[1], hw[2], hw[3]));
+            st_shared_v4(qlo + sw128_offset(r, c), make_uint4(lw[0], lw[1], lw[2], lw[3]));
+          }
         }
         fence_proxy_async_smem();
         mbar_arrive(q_conv);
       }
-      for (int h = 0; h < TPI; ++h, ++jt) {
-      const int rs = static_cast<int>(jt % C::kRawStages);
-      const uint32_t rph = static_cast<uint32_t>((jt / C::kRawStages) & 1);
-      const int bs = static_cast<int>(jt % C::kStages);
-      const uint32_t bph = static_cast<uint32_t>((jt / C::kStages) & 1);
-      if (!mbar_wait(&raw_full[rs], rph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
-      if (!mbar_wait(&empty[bs], bph ^ 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
-      const uint8_t* src = raw + rs * C::kRawBytes;
-      uint8_t* dst = stages + bs * C::kTileBytes;
-      constexpr int kChunks16 = D_I / 16;  // 16-element e4m3 chunks per row
-#pragma unroll 2
-      for (int i = ct; i < kTileKeys * kChunks16; i += C::kConvThreads) {
-        const int r = i / kChunks16, c = i % kChunks16;
-        const uint4 in = *reinterpret_cast<const uint4*>(src + r * D_I + c * 16);
-        const uint32_t w4[4] = {in.x, in.y, in.z, in.w};
-        uint32_t o[8];
+    } else {
+      int64_t jt = 0;  // key tiles converted (the stage sequence)
+      int cur_grp = -1;
+      uint32_t q_phase = 0;
+      bool ok = true;
+      for (int64_t wi = lo; wi < hi && ok; ++wi) {
+        const int grp = static_cast<int>(wi / a.tiles) * P;
+        if (grp != cur_grp) {
+          // the group's queries, staged as bf16 by TMA, become f16 in place
+          // (element by element, so the swizzled positions stay); the slot is
+          // rewritten only after the previous group's MMAs have completed
+          if (!mbar_wait(q_ready, q_phase, abort_flag, a.status, a.wait_ns)) break;
+          q_phase ^= 1;
+          cur_grp = grp;
+          constexpr int kRowChunks = 8;  // 16-byte chunks per 128-byte row
+          const int nchunks = C::kBlocks * ncols * kRowChunks;
+          for (int i = ct; i < nchunks; i += C::kConvThreads) {
+            const int bk = i / (ncols * kRowChunks), rem = i % (ncols * kRowChunks);
+            uint4* pq = reinterpret_cast<uint4*>(qs + bk * (kMaxCols * 128) + rem * 16);
+            const uint4 v = *pq;
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) e4m3x4_to_f16x4(w4[j], o[2 * j], o[2 * j + 1]);
-        // 16 f16 = two 16-byte chunks: element offsets c*16 and c*16+8. The
-        // eight threads of a row write chunks 2(c%4) and 2(c%4)+1 of block
-        // c/4; the odd block's threads write their second chunk first, so
-        // each store instruction covers eight distinct chunk positions of a
-        // row (no bank conflicts).
-        const int e0 = c * 16;
-        const uint32_t base = smem_u32(dst + (e0 >> 6) * (kTileKeys * 128));
-        const int ch = (e0 & 63) >> 3;
-        const bool second_first = D_I == 128 && ((c >> 2) & 1);
-        const uint4 v0 = make_uint4(o[0], o[1], o[2], o[3]), v1 = make_uint4(o[4], o[5], o[6], o[7]);
-        st_shared_v4(base + sw128_offset(r, second_first ? ch + 1 : ch), second_first ? v1 : v0);
-        st_shared_v4(base + sw128_offset(r, second_first ? ch : ch + 1), second_first ? v0 : v1);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&raw_empty[rs]);
-      mbar_arrive(&full[bs]);
+            for (int j = 0; j < 4; ++j) {
+              const __half2 h = __floats2half2_rn(bf16_lane(w4[j], 0), bf16_lane(w4[j], 1));
+              o[j] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            *pq = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(q_conv);
+        }
+        for (int h = 0; h < TPI; ++h, ++jt) {
+        const int rs = static_cast<int>(jt % C::kRawStages);
+        const uint32_t rph = static_cast<uint32_t>((jt / C::kRawStages) & 1);
+        const int bs = static_cast<int>(jt % C::kStages);
+        const uint32_t bph = static_cast<uint32_t>((jt / C::kStages) & 1);
+        if (!mbar_wait(&raw_full[rs], rph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+        if (!mbar_wait(&empty[bs], bph ^ 1, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+        const uint8_t* src = raw + rs * C::kRawBytes;
+        uint8_t* dst = stages + bs * C::kTileBytes;
+        constexpr int kChunks16 = D_I / 16;  // 16-element e4m3 chunks per row
+#pragma unroll 2
+        for (int i = ct; i < kTileKeys * kChunks16; i += C::kConvThreads) {
+          const int r = i / kChunks16, c = i % kChunks16;
+          const uint4 in = *reinterpret_cast<const uint4*>(src + r * D_I + c * 16);
+          const uint32_t w4[4] = {in.x, in.y, in.z, in.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) e4m3x4_to_f16x4(w4[j], o[2 * j], o[2 * j + 1]);
+          // 16 f16 = two 16-byte chunks: element offsets c*16 and c*16+8. The
+          // eight threads of a row write chunks 2(c%4) and 2(c%4)+1 of block
+          // c/4; the odd block's threads write their second chunk first, so
+          // each store instruction covers eight distinct chunk positions of a
+          // row (no bank conflicts).
+          const int e0 = c * 16;
+          const uint32_t base = smem_u32(dst + (e0 >> 6) * (kTileKeys * 128));
+          const int ch = (e0 & 63) >> 3;
+          const bool second_first = D_I == 128 && ((c >> 2) & 1);
+          const uint4 v0 = make_uint4(o[0], o[1], o[2], o[3]), v1 = make_uint4(o[4], o[5], o[6], o[7]);
+          st_shared_v4(base + sw128_offset(r, second_first ? ch + 1 : ch), second_first ? v1 : v0);
+          st_shared_v4(base + sw128_offset(r, second_first ? ch : ch + 1), second_first ? v0 : v1);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&raw_empty[rs]);
+        mbar_arrive(&full[bs]);
+        }
       }
     }
   }

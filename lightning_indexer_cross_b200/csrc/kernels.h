@@ -75,7 +75,9 @@ inline cudaError_t launch_kernel_cluster(void (*kern)(KArgs...), dim3 grid, dim3
 }
 
 struct IndexerArgs {
-  // q [B, H_I, d_I] is read through its tensor map
+  // q [B, H_I, d_I] is read through its tensor map (and directly, to split it
+  // into e4m3 parts, on the e4m3-key path with d_I = 128)
+  const __nv_bfloat16* q;
   const float* w;              // [B, H_I]
   const float* k_scale;        // e4m3 keys: per-token scale
   int64_t scale_batch_stride;  // elements between queries' scales
@@ -97,7 +99,8 @@ struct IndexerArgs {
 
 int indexer_smem_bytes(int d_I, bool fp8);
 // map: the key cache (d_I, N, batch), 128-key boxes; qmap: the queries (d_I, H_I, B)
-// with (64, HP, G) boxes, both 128-byte swizzled (e4m3 keys: unswizzled rows).
+// with (64, HP, G) boxes, both 128-byte swizzled (e4m3 keys: 128-byte swizzle
+// for d_I = 128, unswizzled rows for d_I = 64).
 cudaError_t launch_indexer(const CUtensorMap& map, const CUtensorMap& qmap, const IndexerArgs& a, int HP, int d_I,
                            bool fp8, int grid, cudaStream_t stream, bool pdl);
 
