@@ -80,6 +80,11 @@ const char* ic_status_string(ic_status_t s);
  *   scores   [B, N] fp32 output, row stride N.
  *   Supported: d_I in {64, 128}; 1 <= H_I <= 128; N >= 1; B >= 1.
  *   workspace >= ic_indexer_workspace_size() bytes (holds the status word).
+ *   Arithmetic: the products of q and the (decoded) keys, summed in fp32.
+ *   With e4m3 keys and d_I = 128 each query head is split into two e4m3
+ *   parts with a power-of-two scale, exact except that elements smaller than
+ *   2^-9 of the head's largest |q| carry an error of at most 2^-17 of it;
+ *   with e4m3 keys and d_I = 64 the queries are taken as f16 (|q| < 65504).
  * ------------------------------------------------------------------------- */
 ic_status_t ic_indexer_score(const void* q, const float* w, const void* k, const float* k_scale,
                              ic_dtype_t k_dtype, int B, int H_I, int d_I, int64_t N,
