@@ -59,6 +59,30 @@ def test_indexer_matches_oracle(cuda_dev, B, N, H_I, d_I, shared, fp8, causal):
     assert err.max() <= SCORE_TOL, f"max scaled error {err.max():.3e}"
 
 
+@pytest.mark.parametrize("shared", [False, True])
+def test_indexer_e4m3_queries_with_wide_head_ranges(cuda_dev, shared):
+    """e4m3 keys with d_I = 128 (the path that splits each query head into
+    two e4m3 parts under a power-of-two scale): head h of every query scaled
+    by 2^((h % 29) - 12), from 2^-12 up to 2^16 -- several heads beyond the
+    f16 range -- and every score against the oracle (bf16 scaling by a power
+    of two is exact, so the oracle sees the same queries)."""
+    B, N, H_I, d_I = 3, 5000, 64, 128
+    q, w, k, ks, nv = W.indexer_case(B, N, H_I, d_I, shared=shared, fp8=True, causal=True, seed=91,
+                                     device=cuda_dev)
+    f = 2.0 ** ((torch.arange(H_I, device=cuda_dev) % 29) - 12).float()
+    q = (q.float() * f[None, :, None]).to(torch.bfloat16)
+    got = _ops().indexer_score(q, w, k, ks, nv)
+    torch.cuda.synchronize()
+    ref = oracle.indexer_scores(q, w, k, ks, nv, keys_are_e4m3=True)
+    g = got.double().cpu().numpy()
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(g), fin), "masking differs (or a score overflowed)"
+    scale = np.abs(np.where(fin, ref, 0)).max(axis=1, keepdims=True)
+    scale = np.where(scale == 0, 1.0, scale)
+    err = np.abs(np.where(fin, g, 0) - np.where(fin, ref, 0)) / scale
+    assert err.max() <= SCORE_TOL, f"max scaled error {err.max():.3e}"
+
+
 # ------------------------------------------------------------------ top-k
 TOPK_CASES = [
     # B, N, k, ties, neg_inf_frac, causal
