@@ -360,15 +360,18 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
     uint32_t q_loads = 0;  // query-slot loads issued (by thread et == 0)
     uint32_t conv_phase = 0;  // kF8Mma: the converters' query splits completed
     bool got = true;
-    for (int64_t wi = lo; wi < hi && got; ++wi) {
+    // A warp that gives up on a wait (got = false) does no more work but
+    // keeps meeting every named barrier of the epilogue, so the eight warps
+    // always take the same barriers; at the next query group they all leave
+    // together.
+    for (int64_t wi = lo; wi < hi; ++wi) {
       const int grp = static_cast<int>(wi / a.tiles) * P;
       const int ng = P == 1 ? 1 : (a.groups - grp < P ? a.groups - grp : P);
       const int t = static_cast<int>(wi % a.tiles);
       if (grp != cur_grp) {
         // All MMAs of the previous item's groups finished (their accumulators
         // were drained below), so Q and the weights can be replaced.
-        if (*abort_flag) break;
-        named_bar_sync(1, kNumEpiThreads);
+        if (named_bar_or(1, kNumEpiThreads, !got || *abort_flag != 0)) break;
         // Q of each slot: one TMA load per 64-dim block of the box (d_I 64,
         // HP heads, G queries), written in the 128-byte-swizzled K-major
         // layout the MMA reads; heads past H_I and queries past B are zero
@@ -416,6 +419,10 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         }
         cur_grp = grp;
       }
+      if (!got) {
+        si += ng;  // (this warp gave up: no waits or work until the next group's barrier)
+        continue;
+      }
       for (int sub = 0; sub < ng; ++sub, ++si) {
       const int acc = static_cast<int>(si & 1);
       const uint32_t aph = static_cast<uint32_t>((si >> 1) & 1);
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(IdxCfg<D_I, FP8, PAIR>::kThreads, 1)
         if (s < a.N) scale = __ldg(a.k_scale + zb * a.scale_batch_stride + s);
       }
       got = mbar_wait(&acc_full[acc], aph, abort_flag, a.status, a.wait_ns);
-      __syncwarp();  // tcgen05.ld below is warp-collective
+      got = __all_sync(0xffffffffu, got);  // tcgen05.ld below is warp-collective: one answer per warp
       if (!got) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * 256;
