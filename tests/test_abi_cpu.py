@@ -107,6 +107,79 @@ def test_index_overlap_rejects_bad_arguments(abi):
     assert call(N=1851392 + 1) == abi.IC_ERR_UNSUPPORTED  # one bit per position in shared memory
 
 
+def test_indexer_topk_rejects_bad_arguments(abi):
+    # every case fails on the host before any launch (the pointers are host memory)
+    p, keep = _fake()
+    need = abi.ic_indexer_topk_workspace_size(2, 1000, 64, 0)
+    assert 256 < need < (1 << 20)
+    call = lambda **kw: abi._indexer_topk(*[kw.get(n, d) for n, d in [
+        ("q", p), ("w", p), ("k", p), ("ks", None), ("dt", abi.IC_BF16), ("B", 2), ("H", 64), ("d", 128),
+        ("N", 1000), ("kbs", 0), ("sbs", 0), ("nv", None), ("topk", 64), ("rpp", 0), ("idx", p), ("ws", p),
+        ("wsb", need), ("st", None)]])
+    assert call(q=None) == abi.IC_ERR_INVALID_ARG
+    assert call(idx=None) == abi.IC_ERR_INVALID_ARG
+    assert call(B=0) == abi.IC_ERR_INVALID_ARG
+    assert call(topk=0) == abi.IC_ERR_INVALID_ARG
+    assert call(ws=None) == abi.IC_ERR_INVALID_ARG
+    assert call(wsb=need - 1) == abi.IC_ERR_INVALID_ARG  # one byte short of the score and top-k scratch
+    # a pass of fewer rows needs less scratch
+    assert abi.ic_indexer_topk_workspace_size(256, 264192, 2048, 128) < \
+        abi.ic_indexer_topk_workspace_size(256, 264192, 2048, 0)
+
+
+def test_topk_noalloc_rejects_bad_arguments(abi):
+    p, keep = _fake()
+    call = lambda **kw: abi._topk_noalloc(*[kw.get(n, d) for n, d in [
+        ("s", p), ("B", 2), ("N", 1000), ("nv", None), ("k", 64), ("idx", p), ("st", None)]])
+    assert call(s=None) == abi.IC_ERR_INVALID_ARG
+    assert call(idx=None) == abi.IC_ERR_INVALID_ARG
+    assert call(B=0) == abi.IC_ERR_INVALID_ARG
+    assert call(N=0) == abi.IC_ERR_INVALID_ARG
+    assert call(k=0) == abi.IC_ERR_INVALID_ARG
+    assert call(k=16385) == abi.IC_ERR_INVALID_ARG
+    assert call(B=abi.IC_TOPK_NOALLOC_MAX_ROWS + 1) == abi.IC_ERR_UNSUPPORTED
+
+
+def test_context_parallel_steps_reject_bad_arguments(abi):
+    p, keep = _fake()
+    cand = lambda **kw: abi._cp_cand(*[kw.get(n, d) for n, d in [
+        ("s", p), ("idx", p), ("B", 2), ("Nl", 1000), ("k", 64), ("off", 0), ("cs", p), ("ci", p), ("ws", p),
+        ("wsb", 256), ("st", None)]])
+    assert cand(ws=None) == abi.IC_ERR_INVALID_ARG
+    assert cand(wsb=16) == abi.IC_ERR_INVALID_ARG
+    assert cand(s=None) == abi.IC_ERR_INVALID_ARG
+    assert cand(ci=None) == abi.IC_ERR_INVALID_ARG
+    assert cand(B=0) == abi.IC_ERR_INVALID_ARG
+    assert cand(k=0) == abi.IC_ERR_INVALID_ARG
+    assert cand(Nl=0) == abi.IC_ERR_INVALID_ARG
+    assert cand(off=-1) == abi.IC_ERR_INVALID_ARG
+    assert cand(off=(1 << 31) - 500) == abi.IC_ERR_INVALID_ARG  # global positions past int32
+    merge = lambda **kw: abi._cp_merge(*[kw.get(n, d) for n, d in [
+        ("cs", p), ("ci", p), ("seg", 128), ("G", 2), ("B", 2), ("kin", 64), ("k", 64), ("lo", 0), ("hi", 1000),
+        ("ig", p), ("il", None), ("st", None)]])
+    assert merge(cs=None) == abi.IC_ERR_INVALID_ARG
+    assert merge(ig=None) == abi.IC_ERR_INVALID_ARG
+    assert merge(G=0) == abi.IC_ERR_INVALID_ARG
+    assert merge(kin=0) == abi.IC_ERR_INVALID_ARG
+    assert merge(lo=-1) == abi.IC_ERR_INVALID_ARG
+    assert merge(lo=10, hi=5) == abi.IC_ERR_INVALID_ARG
+    assert merge(seg=100) == abi.IC_ERR_INVALID_ARG  # segments overlap: B kin = 128 per rank
+    assert merge(G=300) == abi.IC_ERR_UNSUPPORTED  # 300 x 64 candidates per row exceed shared memory
+    rows = 2 * 8
+    comb = lambda **kw: abi._cp_combine(*[kw.get(n, d) for n, d in [
+        ("po", p), ("os", rows * 512), ("pl", p), ("ls", rows), ("G", 2), ("B", 2), ("H", 8), ("sink", p),
+        ("gate", None), ("od", abi.IC_BF16), ("out", p), ("lse", None), ("st", None)]])
+    assert comb(po=None) == abi.IC_ERR_INVALID_ARG
+    assert comb(sink=None) == abi.IC_ERR_INVALID_ARG
+    assert comb(out=None) == abi.IC_ERR_INVALID_ARG
+    assert comb(G=0) == abi.IC_ERR_INVALID_ARG
+    assert comb(od=abi.IC_FP8_E4M3) == abi.IC_ERR_UNSUPPORTED
+    assert comb(po=ctypes.c_void_p(p.value + 4)) == abi.IC_ERR_INVALID_ARG  # misaligned
+    assert comb(os=rows * 512 - 4) == abi.IC_ERR_INVALID_ARG  # segments overlap
+    assert comb(os=rows * 512 + 1) == abi.IC_ERR_INVALID_ARG  # a segment off a 16-byte boundary
+    assert comb(ls=rows - 1) == abi.IC_ERR_INVALID_ARG
+
+
 def test_cache_append_rejects_bad_arguments(abi):
     # every case below must fail validation: the pointers are host memory
     p, keep = _fake()
