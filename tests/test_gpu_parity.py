@@ -83,6 +83,24 @@ def test_indexer_e4m3_queries_with_wide_head_ranges(cuda_dev, shared):
     assert err.max() <= SCORE_TOL, f"max scaled error {err.max():.3e}"
 
 
+@pytest.mark.parametrize("shared,fp8", [(True, False), (False, True)])
+def test_indexer_and_fused_call_rerun_bit_identical(cuda_dev, shared, fp8):
+    """A deterministic-rerun check against races: the same inputs twice give
+    the same score bytes, and the fused indexer -> top-k call the same index
+    sets (the order inside a row is unspecified)."""
+    B, N, H_I, d_I, k = 8, 30000, 64, 128, 1024
+    q, w, kk, ks, nv = W.indexer_case(B, N, H_I, d_I, shared=shared, fp8=fp8, causal=True, seed=97,
+                                      device=cuda_dev)
+    ops = _ops()
+    s1 = ops.indexer_score(q, w, kk, ks, nv)
+    s2 = ops.indexer_score(q, w, kk, ks, nv)
+    i1 = ops.indexer_topk(q, w, kk, k, ks, nv, rows_per_pass=8)
+    i2 = ops.indexer_topk(q, w, kk, k, ks, nv, rows_per_pass=8)
+    torch.cuda.synchronize()
+    assert torch.equal(s1.view(torch.int32), s2.view(torch.int32))
+    assert torch.equal(torch.sort(i1, dim=1).values, torch.sort(i2, dim=1).values)
+
+
 # ------------------------------------------------------------------ top-k
 TOPK_CASES = [
     # B, N, k, ties, neg_inf_frac, causal
